@@ -1,0 +1,384 @@
+// C ABI of libmoe: argument checks, workspace carving and kernel launches.
+// Every compute entry point is asynchronous on the caller's stream and
+// allocates nothing; see include/moe.h for the contract of each call.
+#include <new>
+
+#include "moe_internal.cuh"
+
+struct moe_ctx {
+  moe::Ctx c;
+};
+
+namespace moe {
+
+static size_t align_up(size_t n, size_t a) { return (n + a - 1) / a * a; }
+
+WsLayout ws_layout(const moe_layer_cfg& c, int T) {
+  WsLayout w{};
+  const size_t Tz = static_cast<size_t>(T);
+  w.n_pairs = T * c.k;
+  w.n_rows = w.n_pairs + (c.n_shared ? T : 0);
+  w.n_chunks = (w.n_pairs + kGroupChunk - 1) / kGroupChunk;
+  w.n_uniq_max = w.n_pairs < c.E ? w.n_pairs : c.E;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, 256);
+    return at;
+  };
+  w.logits = take(Tz * c.E * 4);
+  w.idx = take(Tz * c.k * 4);
+  w.gate = take(Tz * c.k * 4);
+  w.expert_count = take(static_cast<size_t>(c.E) * 4);
+  w.expert_offset = take((static_cast<size_t>(c.E) + 1) * 4);
+  w.pair_token = take(static_cast<size_t>(w.n_pairs) * 4);
+  w.pair_j = take(static_cast<size_t>(w.n_pairs) * 4);
+  w.pair_gate = take(static_cast<size_t>(w.n_pairs) * 4);
+  w.pair_slot = take(static_cast<size_t>(w.n_pairs) * 4);
+  w.pair_pos = take(static_cast<size_t>(w.n_pairs) * 4);
+  w.uniq_expert = take(static_cast<size_t>(w.n_uniq_max) * 4);
+  w.uniq_slot = take(static_cast<size_t>(w.n_uniq_max) * 4);
+  w.uniq_offset = take((static_cast<size_t>(w.n_uniq_max) + 1) * 4);
+  w.n_uniq = take(16);
+  w.chunk_hist = take(static_cast<size_t>(w.n_chunks) * c.E * 4);
+  w.tile_offset = take((static_cast<size_t>(c.E) + 2) * 4);
+  // h: fp32 rows on the decode path, fp16 rows (padded by one tile) on the prefill path
+  const size_t h32 = static_cast<size_t>(w.n_rows) * c.f * 4;
+  const size_t h16 = (static_cast<size_t>(w.n_rows) + kTileN) * c.f * 2;
+  w.h = take(h32 > h16 ? h32 : h16);
+  w.z = take(T > MOE_DECODE_MAX_T ? static_cast<size_t>(w.n_rows) * c.d * 4 : 0);
+  w.x16 = take(T > MOE_DECODE_MAX_T ? Tz * c.d * 2 : 0);
+  w.total = o;
+  return w;
+}
+
+GroupPtrs group_ptrs(const moe_layer_cfg& c, int T, void* ws) {
+  const WsLayout w = ws_layout(c, T);
+  char* b = static_cast<char*>(ws);
+  GroupPtrs g;
+  g.expert_count = reinterpret_cast<int32_t*>(b + w.expert_count);
+  g.expert_offset = reinterpret_cast<int32_t*>(b + w.expert_offset);
+  g.pair_token = reinterpret_cast<int32_t*>(b + w.pair_token);
+  g.pair_j = reinterpret_cast<int32_t*>(b + w.pair_j);
+  g.pair_gate = reinterpret_cast<float*>(b + w.pair_gate);
+  g.pair_slot = reinterpret_cast<int32_t*>(b + w.pair_slot);
+  g.pair_pos = reinterpret_cast<int32_t*>(b + w.pair_pos);
+  g.uniq_expert = reinterpret_cast<int32_t*>(b + w.uniq_expert);
+  g.uniq_slot = reinterpret_cast<int32_t*>(b + w.uniq_slot);
+  g.uniq_offset = reinterpret_cast<int32_t*>(b + w.uniq_offset);
+  g.n_uniq = reinterpret_cast<int32_t*>(b + w.n_uniq);
+  g.chunk_hist = reinterpret_cast<int32_t*>(b + w.chunk_hist);
+  g.tile_offset = reinterpret_cast<int32_t*>(b + w.tile_offset);
+  return g;
+}
+
+static moe_status check_cfg(const moe_layer_cfg* c) {
+  if (c == nullptr) return MOE_EINVAL;
+  if (c->bits != 2 && c->bits != 3) return MOE_EUNSUPPORTED;
+  if (c->block != kBlock) return MOE_EUNSUPPORTED;
+  if (c->d <= 0 || c->f <= 0 || c->E <= 0 || c->k <= 0) return MOE_EINVAL;
+  if (c->k > c->E || c->k > kMaxK) return MOE_EINVAL;
+  if (c->E > kMaxE) return MOE_EUNSUPPORTED;
+  if (c->n_shared != 0 && c->n_shared != 1) return MOE_EUNSUPPORTED;
+  if (c->d % 128 != 0 || c->f % 64 != 0 || c->d > 4096 || c->f > 4096) return MOE_EUNSUPPORTED;
+  if (!decode_geometry_ok(c->d, c->f)) return MOE_EUNSUPPORTED;
+  return MOE_OK;
+}
+
+static bool aligned(const void* p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+static moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ECUDA; }
+
+// Makes the context's device current for this host thread (kernels launch on
+// the runtime's current device).
+static bool use_device(const moe_ctx* ctx) {
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return false;
+  return cur == ctx->c.device || cudaSetDevice(ctx->c.device) == cudaSuccess;
+}
+
+static moe_expert_layout layout_of(const moe_layer_cfg& c) {
+  moe_expert_layout l;
+  const size_t gu_row = static_cast<size_t>(c.d) * c.bits / 8;
+  const size_t dn_row = static_cast<size_t>(c.f) * c.bits / 8;
+  size_t o = 0;
+  l.gu_codes = o;
+  o = align_up(o + 2 * static_cast<size_t>(c.f) * gu_row, 256);
+  l.dn_codes = o;
+  o = align_up(o + static_cast<size_t>(c.d) * dn_row, 256);
+  l.gu_scales = o;
+  o = align_up(o + 2 * static_cast<size_t>(c.f) * (c.d / kBlock) * 2, 256);
+  l.dn_scales = o;
+  o = align_up(o + static_cast<size_t>(c.d) * (c.f / kBlock) * 2, 256);
+  l.bytes = o;
+  return l;
+}
+
+static moe_status check_pool(const moe_layer_cfg& c, const uint8_t* pool, size_t stride,
+                             const uint8_t* shared) {
+  const moe_expert_layout l = layout_of(c);
+  if (pool == nullptr || !aligned(pool, 256) || stride % 256 != 0 || stride < l.bytes)
+    return MOE_EINVAL;
+  if (c.n_shared && (shared == nullptr || !aligned(shared, 256))) return MOE_EINVAL;
+  return MOE_OK;
+}
+
+static moe_status fill_grouping(const moe_layer_cfg& c, int T, void* ws, moe_grouping* out) {
+  const WsLayout w = ws_layout(c, T);
+  const GroupPtrs g = group_ptrs(c, T, ws);
+  out->T = T;
+  out->k = c.k;
+  out->E = c.E;
+  out->n_pairs = w.n_pairs;
+  out->n_rows = w.n_rows;
+  out->expert_count = g.expert_count;
+  out->expert_offset = g.expert_offset;
+  out->pair_token = g.pair_token;
+  out->pair_j = g.pair_j;
+  out->pair_gate = g.pair_gate;
+  out->pair_slot = g.pair_slot;
+  out->pair_pos = g.pair_pos;
+  out->uniq_expert = g.uniq_expert;
+  out->uniq_slot = g.uniq_slot;
+  out->uniq_offset = g.uniq_offset;
+  out->n_uniq = g.n_uniq;
+  out->internal = ws;
+  return MOE_OK;
+}
+
+static moe_status run_ffn(moe_ctx* ctx, const moe_layer_cfg* cfg, int bits, const void* x,
+                          const moe_grouping* grp, const uint8_t* pool, size_t stride,
+                          const uint8_t* shared, void* ws, size_t ws_bytes, float* z_rows,
+                          void* y, moe_stream stream) {
+  if (ctx == nullptr || grp == nullptr) return MOE_EINVAL;
+  if (!use_device(ctx)) return MOE_ECUDA;
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->bits != bits) return MOE_EINVAL;
+  const int T = grp->T;
+  if (T < 0 || grp->k != cfg->k || grp->E != cfg->E) return MOE_EINVAL;
+  if (T == 0) return MOE_OK;
+  if (ws == nullptr || grp->internal != ws) return MOE_EINVAL;
+  if (ws_bytes < ws_layout(*cfg, T).total) return MOE_ENOSPACE;
+  if ((st = check_pool(*cfg, pool, stride, shared)) != MOE_OK) return st;
+  if (x == nullptr || !aligned(x, 16)) return MOE_EINVAL;
+  const GroupPtrs g = group_ptrs(*cfg, T, ws);
+  const WsLayout w = ws_layout(*cfg, T);
+  FfnArgs a;
+  a.x = static_cast<const uint16_t*>(x);
+  a.T = T;
+  a.g = &g;
+  a.pool = pool;
+  a.stride = stride;
+  a.shared = cfg->n_shared ? shared : nullptr;
+  a.lay = layout_of(*cfg);
+  a.h = reinterpret_cast<float*>(static_cast<char*>(ws) + w.h);
+  a.y = y;
+  a.status = ctx->c.d_status;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (z_rows == nullptr) {
+    if (T > MOE_DECODE_MAX_T || y == nullptr || !aligned(y, 16)) return MOE_EINVAL;
+    return from_cuda(launch_ffn_decode(ctx->c, *cfg, a, s));
+  }
+  if (!aligned(z_rows, 16)) return MOE_EINVAL;
+  const cudaError_t e = launch_ffn_prefill(ctx->c, *cfg, a, ws, z_rows, s);
+  if (e == cudaErrorNotSupported) return MOE_EUNSUPPORTED;
+  return from_cuda(e);
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_ctx_create(int device, moe_ctx** out) {
+  if (out == nullptr || device < 0) return MOE_EINVAL;
+  *out = nullptr;
+  moe_ctx* ctx = new (std::nothrow) moe_ctx;
+  if (ctx == nullptr) return MOE_EINVAL;
+  ctx->c.device = device;
+  if (cudaSetDevice(device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&ctx->c.num_sms, cudaDevAttrMultiProcessorCount, ctx->c.device) !=
+          cudaSuccess ||
+      cudaMalloc(&ctx->c.d_status, 16) != cudaSuccess) {
+    delete ctx;
+    return MOE_ECUDA;
+  }
+  if (cudaMemset(ctx->c.d_status, 0, 16) != cudaSuccess || router_init(ctx->c) != cudaSuccess ||
+      decode_init(ctx->c) != cudaSuccess || prefill_init(ctx->c) != cudaSuccess) {
+    cudaFree(ctx->c.d_status);
+    delete ctx;
+    return MOE_ECUDA;
+  }
+  *out = ctx;
+  return MOE_OK;
+}
+
+void moe_ctx_destroy(moe_ctx* ctx) {
+  if (ctx == nullptr) return;
+  use_device(ctx);
+  cudaFree(ctx->c.d_status);
+  delete ctx;
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_EINVAL: return "invalid argument";
+    case MOE_EUNSUPPORTED: return "unsupported configuration";
+    case MOE_ECUDA: return "CUDA error";
+    case MOE_ETIMEOUT: return "device wait timed out";
+    case MOE_EDEVICE: return "kernel saw an out-of-range expert or slot index";
+    case MOE_ENOSPACE: return "workspace too small";
+    default: return "unknown status";
+  }
+}
+
+moe_status moe_check_device_status(moe_ctx* ctx, moe_stream stream) {
+  if (ctx == nullptr) return MOE_EINVAL;
+  if (!use_device(ctx)) return MOE_ECUDA;
+  int h[4] = {0, 0, 0, 0};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(h, ctx->c.d_status, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return MOE_ECUDA;
+  if (h[0] == 0) return MOE_OK;
+  if (cudaMemsetAsync(ctx->c.d_status, 0, 16, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+    return MOE_ECUDA;
+  return h[0] == kDevTimeout ? MOE_ETIMEOUT : MOE_EDEVICE;
+}
+
+moe_status moe_expert_layout_get(const moe_layer_cfg* cfg, moe_expert_layout* out) {
+  if (out == nullptr) return MOE_EINVAL;
+  const moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  *out = layout_of(*cfg);
+  return MOE_OK;
+}
+
+size_t moe_workspace_bytes(const moe_layer_cfg* cfg, int T) {
+  if (check_cfg(cfg) != MOE_OK || T < 0) return 0;
+  return ws_layout(*cfg, T).total;
+}
+
+moe_status moe_router_topk(moe_ctx* ctx, const moe_layer_cfg* cfg, const void* x,
+                           const float* w_router, const float* logit_bias, int T, float* logits,
+                           int32_t* idx, float* gate, moe_stream stream) {
+  if (ctx == nullptr) return MOE_EINVAL;
+  if (!use_device(ctx)) return MOE_ECUDA;
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0) return MOE_EINVAL;
+  if (T == 0) return MOE_OK;
+  if (x == nullptr || w_router == nullptr || logits == nullptr || idx == nullptr || gate == nullptr)
+    return MOE_EINVAL;
+  if (!aligned(x, 16) || !aligned(w_router, 16)) return MOE_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_router_logits(ctx->c, *cfg, static_cast<const uint16_t*>(x), w_router,
+                                       logit_bias, T, logits, s);
+  if (e != cudaSuccess) return MOE_ECUDA;
+  return from_cuda(launch_topk(ctx->c, *cfg, logits, T, idx, gate, s));
+}
+
+moe_status moe_topk(moe_ctx* ctx, const moe_layer_cfg* cfg, const float* logits, int T,
+                    int32_t* idx, float* gate, moe_stream stream) {
+  if (ctx == nullptr) return MOE_EINVAL;
+  if (!use_device(ctx)) return MOE_ECUDA;
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0) return MOE_EINVAL;
+  if (T == 0) return MOE_OK;
+  if (logits == nullptr || idx == nullptr || gate == nullptr) return MOE_EINVAL;
+  return from_cuda(launch_topk(ctx->c, *cfg, logits, T, idx, gate, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_group_tokens(moe_ctx* ctx, const moe_layer_cfg* cfg, const int32_t* idx,
+                            const float* gate, int T, const int32_t* slot_of, int n_slots,
+                            void* ws, size_t ws_bytes, moe_grouping* out, moe_stream stream) {
+  if (ctx == nullptr || out == nullptr) return MOE_EINVAL;
+  if (!use_device(ctx)) return MOE_ECUDA;
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0 || n_slots <= 0) return MOE_EINVAL;
+  if (ws == nullptr || !aligned(ws, 256)) return MOE_EINVAL;
+  if (ws_bytes < ws_layout(*cfg, T).total) return MOE_ENOSPACE;
+  fill_grouping(*cfg, T, ws, out);
+  if (T == 0) return MOE_OK;
+  if (idx == nullptr || gate == nullptr || slot_of == nullptr) return MOE_EINVAL;
+  const GroupPtrs g = group_ptrs(*cfg, T, ws);
+  return from_cuda(launch_group(ctx->c, *cfg, idx, gate, T, slot_of, n_slots, g,
+                                static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_expert_ffn_q2(moe_ctx* ctx, const moe_layer_cfg* cfg, const void* x,
+                             const moe_grouping* grouping, const uint8_t* slot_pool,
+                             size_t slot_stride, const uint8_t* shared_expert, void* ws,
+                             size_t ws_bytes, float* z_rows, void* y, moe_stream stream) {
+  return run_ffn(ctx, cfg, 2, x, grouping, slot_pool, slot_stride, shared_expert, ws, ws_bytes,
+                 z_rows, y, stream);
+}
+
+moe_status moe_expert_ffn_q3(moe_ctx* ctx, const moe_layer_cfg* cfg, const void* x,
+                             const moe_grouping* grouping, const uint8_t* slot_pool,
+                             size_t slot_stride, const uint8_t* shared_expert, void* ws,
+                             size_t ws_bytes, float* z_rows, void* y, moe_stream stream) {
+  return run_ffn(ctx, cfg, 3, x, grouping, slot_pool, slot_stride, shared_expert, ws, ws_bytes,
+                 z_rows, y, stream);
+}
+
+moe_status moe_combine(moe_ctx* ctx, const moe_layer_cfg* cfg, const moe_grouping* grouping,
+                       const float* z_rows, const void* x, int T, void* y, moe_stream stream) {
+  if (ctx == nullptr || grouping == nullptr) return MOE_EINVAL;
+  if (!use_device(ctx)) return MOE_ECUDA;
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0 || grouping->T != T || grouping->k != cfg->k) return MOE_EINVAL;
+  if (T == 0) return MOE_OK;
+  if (z_rows == nullptr || y == nullptr || !aligned(z_rows, 16) || !aligned(y, 16)) return MOE_EINVAL;
+  if (cfg->residual && (x == nullptr || !aligned(x, 16))) return MOE_EINVAL;
+  return from_cuda(launch_combine(ctx->c, *cfg, grouping->pair_pos, grouping->n_pairs, z_rows,
+                                  static_cast<const uint16_t*>(x), T, y,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_layer_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, const void* x, int T,
+                             const float* w_router, const float* logit_bias,
+                             const int32_t* slot_of, int n_slots, const uint8_t* slot_pool,
+                             size_t slot_stride, const uint8_t* shared_expert, void* ws,
+                             size_t ws_bytes, void* y, moe_stream stream) {
+  if (ctx == nullptr) return MOE_EINVAL;
+  if (!use_device(ctx)) return MOE_ECUDA;
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0 || n_slots <= 0) return MOE_EINVAL;
+  if (T == 0) return MOE_OK;
+  if (x == nullptr || w_router == nullptr || slot_of == nullptr || y == nullptr) return MOE_EINVAL;
+  if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(y, 16)) return MOE_EINVAL;
+  if (ws == nullptr || !aligned(ws, 256)) return MOE_EINVAL;
+  const WsLayout w = ws_layout(*cfg, T);
+  if (ws_bytes < w.total) return MOE_ENOSPACE;
+  if ((st = check_pool(*cfg, slot_pool, slot_stride, shared_expert)) != MOE_OK) return st;
+  char* b = static_cast<char*>(ws);
+  float* logits = reinterpret_cast<float*>(b + w.logits);
+  int32_t* idx = reinterpret_cast<int32_t*>(b + w.idx);
+  float* gate = reinterpret_cast<float*>(b + w.gate);
+  if ((st = moe_router_topk(ctx, cfg, x, w_router, logit_bias, T, logits, idx, gate, stream)) != MOE_OK)
+    return st;
+  moe_grouping g;
+  if ((st = moe_group_tokens(ctx, cfg, idx, gate, T, slot_of, n_slots, ws, ws_bytes, &g, stream)) !=
+      MOE_OK)
+    return st;
+  if (T <= MOE_DECODE_MAX_T)
+    return run_ffn(ctx, cfg, cfg->bits, x, &g, slot_pool, slot_stride, shared_expert, ws, ws_bytes,
+                   nullptr, y, stream);
+  float* z = reinterpret_cast<float*>(b + w.z);
+  if ((st = run_ffn(ctx, cfg, cfg->bits, x, &g, slot_pool, slot_stride, shared_expert, ws, ws_bytes, z,
+                    nullptr, stream)) != MOE_OK)
+    return st;
+  return moe_combine(ctx, cfg, &g, z, x, T, y, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,127 @@
+// Internal declarations shared by the libmoe translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- constants
+
+constexpr int kBlock = 32;            // weights per fp16 scale
+constexpr int kMaxE = 1024;           // experts per layer
+constexpr int kMaxK = 32;             // experts per token
+constexpr int kGroupChunk = 512;      // pairs per chunk in the multi-CTA grouping
+constexpr int kTileN = 128;           // tokens per tile of the prefill grouped GEMM
+
+// Device status word codes (word 0 holds the first error seen).
+constexpr int kDevBadExpert = 1;
+constexpr int kDevBadSlot = 2;
+constexpr int kDevTimeout = 3;
+
+struct Ctx {
+  int device = 0;
+  int num_sms = 0;
+  int* d_status = nullptr;  // [4] ints: code, detail, spare, spare
+};
+
+// ---------------------------------------------------------------- workspace
+
+struct WsLayout {
+  size_t logits, idx, gate;
+  size_t expert_count, expert_offset, pair_token, pair_j, pair_gate, pair_slot, pair_pos;
+  size_t uniq_expert, uniq_slot, uniq_offset, n_uniq;
+  size_t chunk_hist, tile_offset;
+  size_t h, z, x16;
+  size_t total;
+  int n_pairs, n_rows, n_chunks, n_uniq_max;
+};
+
+WsLayout ws_layout(const moe_layer_cfg& c, int T);
+
+// ---------------------------------------------------------------- device helpers
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ void report(int* status, int code, int detail) {
+  if (status != nullptr) {
+    if (atomicCAS(status, 0, code) == 0) status[1] = detail;
+  }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Sum over aligned groups of `width` lanes (width a power of two <= 32).
+__device__ __forceinline__ float group_sum(float v, int width) {
+  for (int o = width >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Loads that bypass L1 (data written by an earlier kernel of the same stream).
+__device__ __forceinline__ int ld_cg(const int* p) { return __ldcg(p); }
+__device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
+
+// ---------------------------------------------------------------- launchers (host)
+
+// router.cu
+cudaError_t launch_router_logits(const Ctx& ctx, const moe_layer_cfg& c, const uint16_t* x,
+                                 const float* wr, const float* bias, int T, float* logits,
+                                 cudaStream_t s);
+cudaError_t launch_topk(const Ctx& ctx, const moe_layer_cfg& c, const float* logits, int T,
+                        int32_t* idx, float* gate, cudaStream_t s);
+
+// group.cu
+struct GroupPtrs {
+  int32_t *expert_count, *expert_offset, *pair_token, *pair_j, *pair_slot, *pair_pos;
+  float* pair_gate;
+  int32_t *uniq_expert, *uniq_slot, *uniq_offset, *n_uniq;
+  int32_t *chunk_hist, *tile_offset;
+};
+GroupPtrs group_ptrs(const moe_layer_cfg& c, int T, void* ws);
+cudaError_t launch_group(const Ctx& ctx, const moe_layer_cfg& c, const int32_t* idx,
+                         const float* gate, int T, const int32_t* slot_of, int n_slots,
+                         const GroupPtrs& g, cudaStream_t s);
+
+// ffn_decode.cu
+struct FfnArgs {
+  const uint16_t* x;        // [T, d] bf16
+  int T;
+  const GroupPtrs* g;
+  const uint8_t* pool;
+  size_t stride;
+  const uint8_t* shared;    // record or null
+  moe_expert_layout lay;
+  float* h;                 // decode: fp32 [n_rows, f]
+  void* y;
+  int* status;
+};
+cudaError_t launch_ffn_decode(const Ctx& ctx, const moe_layer_cfg& c, const FfnArgs& a,
+                              cudaStream_t s);
+bool decode_geometry_ok(int d, int f);
+
+// ffn_prefill.cu
+cudaError_t launch_ffn_prefill(const Ctx& ctx, const moe_layer_cfg& c, const FfnArgs& a,
+                               void* ws, float* z_rows, cudaStream_t s);
+cudaError_t prefill_init(const Ctx& ctx);
+
+// combine.cu
+cudaError_t launch_combine(const Ctx& ctx, const moe_layer_cfg& c, const int32_t* pair_pos,
+                           int n_pairs, const float* z_rows, const uint16_t* x, int T, void* y,
+                           cudaStream_t s);
+
+// kernel attribute set-up, once per context
+cudaError_t decode_init(const Ctx& ctx);
+cudaError_t router_init(const Ctx& ctx);
+
+}  // namespace moe

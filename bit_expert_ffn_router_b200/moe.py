@@ -1,0 +1,226 @@
+"""ctypes binding of libmoe (include/moe.h): argument marshalling only.
+
+Every step of the MoE FFN runs inside libmoe's CUDA kernels; this module turns
+torch tensors into device pointers and the current torch stream into a
+cudaStream_t. If libmoe.so is missing, loading fails with an error: there is
+no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "lib", "libmoe.so")
+
+OK, EINVAL, EUNSUPPORTED, ECUDA, ETIMEOUT, EDEVICE, ENOSPACE = range(7)
+DECODE_MAX_T = 8
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in
+                ("d", "f", "E", "k", "n_shared", "bits", "block", "renorm", "out_fp32", "residual")]
+
+
+class _Layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in ("gu_codes", "dn_codes", "gu_scales", "dn_scales", "bytes")]
+
+
+class Grouping(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int), ("k", ctypes.c_int), ("E", ctypes.c_int),
+                ("n_pairs", ctypes.c_int), ("n_rows", ctypes.c_int)] + [
+        (n, ctypes.c_void_p) for n in
+        ("expert_count", "expert_offset", "pair_token", "pair_j", "pair_gate", "pair_slot", "pair_pos",
+         "uniq_expert", "uniq_slot", "uniq_offset", "n_uniq", "internal")]
+
+
+@dataclasses.dataclass(frozen=True)
+class LayerCfg:
+    d: int
+    f: int
+    E: int
+    k: int
+    n_shared: int = 1
+    bits: int = 2
+    block: int = 32
+    renorm: int = 1
+    out_fp32: int = 1
+    residual: int = 0
+
+    def c(self) -> _Cfg:
+        return _Cfg(*(getattr(self, f.name) for f in dataclasses.fields(self)))
+
+    def replace(self, **kw) -> "LayerCfg":
+        return dataclasses.replace(self, **kw)
+
+
+# Named shapes: the tiny parity layer and the full Qwen3.8-Flash-Next-shaped layer.
+TINY = LayerCfg(d=256, f=128, E=16, k=2)
+FULL = LayerCfg(d=2048, f=768, E=512, k=10)
+
+_P, _I, _Z, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+_SIGS = {
+    "moe_ctx_create": (_I, [_I, ctypes.POINTER(ctypes.c_void_p)]),
+    "moe_ctx_destroy": (None, [_P]),
+    "moe_status_string": (ctypes.c_char_p, [_I]),
+    "moe_check_device_status": (_I, [_P, _S]),
+    "moe_expert_layout_get": (_I, [ctypes.POINTER(_Cfg), ctypes.POINTER(_Layout)]),
+    "moe_workspace_bytes": (_Z, [ctypes.POINTER(_Cfg), _I]),
+    "moe_router_topk": (_I, [_P, ctypes.POINTER(_Cfg), _P, _P, _P, _I, _P, _P, _P, _S]),
+    "moe_topk": (_I, [_P, ctypes.POINTER(_Cfg), _P, _I, _P, _P, _S]),
+    "moe_group_tokens": (_I, [_P, ctypes.POINTER(_Cfg), _P, _P, _I, _P, _I, _P, _Z,
+                              ctypes.POINTER(Grouping), _S]),
+    "moe_expert_ffn_q2": (_I, [_P, ctypes.POINTER(_Cfg), _P, ctypes.POINTER(Grouping), _P, _Z, _P, _P, _Z,
+                               _P, _P, _S]),
+    "moe_expert_ffn_q3": (_I, [_P, ctypes.POINTER(_Cfg), _P, ctypes.POINTER(Grouping), _P, _Z, _P, _P, _Z,
+                               _P, _P, _S]),
+    "moe_combine": (_I, [_P, ctypes.POINTER(_Cfg), ctypes.POINTER(Grouping), _P, _P, _I, _P, _S]),
+    "moe_layer_forward": (_I, [_P, ctypes.POINTER(_Cfg), _P, _I, _P, _P, _P, _I, _P, _Z, _P, _P, _Z, _P,
+                               _S]),
+}
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Opens libmoe.so (built in-tree by bit_expert_ffn_router_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise FileNotFoundError(f"{path} is missing: build it with `python -m bit_expert_ffn_router_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_string(s: int) -> str:
+    return load_library().moe_status_string(s).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != OK:
+        raise MoeError(status, what)
+
+
+def expert_layout(cfg: LayerCfg) -> dict:
+    lay = _Layout()
+    _check(load_library().moe_expert_layout_get(ctypes.byref(cfg.c()), ctypes.byref(lay)), "moe_expert_layout_get")
+    return {n: getattr(lay, n) for n, _ in _Layout._fields_}
+
+
+def workspace_bytes(cfg: LayerCfg, T: int) -> int:
+    return int(load_library().moe_workspace_bytes(ctypes.byref(cfg.c()), T))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class Context:
+    """One libmoe context (device status word + SM count) on a CUDA device."""
+
+    def __init__(self, device: int = 0):
+        self.lib = load_library()
+        h = ctypes.c_void_p()
+        _check(self.lib.moe_ctx_create(device, ctypes.byref(h)), "moe_ctx_create")
+        self.h = h
+        self.device = device
+
+    def close(self):
+        if self.h:
+            self.lib.moe_ctx_destroy(self.h)
+            self.h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- raw entry points (status codes returned, not raised) --------------------
+    def router_topk_status(self, cfg, x, w_router, bias, T, logits, idx, gate, stream=None):
+        return self.lib.moe_router_topk(self.h, ctypes.byref(cfg.c()), _ptr(x), _ptr(w_router), _ptr(bias), T,
+                                        _ptr(logits), _ptr(idx), _ptr(gate), _stream(stream))
+
+    def layer_forward_status(self, cfg, x, T, w_router, bias, slot_of, n_slots, pool, stride, shared, ws, y,
+                             stream=None):
+        return self.lib.moe_layer_forward(self.h, ctypes.byref(cfg.c()), _ptr(x), T, _ptr(w_router), _ptr(bias),
+                                          _ptr(slot_of), n_slots, _ptr(pool), stride, _ptr(shared), _ptr(ws),
+                                          0 if ws is None else ws.numel() * ws.element_size(), _ptr(y),
+                                          _stream(stream))
+
+    # -- checked wrappers ---------------------------------------------------------
+    def router_topk(self, cfg, x, w_router, bias, T, logits, idx, gate, stream=None):
+        _check(self.router_topk_status(cfg, x, w_router, bias, T, logits, idx, gate, stream), "moe_router_topk")
+
+    def topk(self, cfg, logits, T, idx, gate, stream=None):
+        _check(self.lib.moe_topk(self.h, ctypes.byref(cfg.c()), _ptr(logits), T, _ptr(idx), _ptr(gate),
+                                 _stream(stream)), "moe_topk")
+
+    def group_tokens(self, cfg, idx, gate, T, slot_of, n_slots, ws, stream=None) -> Grouping:
+        g = Grouping()
+        _check(self.lib.moe_group_tokens(self.h, ctypes.byref(cfg.c()), _ptr(idx), _ptr(gate), T, _ptr(slot_of),
+                                         n_slots, _ptr(ws), ws.numel() * ws.element_size(), ctypes.byref(g),
+                                         _stream(stream)), "moe_group_tokens")
+        return g
+
+    def expert_ffn(self, cfg, x, grouping, pool, stride, shared, ws, z_rows=None, y=None, stream=None):
+        fn = self.lib.moe_expert_ffn_q2 if cfg.bits == 2 else self.lib.moe_expert_ffn_q3
+        _check(fn(self.h, ctypes.byref(cfg.c()), _ptr(x), ctypes.byref(grouping), _ptr(pool), stride, _ptr(shared),
+                  _ptr(ws), ws.numel() * ws.element_size(), _ptr(z_rows), _ptr(y), _stream(stream)),
+               f"moe_expert_ffn_q{cfg.bits}")
+
+    def combine(self, cfg, grouping, z_rows, x, T, y, stream=None):
+        _check(self.lib.moe_combine(self.h, ctypes.byref(cfg.c()), ctypes.byref(grouping), _ptr(z_rows), _ptr(x),
+                                    T, _ptr(y), _stream(stream)), "moe_combine")
+
+    def layer_forward(self, cfg, x, T, w_router, bias, slot_of, n_slots, pool, stride, shared, ws, y,
+                      stream=None):
+        _check(self.layer_forward_status(cfg, x, T, w_router, bias, slot_of, n_slots, pool, stride, shared, ws, y,
+                                         stream), "moe_layer_forward")
+
+    def check_device_status(self, stream=None) -> int:
+        return self.lib.moe_check_device_status(self.h, _stream(stream))
+
+
+# ------------------------------------------------------------------ buffers
+
+def workspace(cfg: LayerCfg, T: int, device="cuda"):
+    import torch
+    n = workspace_bytes(cfg, T)
+    if n == 0:
+        raise MoeError(EINVAL, "moe_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def place_records(cfg: LayerCfg, sections: list, device="cuda", stride: int | None = None):
+    """Packs per-expert section arrays (gu_codes, dn_codes, gu_scales, dn_scales)
+    into one uint8 pool tensor [n, stride] at libmoe's record offsets."""
+    import numpy as np
+    import torch
+    lay = expert_layout(cfg)
+    stride = stride or lay["bytes"]
+    host = np.zeros((len(sections), stride), dtype=np.uint8)
+    for i, sec in enumerate(sections):
+        for name in ("gu_codes", "dn_codes", "gu_scales", "dn_scales"):
+            raw = np.ascontiguousarray(sec[name]).view(np.uint8).reshape(-1)
+            host[i, lay[name]:lay[name] + raw.size] = raw
+    return torch.from_numpy(host).to(device), stride

@@ -1,0 +1,214 @@
+/*
+ * moe.h -- C ABI of libmoe: the per-layer sparse Mixture-of-Experts FFN step
+ * of a Qwen3.8-Flash-Next-shaped model on one NVIDIA B200 (sm_100a).
+ *
+ * The step (per layer, per token t):
+ *   1. router logits  l[t,e] = sum_i x[t,i] * W_r[e,i]  (+ an optional bias)
+ *   2. top-k          the k largest logits, ties to the lower expert index,
+ *                     gates = softmax over the k chosen logits
+ *   3. grouping       the T*k (token, j) pairs stably sorted by expert, each
+ *                     expert mapped to its slot in an expert pool
+ *   4. experts        h = silu(W_g x) * (W_u x), z = W_d h on 2- or 3-bit
+ *                     block-quantised weights, dequantised inside the kernels
+ *   5. combine        y[t] = sum_j gate[t,j] * z_(t,j) + z_shared[t]
+ *
+ * The pages this follows describe the model as 48 layers x 512 experts, of
+ * which a token uses 10 plus one always-on shared expert (Strataとは,
+ * news.blueqat.app/post/3262, first section; geekoyaji.com
+ * "freetoken-vs-strata-moe-offload", section 共通の仕組み), expert weights at 2
+ * to 3 bits (news.blueqat.app, section 量子化の種類とサイズ), a router and shared
+ * expert that run on the GPU for every token (news.blueqat.app, section
+ * GPU・CPU・RAM・SSDの分担), decode passes that verify up to 3 drafted tokens
+ * at once, so T <= 4 (vramglass.com, section その3), and prefill chunks of up to
+ * 8,192 tokens (news.blueqat.app, section GPU・CPU・RAM・SSDの分担). The pages
+ * give no formulas and no bit layout; both are defined here.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller. The
+ *     library allocates no device memory on any compute call; scratch comes
+ *     from a caller workspace of moe_workspace_bytes() bytes.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream). Errors detected on the host are returned at once;
+ *     errors detected by a kernel are recorded in the context's device status
+ *     word and returned by moe_check_device_status().
+ *   - No exception or abort crosses the ABI. A context may be used by one host
+ *     thread at a time; it belongs to the device named at its creation, and
+ *     every call made with it launches there.
+ *
+ * Expert record (one routed or shared expert, `moe_expert_layout`):
+ *   gu_codes  [2f rows, d cols] packed codes; row 2c is gate channel c,
+ *             row 2c+1 is up channel c
+ *   dn_codes  [d rows, f cols] packed codes
+ *   gu_scales [2f rows, d/32] fp16 (raw bits), one scale per 32 weights
+ *   dn_scales [d rows, f/32] fp16
+ *   Each section starts on a 256-byte boundary. A weight is
+ *   w = scale * (q - 2^(bits-1)), q in [0, 2^bits). Blocks of 32 run along the
+ *   reduction (column) axis. 2-bit rows: code c in byte c/4 at bits 2*(c%4).
+ *   3-bit rows: that 2-bit plane for the low bits (cols/4 bytes) followed by a
+ *   1-bit plane (cols/8 bytes) with the high bit of code c at bit c%8 of byte
+ *   c/8. The pages name Q2_0 and the IQ2/IQ3 formats but print none of their
+ *   bits; this format costs 2.5 / 3.5 bits per weight, the IQ2_XS / IQ3_S rows
+ *   of the pages' quantisation table.
+ *
+ * Expert pool: expert e of a layer lives at slot_pool + slot_of[e]*slot_stride
+ * (the slot table stands for the pages' hot-expert cache; on one B200 every
+ * expert is in HBM and the table is only an indirection).
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef int moe_status;
+#define MOE_OK            0
+#define MOE_EINVAL        1  /* bad shape, NULL pointer, misalignment, k > E, k > 32 */
+#define MOE_EUNSUPPORTED  2  /* bits not in {2,3}, block != 32, shape outside the kernels' range */
+#define MOE_ECUDA         3  /* a CUDA runtime call or kernel launch failed */
+#define MOE_ETIMEOUT      4  /* a bounded device-side wait gave up (read by moe_check_device_status) */
+#define MOE_EDEVICE       5  /* a kernel found a bad index (expert >= E, slot >= n_slots) */
+#define MOE_ENOSPACE      6  /* workspace smaller than moe_workspace_bytes() */
+
+typedef struct moe_ctx moe_ctx;
+typedef void* moe_stream; /* cudaStream_t */
+
+/* Largest T that takes the decode path (weight streaming, fused combine). */
+#define MOE_DECODE_MAX_T 8
+
+typedef struct {
+  int d;         /* hidden size (multiple of 128) */
+  int f;         /* expert intermediate size (multiple of 64) */
+  int E;         /* routed experts per layer, 1..1024 */
+  int k;         /* experts per token, 1..min(E, 32) */
+  int n_shared;  /* 0 or 1 shared expert */
+  int bits;      /* 2 or 3 */
+  int block;     /* weights per scale; must be 32 */
+  int renorm;    /* 1: gates = softmax over the k chosen logits; 0: full softmax read at them */
+  int out_fp32;  /* 1: y is fp32; 0: y is bf16 (round to nearest even) */
+  int residual;  /* 1: y = x + moe(x) */
+} moe_layer_cfg;
+
+typedef struct {
+  size_t gu_codes, dn_codes, gu_scales, dn_scales; /* byte offsets inside a record */
+  size_t bytes;                                    /* record size, a multiple of 256 */
+} moe_expert_layout;
+
+/* Token grouping: device pointers into the caller's workspace, filled by
+ * moe_group_tokens. Sorted order is (expert, token, j); the shared expert's
+ * rows follow the routed pairs, token t at row n_pairs + t. */
+typedef struct {
+  int T, k, E;
+  int n_pairs;            /* T*k */
+  int n_rows;             /* n_pairs + T*n_shared */
+  int32_t* expert_count;  /* [E]    pairs per expert */
+  int32_t* expert_offset; /* [E+1]  exclusive prefix sum of expert_count */
+  int32_t* pair_token;    /* [n_pairs] token of each sorted pair */
+  int32_t* pair_j;        /* [n_pairs] rank j of the pair in its token's top-k */
+  float*   pair_gate;     /* [n_pairs] gate of the pair */
+  int32_t* pair_slot;     /* [n_pairs] pool slot of the pair's expert */
+  int32_t* pair_pos;      /* [T*k]  sorted position of pair (t, j) at t*k + j */
+  int32_t* uniq_expert;   /* [min(E, n_pairs)] experts with >= 1 pair, ascending */
+  int32_t* uniq_slot;     /* [min(E, n_pairs)] their pool slots */
+  int32_t* uniq_offset;   /* [min(E, n_pairs) + 1] first sorted pair of each */
+  int32_t* n_uniq;        /* [1] number of such experts */
+  void*    internal;      /* library-private scratch (tile lists, histograms) */
+} moe_grouping;
+
+/* ---- context ------------------------------------------------------------ */
+
+/* Creates a context on CUDA device `device`: queries the SM count, allocates
+ * the 16-byte device status word (the only device allocation the library
+ * makes) and sets kernel attributes. Every later call with this context
+ * launches on that device. Call outside stream capture. */
+MOE_API moe_status moe_ctx_create(int device, moe_ctx** out);
+MOE_API void moe_ctx_destroy(moe_ctx* ctx);
+MOE_API const char* moe_status_string(moe_status s);
+
+/* Synchronises `stream`, reads and clears the device status word. Returns
+ * MOE_OK, MOE_EDEVICE (bad expert or slot index seen by a kernel) or
+ * MOE_ETIMEOUT (a bounded wait ran out). */
+MOE_API moe_status moe_check_device_status(moe_ctx* ctx, moe_stream stream);
+
+/* ---- sizes -------------------------------------------------------------- */
+
+/* Layout of one expert record for cfg (see the header comment). */
+MOE_API moe_status moe_expert_layout_get(const moe_layer_cfg* cfg, moe_expert_layout* out);
+
+/* Bytes of workspace every call below needs for T tokens (0 if cfg is invalid). */
+MOE_API size_t moe_workspace_bytes(const moe_layer_cfg* cfg, int T);
+
+/* ---- steps -------------------------------------------------------------- */
+
+/* Router + top-k. x: [T, d] bf16 row-major (16-byte aligned); w_router: [E, d]
+ * fp32 row-major; logit_bias: NULL or [T, E] fp32 added to the logits;
+ * logits (out): [T, E] fp32; idx (out): [T, k] int32 in descending-logit
+ * order; gate (out): [T, k] fp32. The router runs for every token on the GPU
+ * (news.blueqat.app/post/3262, section GPU・CPU・RAM・SSDの分担). T = 0 is a
+ * no-op. */
+MOE_API moe_status moe_router_topk(moe_ctx* ctx, const moe_layer_cfg* cfg, const void* x,
+                           const float* w_router, const float* logit_bias, int T,
+                           float* logits, int32_t* idx, float* gate, moe_stream stream);
+
+/* Top-k and gates from given fp32 logits [T, E] (the selection step alone). */
+MOE_API moe_status moe_topk(moe_ctx* ctx, const moe_layer_cfg* cfg, const float* logits, int T,
+                    int32_t* idx, float* gate, moe_stream stream);
+
+/* Stable counting sort of the T*k pairs by expert, without atomics, and the
+ * slot lookup slot = slot_of[e]. idx, gate: [T, k] from moe_topk; slot_of:
+ * [E] int32 (this layer's slice of the slot table); n_slots bounds the slots
+ * (a slot >= n_slots is reported as MOE_EDEVICE). Fills *out with views into
+ * ws. The slot table stands for the pages' hot-expert cache (vramglass.com,
+ * section その1：よく使うエキスパートを選んでGPUに置く). */
+MOE_API moe_status moe_group_tokens(moe_ctx* ctx, const moe_layer_cfg* cfg, const int32_t* idx,
+                            const float* gate, int T, const int32_t* slot_of, int n_slots,
+                            void* ws, size_t ws_bytes, moe_grouping* out, moe_stream stream);
+
+/* Expert FFN over 2-bit (q2) or 3-bit (q3) records: for every sorted pair and
+ * every shared-expert row, h = silu(W_g x) * (W_u x) and z = W_d h.
+ * slot_pool: base of the pool (256-byte aligned), slot_stride: bytes between
+ * slots (a multiple of 256, >= the record size); shared_expert: one record or
+ * NULL when cfg->n_shared == 0; ws: the workspace the grouping came from.
+ *   z_rows == NULL: decode path (T <= MOE_DECODE_MAX_T). The combine is fused:
+ *       y [T, d] (fp32 or bf16 per cfg->out_fp32) is written directly.
+ *   z_rows != NULL: z_rows [n_rows, d] fp32 receives gate * z for each sorted
+ *       pair and z for each shared row; y is not touched (pass NULL) and
+ *       moe_combine finishes the step. Any T. */
+MOE_API moe_status moe_expert_ffn_q2(moe_ctx* ctx, const moe_layer_cfg* cfg, const void* x,
+                             const moe_grouping* grouping, const uint8_t* slot_pool,
+                             size_t slot_stride, const uint8_t* shared_expert, void* ws,
+                             size_t ws_bytes, float* z_rows, void* y, moe_stream stream);
+MOE_API moe_status moe_expert_ffn_q3(moe_ctx* ctx, const moe_layer_cfg* cfg, const void* x,
+                             const moe_grouping* grouping, const uint8_t* slot_pool,
+                             size_t slot_stride, const uint8_t* shared_expert, void* ws,
+                             size_t ws_bytes, float* z_rows, void* y, moe_stream stream);
+
+/* y[t] = sum_j z_rows[pair_pos[t,j]] (j ascending) + z_rows[n_pairs + t]
+ * (+ x[t] when cfg->residual), written as fp32 or bf16. x may be NULL unless
+ * residual. This is the pages' per-layer join of the routed experts' results
+ * (vramglass.com, section その2：GPUとCPUで同時に計算する). */
+MOE_API moe_status moe_combine(moe_ctx* ctx, const moe_layer_cfg* cfg, const moe_grouping* grouping,
+                       const float* z_rows, const void* x, int T, void* y, moe_stream stream);
+
+/* The whole step: router -> top-k -> grouping -> experts -> combine. Picks the
+ * decode path for T <= MOE_DECODE_MAX_T and the tensor-core grouped GEMM path
+ * otherwise. Arguments as above; ws must hold moe_workspace_bytes(cfg, T). */
+MOE_API moe_status moe_layer_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, const void* x, int T,
+                             const float* w_router, const float* logit_bias,
+                             const int32_t* slot_of, int n_slots, const uint8_t* slot_pool,
+                             size_t slot_stride, const uint8_t* shared_expert, void* ws,
+                             size_t ws_bytes, void* y, moe_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */
