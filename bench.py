@@ -2,12 +2,15 @@
 
 Default workload (decode): the full-size layer (d=2048, f=768, 512 routed
 experts, top-10 plus 1 shared, 2-bit block-32 fp16-scale weights, Zipf(1.1)
-routing) at T=1, stacked 48 deep with x_{l+1} = bf16(x_l + y_l), every layer
-with its own router, shared expert and 512 experts in a 24,576-slot pool
+routing) at T=1, run for 48 layers in a row, every layer with its own seeded
+input tokens, router, shared expert and 512 experts in a 24,576-slot pool
 (36.2 GB) behind a slot table whose 4,500 most popular experts sit in slots
-0..4,499. One step = one pass of all 48 layers; the 48 layers' weights
-(~1 GB touched per step) do not fit in the 126 MB L2, so every layer reads
-its weights from HBM.
+0..4,499. (Chaining x_{l+1} = x_l + y_l through random-weight layers with no
+normalisation diverges within three layers, after which the router no longer
+follows the seeded routing; each layer therefore reads its own seeded x_l.)
+One step = one pass of all 48 layers; the 48 layers' weights (~1 GB touched
+per step) do not fit in the 126 MB L2, so every layer reads its weights from
+HBM.
 
 --workload prefill: one layer at T=8192 (81,920 token-expert pairs).
 
@@ -33,7 +36,7 @@ METRIC = "MoE decode tok/s & expert-weight GB/s vs HBM peak (2-bit, top-10 of 51
 LAYERS = 48
 HOT = 4500
 SEED = 0
-KERNELS_PER_LAYER_DECODE = 5  # router, top-k, grouping, gate/up, down+combine
+KERNELS_PER_LAYER_DECODE = 1  # one fused decode-layer kernel
 
 
 def peaks():
@@ -141,7 +144,7 @@ class DecodeStack:
         from bit_expert_ffn_router_b200 import synth
         self.M, self.torch = M, torch
         self.T, self.L = T, layers
-        self.cfg = M.FULL.replace(bits=bits, out_fp32=0, residual=1)
+        self.cfg = M.FULL.replace(bits=bits, out_fp32=0)
         cfg = self.cfg
         self.lay = M.expert_layout(cfg)
         self.stride = self.lay["bytes"]
@@ -166,11 +169,9 @@ class DecodeStack:
         bias = np.stack([synth.bias_from_sets(synth.zipf_sets(T, cfg.E, cfg.k, seed + 1000 * l), cfg.E)
                          for l in range(layers)])
         self.bias = torch.from_numpy(bias).to(dev)
-        self.x0_host = synth.activations(T, cfg.d, seed + 16)
-        self.xbuf = [torch.empty(T, cfg.d, dtype=torch.bfloat16, device=dev) for _ in range(2)]
-        self.xbuf[0].copy_(torch.from_numpy(self.x0_host.view(np.int16)).view(torch.bfloat16))
-        self.x_in = torch.empty_like(self.xbuf[0])
-        self.x_in.copy_(self.xbuf[0])
+        self.x_host = np.stack([synth.activations(T, cfg.d, seed + 1000 * l + 16) for l in range(layers)])
+        self.x_in = torch.from_numpy(self.x_host.view(np.int16)).to(dev).view(torch.bfloat16)  # [L, T, d]
+        self.y_out = torch.empty(layers, T, cfg.d, dtype=torch.bfloat16, device=dev)
         self.ws = M.workspace(cfg, T)
         self.ctx = M.Context(torch.cuda.current_device())
         self.graph = None
@@ -186,13 +187,9 @@ class DecodeStack:
                                self.n_slots, self.pool, self.stride, self.shared[l], self.ws, y)
 
     def step_eager(self):
-        # x_in -> 48 layers -> xbuf[L % 2]
-        src = self.x_in
         for l in range(self.L):
-            dst = self.xbuf[(l + 1) % 2]
-            self.layer(l, src, dst)
-            src = dst
-        return src
+            self.layer(l, self.x_in[l], self.y_out[l])
+        return self.y_out
 
     def capture(self):
         torch = self.torch
@@ -218,7 +215,7 @@ class DecodeStack:
         wss = []
         for l in range(self.L):
             ws = M.workspace(cfg, self.T)
-            self.ctx.router_topk(cfg, self.x_in, self.wr[l], self.bias[l], self.T, logits, idx, gate)
+            self.ctx.router_topk(cfg, self.x_in[l], self.wr[l], self.bias[l], self.T, logits, idx, gate)
             groups.append(self.ctx.group_tokens(cfg, idx, gate, self.T, self.slot_of[l * cfg.E:(l + 1) * cfg.E],
                                                 self.n_slots, ws))
             wss.append(ws)
@@ -228,7 +225,8 @@ class DecodeStack:
             for l in range(self.L):
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(st)
-                self.ctx.expert_ffn(cfg, self.x_in, groups[l], self.pool, self.stride, self.shared[l], wss[l], None, y)
+                self.ctx.expert_ffn(cfg, self.x_in[l], groups[l], self.pool, self.stride, self.shared[l], wss[l], None,
+                                    y)
                 b.record(st)
                 if r > 0:
                     evs.append((a, b, l))
@@ -269,7 +267,7 @@ def run_ours(args):
     achieved = ffn_bytes / (ffn_ms / 1e3) / 1e9
 
     # end to end through the public API: pinned host x in, 48 eager layer calls, host y out
-    xh = torch.from_numpy(st.x0_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+    xh = torch.from_numpy(st.x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
     yh = torch.empty_like(xh).pin_memory()
     for _ in range(2):
         st.x_in.copy_(xh, non_blocking=True)
@@ -323,8 +321,9 @@ def run_ours(args):
             "traffic": None, "avg_launch_us": round(ffn_ms * 1e3, 3), "bytes_per_launch": ffn_bytes,
         },
         "e2e": {"value": round(e2e_value, 2), "unit": "tokens/s (48-layer MoE stack)",
-                "h2d_bytes_per_step": st.T * st.cfg.d * 2, "d2h_bytes_per_step": st.T * st.cfg.d * 2,
-                "how": "pinned host x -> 48 eager moe_layer_forward calls -> pinned host y, CUDA events"},
+                "h2d_bytes_per_step": st.L * st.T * st.cfg.d * 2, "d2h_bytes_per_step": st.L * st.T * st.cfg.d * 2,
+                "how": "pinned host x (48 layers' tokens) -> 48 eager moe_layer_forward calls -> pinned host y, "
+                       "CUDA events"},
         "gpu_launches": KERNELS_PER_LAYER_DECODE * st.L * args.steps,
         "clocks": clk.summary(),
     }
@@ -358,15 +357,12 @@ def cpu_baseline(st, n_layers):
     import threadpoolctl
     cfg = st.cfg
     inputs = [oracle_layer_inputs(st, l) for l in range(n_layers)]
-    x = st.x0_host
     t0 = time.perf_counter()
-    for wr, bias, recs, shared in inputs:
+    for l, (wr, bias, recs, shared) in enumerate(inputs):
         cache = O.ExpertCache(lambda e, r=recs: O.sections_from_record(r[e], cfg.d, cfg.f, cfg.bits),
                               cfg.d, cfg.f, cfg.bits)
         sh = O.expert_weights(O.sections_from_record(shared, cfg.d, cfg.f, cfg.bits), cfg.d, cfg.f, cfg.bits)
-        out = O.layer_forward(x, wr, cfg.k, cache, sh, bias=bias, residual=True)
-        from bit_expert_ffn_router_b200 import synth
-        x = synth.f32_to_bf16_bits(out["y"].astype(np.float32))
+        O.layer_forward(st.x_host[l], wr, cfg.k, cache, sh, bias=bias)
     dt = time.perf_counter() - t0
     per_layer = dt / n_layers
     info = threadpoolctl.threadpool_info()
@@ -395,17 +391,15 @@ def run_reference(args):
         sel = np.unique(np.argsort(-bias, axis=1)[:, :k])
         secs = {int(e): synth.expert_sections(cfg_d, cfg_f, bits, SEED + 100 + 1000 * l + int(e)) for e in sel}
         shared = synth.expert_sections(cfg_d, cfg_f, bits, SEED + 99 + 1000 * l)
-        layers.append((wr, bias, secs, shared))
-    x0 = synth.activations(T, cfg_d, SEED + 16)
+        x = synth.activations(T, cfg_d, SEED + 1000 * l + 16)
+        layers.append((x, wr, bias, secs, shared))
     times = []
     for step in range(args.warmup + args.steps):
-        x = x0
         t0 = time.perf_counter()
-        for wr, bias, secs, shared in layers:
+        for x, wr, bias, secs, shared in layers:
             cache = O.ExpertCache(lambda e, s=secs: s[e], cfg_d, cfg_f, bits)
             sh = O.expert_weights(shared, cfg_d, cfg_f, bits)
-            out = O.layer_forward(x, wr, k, cache, sh, bias=bias, residual=True)
-            x = synth.f32_to_bf16_bits(out["y"].astype(np.float32))
+            O.layer_forward(x, wr, k, cache, sh, bias=bias)
         dt = time.perf_counter() - t0
         if step >= args.warmup:
             times.append(dt / layers_per_step)

@@ -1,0 +1,950 @@
+// Decode path (T <= MOE_DECODE_MAX_T): one persistent kernel per layer.
+//
+// The pages' engine reads, per token and layer, the router, the shared expert
+// and the 10 routed experts it picks, and its speed is set by how fast those
+// bytes arrive (vramglass.com, sections なぜVRAM 12GBで足りるのか and
+// その2：GPUとCPUで同時に計算する; news.blueqat.app/post/3262, section
+// GPU・CPU・RAM・SSDの分担). On a B200 every expert sits in HBM, so the step is
+// a chain of HBM-bound GEMVs whose cost is mostly latency: this kernel keeps
+// the weight stream continuous across the whole layer.
+//
+// One CTA per SM, 15 consumer warps + 1 producer warp:
+//   producer: cp.async.bulk copies of this CTA's weight rows into a
+//             shared-memory byte ring, one mbarrier per stage, issued as far
+//             ahead as the ring allows (the down-projection rows stream in
+//             while gate/up is still computing);
+//   consumers: [router rows -> grid barrier -> top-k + grouping (every CTA
+//             computes it, CTA 0 publishes it)] -> gate/up + SwiGLU into h ->
+//             grid barrier -> down rows of this CTA's output slice for every
+//             (expert, token) -> combine in top-k order -> y.
+// The shared expert's gate/up rows are fetched before routing is known and
+// are computed while other CTAs finish their router rows.
+//
+// Grid barriers and every mbarrier wait are bounded by a global-timer limit;
+// on expiry the kernel records MOE_ETIMEOUT in the context's status word,
+// drains its own copies and returns.
+#include "moe_internal.cuh"
+#include "dequant.cuh"
+
+namespace moe {
+
+// Consumer warps per CTA (plus one producer warp): 15 for 2-bit rows (four
+// warps per SM sub-partition, <= 128 registers each), 11 for 3-bit rows,
+// whose high-plane operands need more registers.
+__host__ __device__ constexpr int consumer_warps(int bits) { return bits == 2 ? 15 : 11; }
+constexpr int kNB = 32;               // stage mbarrier ring
+constexpr int kStageAlign = 128;
+
+enum : int { kStGU = 0, kStDN = 1 };
+constexpr int kShared = -1;  // expert id of the shared expert in stage records
+
+struct StageRec {
+  int type, u, a, b;  // GU: expert u, channels [a, b); DN: expert u, rows [a, b)
+  int off, bytes, code_bytes, pad;
+};
+
+struct DLParams {
+  const uint16_t* x;
+  int T, d, f, E, k, renorm, residual, has_shared, out_f32;
+  const float* wr;
+  const float* bias;
+  float* logits;
+  int32_t* idx;
+  float* gate;
+  const int32_t* slot_of;
+  int n_slots;
+  GroupPtrs g;
+  const uint8_t* pool;
+  size_t stride;
+  const uint8_t* shared;
+  moe_expert_layout lay;
+  float* h;
+  void* y;
+  int* status;
+  unsigned long long* gbar;  // grid-barrier arrival counter
+  unsigned long long timeout_ns;
+  unsigned long long* trace;  // null, or kTraceSlots timestamps per CTA
+  int rpc;         // down rows per CTA
+  int gu_lpr, dn_lpr;
+  int gu_row, gu_sc, dn_row, dn_sc;  // bytes per row: codes and scales
+  int gu_chan;     // channels per gate/up stage (one per consumer warp)
+  // shared-memory map (byte offsets), computed on the host
+  int sm_stages, sm_route, sm_zs, sm_xq, sm_wr, sm_hq, sm_ring, ring_bytes, max_stages, wr_rows;
+  int h_rows;      // quantised h rows the staging area holds
+};
+
+// ------------------------------------------------------------------ grid barrier
+// A monotonic 64-bit arrival counter shared by all launches on a context:
+// every CTA arrives exactly once per barrier episode and none arrives at the
+// next episode before the current one completes, so an arrival that reads
+// `old` belongs to the episode ending at (old / G + 1) * G.
+__device__ __forceinline__ unsigned long long gbar_arrive(unsigned long long* gb, unsigned nctas) {
+  __threadfence();
+  const unsigned long long old = atomicAdd(gb, 1ull);
+  return (old / nctas + 1) * nctas;
+}
+
+__device__ __forceinline__ bool gbar_wait(const unsigned long long* gb, unsigned long long target,
+                                          uint64_t deadline) {
+  while (ld_acquire_gpu_u64(gb) < target) {
+    if (global_timer_ns() > deadline) return false;
+    __nanosleep(32);
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------ shared state
+struct DLShared {
+  uint64_t full[kNB];
+  uint64_t empty[kNB];
+  uint64_t wr_bar;
+  uint64_t list_bar;
+  int abort_flag;
+  int n_sh, n_gu, n_st;  // shared-expert GU stages, all GU stages, all stages
+  int n_uniq;
+  unsigned long long bar_target;
+};
+
+struct RouteSmem {
+  int32_t* idx;        // [T*k]
+  float* gate;         // [T*k]
+  int32_t* sorted_e;   // [np]
+  int32_t* pair_token; // [np]
+  float* pair_gate;    // [np]
+  int32_t* pair_pos;   // [T*k]
+  int32_t* uniq_e;     // [np]
+  int32_t* uniq_slot;  // [np]
+  int32_t* uniq_off;   // [np + 1]
+};
+
+__device__ __forceinline__ RouteSmem route_smem(char* base, int np) {
+  RouteSmem r;
+  int32_t* p = reinterpret_cast<int32_t*>(base);
+  r.idx = p;
+  r.gate = reinterpret_cast<float*>(p + np);
+  r.sorted_e = p + 2 * np;
+  r.pair_token = p + 3 * np;
+  r.pair_gate = reinterpret_cast<float*>(p + 4 * np);
+  r.pair_pos = p + 5 * np;
+  r.uniq_e = p + 6 * np;
+  r.uniq_slot = p + 7 * np;
+  r.uniq_off = p + 8 * np;
+  return r;
+}
+
+__device__ __forceinline__ void set_abort(DLShared* S, int* status, int where) {
+  report(status, kDevTimeout, where);
+  *reinterpret_cast<volatile int*>(&S->abort_flag) = 1;
+}
+
+__device__ __forceinline__ bool aborted(DLShared* S) {
+  return *reinterpret_cast<volatile int*>(&S->abort_flag) != 0;
+}
+
+// ------------------------------------------------------------------ stage list
+// GU stages for channels [c0, c1) of expert u, at most gu_chan channels each.
+__device__ int push_gu(StageRec* st, int n, int u, int c0, int c1, const DLParams& P) {
+  const int gu_row = P.gu_row, gu_sc = P.gu_sc;
+  for (int c = c0; c < c1; c += P.gu_chan) {
+    const int e = min(c + P.gu_chan, c1);
+    StageRec r;
+    r.type = kStGU;
+    r.u = u;
+    r.a = c;
+    r.b = e;
+    r.code_bytes = 2 * (e - c) * gu_row;
+    r.bytes = r.code_bytes + 2 * (e - c) * gu_sc;
+    r.off = 0;
+    r.pad = 0;
+    st[n++] = r;
+  }
+  return n;
+}
+
+__device__ int push_dn(StageRec* st, int n, int u, int r0, int r1, const DLParams& P) {
+  if (r1 <= r0) return n;
+  const int dn_row = P.dn_row, dn_sc = P.dn_sc;
+  StageRec r;
+  r.type = kStDN;
+  r.u = u;
+  r.a = r0;
+  r.b = r1;
+  r.code_bytes = (r1 - r0) * dn_row;
+  r.bytes = r.code_bytes + (r1 - r0) * dn_sc;
+  r.off = 0;
+  r.pad = 0;
+  st[n++] = r;
+  return n;
+}
+
+// ------------------------------------------------------------------ producer
+struct Ring {
+  int head;       // end of the newest live stage
+  int tail;       // oldest live stage index
+  int issued;     // stages issued so far
+};
+
+__device__ __forceinline__ const uint8_t* expert_record(const DLParams& P, const RouteSmem& R, int u) {
+  return u == kShared ? P.shared : P.pool + static_cast<size_t>(R.uniq_slot[u]) * P.stride;
+}
+
+// Sorted rows (pairs) an expert's FFN runs for: routed u -> its pairs; shared -> np + t.
+__device__ __forceinline__ void expert_rows(const RouteSmem& R, int u, int np, int T, int& p0, int& p1) {
+  if (u == kShared) {
+    p0 = np;
+    p1 = np + T;
+  } else {
+    p0 = R.uniq_off[u];
+    p1 = R.uniq_off[u + 1];
+  }
+}
+
+// Frees the oldest live stage (waits for its consumer). False on timeout.
+__device__ bool ring_pop(DLShared* S, StageRec* st, Ring& rg, uint64_t deadline) {
+  const int j = rg.tail;
+  if (!mbar_wait(&S->empty[j % kNB], (j / kNB) & 1, deadline)) return false;
+  rg.tail++;
+  if (rg.tail == rg.issued) rg.head = 0;
+  return true;
+}
+
+__device__ bool ring_issue(DLShared* S, StageRec* st, Ring& rg, int i, uint8_t* ring, int cap,
+                           const DLParams& P, const RouteSmem& R, uint64_t deadline) {
+  StageRec& s = st[i];
+  const int need = (s.bytes + kStageAlign - 1) / kStageAlign * kStageAlign;
+  int start = -1;
+  while (true) {
+    if (aborted(S)) return false;
+    if (rg.tail == rg.issued) {
+      rg.head = 0;
+      start = 0;
+      break;
+    }
+    if (i - rg.tail < kNB) {
+      const int toff = st[rg.tail].off;
+      if (rg.head > toff) {  // live region does not wrap
+        if (rg.head + need <= cap) { start = rg.head; break; }
+        if (need <= toff) { start = 0; break; }
+      } else if (rg.head + need <= toff) {
+        start = rg.head;
+        break;
+      }
+    }
+    if (!ring_pop(S, st, rg, deadline)) return false;
+  }
+  s.off = start;
+  rg.head = start + need;
+  const uint8_t* rec = expert_record(P, R, s.u);
+  uint8_t* dst = ring + start;
+  uint64_t* bar = &S->full[i % kNB];
+  mbar_arrive_expect_tx(bar, static_cast<uint32_t>(s.bytes));
+  if (s.type == kStGU) {
+    const int rows = 2 * (s.b - s.a);
+    const int row_b = s.code_bytes / rows;
+    const int sc_b = (s.bytes - s.code_bytes) / rows;
+    bulk_g2s(dst, rec + P.lay.gu_codes + static_cast<size_t>(2 * s.a) * row_b, s.code_bytes, bar);
+    bulk_g2s(dst + s.code_bytes, rec + P.lay.gu_scales + static_cast<size_t>(2 * s.a) * sc_b,
+             s.bytes - s.code_bytes, bar);
+  } else {
+    const int rows = s.b - s.a;
+    const int row_b = s.code_bytes / rows;
+    const int sc_b = (s.bytes - s.code_bytes) / rows;
+    bulk_g2s(dst, rec + P.lay.dn_codes + static_cast<size_t>(s.a) * row_b, s.code_bytes, bar);
+    bulk_g2s(dst + s.code_bytes, rec + P.lay.dn_scales + static_cast<size_t>(s.a) * sc_b,
+             s.bytes - s.code_bytes, bar);
+  }
+  rg.issued = i + 1;
+  return true;
+}
+
+// ------------------------------------------------------------------ consumers
+// Quantises the T token rows of x (bf16, global) into the gate/up layout.
+template <int BITS>
+__device__ void quantise_x(const DLParams& P, int* xq, int nct) {
+  const int nb = P.d / kBlock, bpl = nb / P.gu_lpr;
+  const int words = QV<BITS>::kWords * nb;
+  for (int job = threadIdx.x; job < P.T * nb; job += nct) {
+    const int t = job / nb, blk = job % nb;
+    const uint4* src = reinterpret_cast<const uint4*>(P.x + static_cast<size_t>(t) * P.d + blk * kBlock);
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 q = __ldcg(src + i);
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+        v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+      }
+    }
+    const int gl = blk / bpl, bb = blk % bpl;
+    quant_block<BITS>(v, xq + t * words, nb, bb * P.gu_lpr + gl);
+  }
+}
+
+// Quantises h rows [lo, hi) (fp32, global) into the down layout.
+template <int BITS>
+__device__ void quantise_h(const DLParams& P, int lo, int hi, int* hq, int nct) {
+  const int nb = P.f / kBlock, bpl = nb / P.dn_lpr;
+  const int words = QV<BITS>::kWords * nb;
+  for (int job = threadIdx.x; job < (hi - lo) * nb; job += nct) {
+    const int r = job / nb, blk = job % nb;
+    const float4* src = reinterpret_cast<const float4*>(P.h + static_cast<size_t>(lo + r) * P.f + blk * kBlock);
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 q = __ldcg(src + i);
+      v[4 * i] = q.x;
+      v[4 * i + 1] = q.y;
+      v[4 * i + 2] = q.z;
+      v[4 * i + 3] = q.w;
+    }
+    const int gl = blk / bpl, bb = blk % bpl;
+    quant_block<BITS>(v, hq + r * words, nb, bb * P.dn_lpr + gl);
+  }
+}
+
+// Gate/up stage: warp w computes channel a + w (gate row and up row side by
+// side) for every token of the stage's expert and writes h.
+template <int BITS, int BPL>
+__device__ __forceinline__ void process_gu(const StageRec& s, const uint8_t* ring, const DLParams& P,
+                                           const RouteSmem& R, int np, const int* xq, int& cur_t, XR<BITS>* xr) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c = s.a + warp;
+  const int lpr = P.gu_lpr, gl = lane % lpr;
+  const bool active = lane < lpr;  // lane group 0 holds the channel's two rows
+  const int rows = 2 * (s.b - s.a);
+  const int row_b = s.code_bytes / rows;
+  const int nb = P.d / kBlock, sc_n = nb;
+  const uint8_t* cg = ring + s.off + 2 * (c - s.a) * row_b;
+  const uint16_t* sg = reinterpret_cast<const uint16_t*>(ring + s.off + s.code_bytes) + 2 * (c - s.a) * sc_n;
+  int p0, p1;
+  expert_rows(R, s.u, np, P.T, p0, p1);
+#pragma unroll 1
+  for (int p = p0; p < p1; ++p) {
+    const int t = (s.u == kShared) ? p - np : R.pair_token[p];
+    if (t != cur_t) {
+      load_xr<BITS, BPL>(xq + t * QV<BITS>::kWords * nb, nb, lpr, gl, xr);
+      cur_t = t;
+    }
+    float2 v = make_float2(0.f, 0.f);
+    if (active) v = row_dot2<BITS, BPL>(cg, sg, cg + row_b, sg + sc_n, P.d, gl, xr);
+    v.x = group_sum(v.x, lpr);
+    v.y = group_sum(v.y, lpr);
+    if (lane == 0) P.h[static_cast<size_t>(p) * P.f + c] = v.x / (1.f + expf(-v.x)) * v.y;
+  }
+}
+
+// Down stage (one expert, this CTA's output rows) by one warp: for every
+// token of the expert, its quantised h row is held in registers and the
+// rows are swept RPW at a time.
+template <int BITS, int BPL>
+__device__ __forceinline__ void process_dn(const StageRec& s, const uint8_t* ring, const DLParams& P,
+                                           const RouteSmem& R, int np, const int* hq, int h_lo, float* zs) {
+  const int lane = threadIdx.x & 31;
+  const int lpr = P.dn_lpr, rpw = 32 / lpr;
+  const int rl = lane / lpr, gl = lane % lpr;
+  const int rows = s.b - s.a;
+  const uint8_t* codes = ring + s.off;
+  const uint16_t* scales = reinterpret_cast<const uint16_t*>(ring + s.off + s.code_bytes);
+  const int row_b = s.code_bytes / rows;
+  const int nb = P.f / kBlock, sc_n = nb;
+  int p0, p1;
+  expert_rows(R, s.u, np, P.T, p0, p1);
+  XR<BITS> hr[BPL];
+#pragma unroll 1
+  for (int p = p0; p < p1; ++p) {
+    load_xr<BITS, BPL>(hq + (p - h_lo) * QV<BITS>::kWords * nb, nb, lpr, gl, hr);
+#pragma unroll 1
+    for (int r0 = 0; r0 < rows; r0 += rpw) {
+      const int r = r0 + rl;
+      float v = 0.f;
+      if (r < rows) v = row_dot<BITS, BPL>(codes + r * row_b, scales + r * sc_n, P.f, gl, hr);
+      v = group_sum(v, lpr);
+      if (gl == 0 && r < rows) zs[p * P.rpc + r] = v;
+    }
+  }
+}
+
+// Stable sort of the T*k pairs by expert inside the CTA, unique experts and
+// slot lookup. Every consumer thread takes part.
+__device__ void group_in_smem(const DLParams& P, const RouteSmem& R, DLShared* S, int np, int nct) {
+  const int tid = threadIdx.x;
+  for (int p = tid; p < np; p += nct) {
+    const int e = min(max(R.idx[p], 0), P.E - 1);
+    int pos = 0;
+    for (int q = 0; q < np; ++q) {
+      const int eq = min(max(R.idx[q], 0), P.E - 1);
+      pos += (eq < e) || (eq == e && q < p);
+    }
+    R.sorted_e[pos] = e;
+    R.pair_token[pos] = p / P.k;
+    R.pair_gate[pos] = R.gate[p];
+    R.pair_pos[p] = pos;
+  }
+  named_sync(1, nct);
+  if (tid < 32) {
+    int base = 0;
+    for (int c = 0; c < np; c += 32) {
+      const int i = c + tid;
+      const bool first = i < np && (i == 0 || R.sorted_e[i - 1] != R.sorted_e[i]);
+      const unsigned m = __ballot_sync(0xffffffffu, first);
+      if (first) {
+        const int u = base + __popc(m & ((1u << tid) - 1u));
+        const int e = R.sorted_e[i];
+        int slot = P.slot_of[e];
+        if (slot < 0 || slot >= P.n_slots) {
+          report(P.status, kDevBadSlot, e);
+          slot = 0;
+        }
+        R.uniq_e[u] = e;
+        R.uniq_slot[u] = slot;
+        R.uniq_off[u] = i;
+      }
+      base += __popc(m);
+    }
+    if (tid == 0) {
+      R.uniq_off[base] = np;
+      S->n_uniq = base;
+    }
+  }
+  named_sync(1, nct);
+}
+
+// CTA 0 publishes the grouping in the layout of moe_grouping.
+__device__ void publish_grouping(const DLParams& P, const RouteSmem& R, int n_uniq, int np, int nct) {
+  const int tid = threadIdx.x;
+  for (int p = tid; p < np; p += nct) {
+    P.g.pair_token[p] = R.pair_token[p];
+    P.g.pair_gate[p] = R.pair_gate[p];
+    P.g.pair_pos[p] = R.pair_pos[p];
+    int j = 0;
+    for (int q = 0; q < P.k; ++q) j = (R.pair_pos[R.pair_token[p] * P.k + q] == p) ? q : j;
+    P.g.pair_j[p] = j;
+    int u = 0;
+    for (int v = 0; v < n_uniq; ++v) u = (R.uniq_off[v] <= p) ? v : u;
+    P.g.pair_slot[p] = R.uniq_slot[u];
+  }
+  for (int u = tid; u < n_uniq; u += nct) {
+    P.g.uniq_expert[u] = R.uniq_e[u];
+    P.g.uniq_slot[u] = R.uniq_slot[u];
+    P.g.uniq_offset[u] = R.uniq_off[u];
+  }
+  if (tid == 0) {
+    P.g.uniq_offset[n_uniq] = np;
+    *P.g.n_uniq = n_uniq;
+  }
+  for (int e = tid; e < P.E; e += nct) {
+    int below = 0, cnt = 0;
+    for (int q = 0; q < np; ++q) {
+      below += R.sorted_e[q] < e;
+      cnt += R.sorted_e[q] == e;
+    }
+    P.g.expert_count[e] = cnt;
+    P.g.expert_offset[e] = below;
+    if (e == P.E - 1) P.g.expert_offset[P.E] = below + cnt;
+  }
+}
+
+// Top-k of token t by one warp over the fp32 logits in global memory, with
+// the selection rule of the standalone top-k kernel: largest first, equal
+// logits to the lower expert index, NaN below every number, -0 == +0.
+// Key per value: order-preserving bits + 1 (NaN -> 1, taken/absent -> 0).
+// Each round: warp max of the keys, then the lowest index holding it.
+// E <= 512 (16 values per lane).
+__device__ __forceinline__ uint32_t order_key(float v) {
+  if (v != v) return 1u;
+  uint32_t u = __float_as_uint(v);
+  if (u == 0x80000000u) u = 0u;
+  return ((u & 0x80000000u) ? ~u : (u | 0x80000000u)) + 1u;
+}
+
+__device__ __forceinline__ float key_value(uint32_t k) {
+  if (k <= 1u) return __uint_as_float(0x7fc00000u);
+  const uint32_t o = k - 1u;
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
+__device__ void topk_warp(const DLParams& P, const RouteSmem& R, int t) {
+  constexpr int VPL = 16;
+  const int lane = threadIdx.x & 31;
+  const float* row = P.logits + static_cast<size_t>(t) * P.E;
+  uint32_t key[VPL];
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) {
+    const int e = v * 32 + lane;
+    key[v] = e < P.E ? order_key(__ldcg(row + e)) : 0u;
+  }
+  uint32_t mine_key = 0u;
+  int mine_e = 0;
+#pragma unroll 1
+  for (int j = 0; j < P.k; ++j) {
+    uint32_t lm = 0u;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) lm = max(lm, key[v]);
+    const uint32_t M = __reduce_max_sync(0xffffffffu, lm);
+    uint32_t my = 0xffffffffu;
+#pragma unroll
+    for (int v = VPL - 1; v >= 0; --v)
+      if (key[v] == M) my = static_cast<uint32_t>(v * 32 + lane);
+    const int e = static_cast<int>(__reduce_min_sync(0xffffffffu, lm == M ? my : 0xffffffffu));
+    if ((e & 31) == lane) {
+#pragma unroll
+      for (int v = 0; v < VPL; ++v)
+        if (v == (e >> 5)) key[v] = 0u;
+    }
+    if (lane == j) {
+      mine_key = M;
+      mine_e = e;
+    }
+  }
+  const bool sel = lane < P.k;
+  const float lj = sel ? key_value(mine_key) : 0.f;
+  const float l0 = __shfl_sync(0xffffffffu, lj, 0);
+  const float ex = sel ? expf(lj - l0) : 0.f;
+  float denom;
+  if (P.renorm) {
+    denom = warp_sum(ex);
+  } else {
+    float s = 0.f;
+    for (int e = lane; e < P.E; e += 32) s += expf(__ldcg(row + e) - l0);
+    denom = warp_sum(s);
+  }
+  if (sel) {
+    R.idx[t * P.k + lane] = mine_e;
+    R.gate[t * P.k + lane] = ex / denom;
+  }
+}
+
+// Router rows [e0, e1) of this CTA for every token: lanes read W_r (shared
+// memory) and x (global, bf16) in interleaved 4-column groups.
+__device__ void router_rows(const DLParams& P, const float* wrs, int e0, int e1, int cw) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n4 = P.d / 4;
+  for (int t = 0; t < P.T; ++t) {
+    const uint2* x2 = reinterpret_cast<const uint2*>(P.x + static_cast<size_t>(t) * P.d);
+#pragma unroll 1
+    for (int e = e0 + warp; e < e1; e += cw) {
+      const float4* w4 = reinterpret_cast<const float4*>(wrs + static_cast<size_t>(e - e0) * P.d);
+      float acc = 0.f;
+#pragma unroll 4
+      for (int c4 = lane; c4 < n4; c4 += 32) {
+        const float4 w = w4[c4];
+        const uint2 xb = __ldcg(x2 + c4);
+        acc = fmaf(w.x, __uint_as_float(xb.x << 16), acc);
+        acc = fmaf(w.y, __uint_as_float(xb.x & 0xffff0000u), acc);
+        acc = fmaf(w.z, __uint_as_float(xb.y << 16), acc);
+        acc = fmaf(w.w, __uint_as_float(xb.y & 0xffff0000u), acc);
+      }
+      acc = warp_sum(acc);
+      if (lane == 0) {
+        const size_t o = static_cast<size_t>(t) * P.E + e;
+        P.logits[o] = P.bias ? acc + P.bias[o] : acc;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ the kernel
+// Control flow is the same for every consumer thread (all named barriers are
+// reached by all of them); a timeout only turns the remaining work off.
+template <int BITS, int GBPL, int DBPL, bool ROUTE>
+__global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_layer_kernel(const DLParams P) {
+  constexpr int CW = consumer_warps(BITS);
+  constexpr int CT = CW * 32;
+  extern __shared__ __align__(128) char smem[];
+  DLShared* S = reinterpret_cast<DLShared*>(smem);
+  StageRec* st = reinterpret_cast<StageRec*>(smem + P.sm_stages);
+  const int np = P.T * P.k;
+  const RouteSmem R = route_smem(smem + P.sm_route, np);
+  float* zs = reinterpret_cast<float*>(smem + P.sm_zs);
+  int* xq = reinterpret_cast<int*>(smem + P.sm_xq);
+  float* wrs = reinterpret_cast<float*>(smem + P.sm_wr);
+  int* hq = reinterpret_cast<int*>(smem + P.sm_hq);
+  uint8_t* ring = reinterpret_cast<uint8_t*>(smem + P.sm_ring);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = gridDim.x, b = blockIdx.x;
+  const uint64_t t_start = global_timer_ns();
+  const uint64_t deadline = t_start + P.timeout_ns;
+  unsigned long long* trace = P.trace != nullptr && b < kTraceCtas ? P.trace + b * kTraceSlots : nullptr;
+#define MOE_TRACE(slot) \
+  if (trace != nullptr) trace[(slot)] = global_timer_ns();
+
+  // static splits: router rows, shared-expert channels, output rows of this CTA
+  const int e0 = static_cast<int>((static_cast<long long>(P.E) * b) / G);
+  const int e1 = static_cast<int>((static_cast<long long>(P.E) * (b + 1)) / G);
+  const int cs0 = static_cast<int>((static_cast<long long>(P.f) * b) / G);
+  const int cs1 = static_cast<int>((static_cast<long long>(P.f) * (b + 1)) / G);
+  const int r0 = min(b * P.rpc, P.d), r1 = min(r0 + P.rpc, P.d);
+
+  if (threadIdx.x == 0) {
+    if (trace != nullptr) {
+      trace[0] = t_start;
+      trace[14] = clock64();
+    }
+    for (int i = 0; i < kNB; ++i) {
+      mbar_init(&S->full[i], 1);
+      mbar_init(&S->empty[i], CW);
+    }
+    mbar_init(&S->wr_bar, 1);
+    mbar_init(&S->list_bar, 1);
+    S->abort_flag = 0;
+    S->n_sh = P.has_shared ? push_gu(st, 0, kShared, cs0, cs1, P) : 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == CW) {
+    // ------------------------------------------------------------ producer
+    if (lane != 0) return;
+    Ring rg{0, 0, 0};
+    bool ok = true, wr_issued = false;
+    if (ROUTE && e1 > e0) {
+      const uint32_t bytes = static_cast<uint32_t>((e1 - e0) * P.d * 4);
+      mbar_arrive_expect_tx(&S->wr_bar, bytes);
+      bulk_g2s(wrs, P.wr + static_cast<size_t>(e0) * P.d, bytes, &S->wr_bar);
+      wr_issued = true;
+    }
+    const int n_sh = S->n_sh;
+    int n_st = n_sh;
+    for (int i = 0; ok; ++i) {
+      if (i == n_sh) {
+        if (!mbar_wait(&S->list_bar, 0, deadline)) {
+          ok = false;
+          break;
+        }
+        MOE_TRACE(12)
+        n_st = S->n_st;
+      }
+      if (i >= n_st) break;
+      ok = ring_issue(S, st, rg, i, ring, P.ring_bytes, P, R, deadline);
+    }
+    MOE_TRACE(13)
+    if (!ok) {
+      if (!aborted(S)) set_abort(S, P.status, 10);
+      // every issued copy must land before the CTA may exit; copies finish
+      // in microseconds, the 100 ms bound only guards against the impossible
+      const uint64_t d2 = global_timer_ns() + 100000000ull;
+      for (int j = rg.tail; j < rg.issued; ++j) mbar_wait(&S->full[j % kNB], (j / kNB) & 1, d2);
+      if (wr_issued) mbar_wait(&S->wr_bar, 0, d2);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int tid = threadIdx.x;
+  grid_dep_wait();  // x (and the workspace) may come from the previous kernel
+  quantise_x<BITS>(P, xq, CT);
+  named_sync(1, CT);
+  if (tid == 0) MOE_TRACE(1)
+
+  if (ROUTE) {
+    if (e1 > e0 && !mbar_wait_warp(&S->wr_bar, 0, deadline)) set_abort(S, P.status, 1);
+    if (!aborted(S)) router_rows(P, wrs, e0, e1, CW);
+    named_sync(1, CT);
+    if (tid == 0) MOE_TRACE(2)
+    if (tid == 0 && !aborted(S)) S->bar_target = gbar_arrive(P.gbar, G);
+  }
+
+  // gate/up stages: the shared expert's [0, n_sh) need no routing; routing is
+  // resolved when the loop reaches n_sh, then the routed stages follow
+  XR<BITS> xr[GBPL];
+  int cur_t = -1;
+  const int n_sh = S->n_sh;
+  int n_gu = n_sh;
+#pragma unroll 1
+  for (int i = 0;; ++i) {
+    if (i == n_sh) {
+      if (tid == 0) MOE_TRACE(3)
+      if (ROUTE) {
+        if (tid == 0 && !aborted(S) && !gbar_wait(P.gbar, S->bar_target, deadline)) set_abort(S, P.status, 3);
+        named_sync(1, CT);
+        if (tid == 0) MOE_TRACE(4)
+        if (!aborted(S))
+          for (int t = warp; t < P.T; t += CW) topk_warp(P, R, t);
+        named_sync(1, CT);
+        if (tid == 0) MOE_TRACE(10)
+        if (b == 0)
+          for (int q = tid; q < np; q += CT) {
+            P.idx[q] = R.idx[q];
+            P.gate[q] = R.gate[q];
+          }
+        group_in_smem(P, R, S, np, CT);
+        if (b == 0) publish_grouping(P, R, S->n_uniq, np, CT);
+      } else {
+        // grouping written by moe_group_tokens
+        const int nu = min(max(__ldcg(P.g.n_uniq), 0), min(np, P.E));
+        for (int p = tid; p < np; p += CT) {
+          R.pair_token[p] = min(max(__ldcg(P.g.pair_token + p), 0), P.T - 1);
+          R.pair_gate[p] = __ldcg(P.g.pair_gate + p);
+          R.pair_pos[p] = min(max(__ldcg(P.g.pair_pos + p), 0), np - 1);
+        }
+        for (int u = tid; u <= nu; u += CT) {
+          R.uniq_off[u] = min(max(__ldcg(P.g.uniq_offset + u), 0), np);
+          if (u < nu) {
+            int slot = __ldcg(P.g.uniq_slot + u);
+            if (slot < 0 || slot >= P.n_slots) {
+              report(P.status, kDevBadSlot, u);
+              slot = 0;
+            }
+            R.uniq_slot[u] = slot;
+          }
+        }
+        if (tid == 0) S->n_uniq = nu;
+        named_sync(1, CT);
+      }
+      // routed stage list: this CTA's share of the n_uniq*f routed gate/up
+      // channels, then the down slices: routed experts in order, shared last,
+      // so that the h rows they read are one ascending range
+      if (tid == 0) {
+        const int nu = S->n_uniq;
+        int n = n_sh;
+        const long long tot = static_cast<long long>(nu) * P.f;
+        long long c = tot * b / G;
+        const long long c1 = tot * (b + 1) / G;
+        while (c < c1) {
+          const int u = static_cast<int>(c / P.f);
+          const long long ub = static_cast<long long>(u) * P.f;
+          const int ce = static_cast<int>(min(c1, ub + P.f) - ub);
+          n = push_gu(st, n, u, static_cast<int>(c - ub), ce, P);
+          c = ub + ce;
+        }
+        S->n_gu = n;
+        for (int u = 0; u < nu; ++u) n = push_dn(st, n, u, r0, r1, P);
+        if (P.has_shared) n = push_dn(st, n, kShared, r0, r1, P);
+        S->n_st = n;
+        mbar_arrive(&S->list_bar);
+      }
+      named_sync(1, CT);
+      if (tid == 0) MOE_TRACE(5)
+      n_gu = S->n_gu;
+    }
+    if (i >= n_gu) break;
+    if (!aborted(S) && warp < st[i].b - st[i].a) {
+      if (mbar_wait_warp(&S->full[i % kNB], (i / kNB) & 1, deadline))
+        process_gu<BITS, GBPL>(st[i], ring, P, R, np, xq, cur_t, xr);
+      else
+        set_abort(S, P.status, 4);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S->empty[i % kNB]);
+  }
+  const int n_st = S->n_st;
+
+  // every h row of every CTA must be written before any down row is computed
+  named_sync(1, CT);
+  if (tid == 0) MOE_TRACE(6)
+  if (tid == 0 && !aborted(S)) {
+    const unsigned long long target = gbar_arrive(P.gbar, G);
+    if (!gbar_wait(P.gbar, target, deadline)) set_abort(S, P.status, 5);
+  }
+  named_sync(1, CT);
+  if (tid == 0) MOE_TRACE(7)
+  grid_dep_launch();
+
+  // down stages, in chunks whose h rows fit the quantised staging area
+#pragma unroll 1
+  for (int i0 = n_gu; i0 < n_st;) {
+    int q0, q1;
+    expert_rows(R, st[i0].u, np, P.T, q0, q1);
+    const int h_lo = q0;
+    int i1 = i0, h_hi = q0;
+    while (i1 < n_st) {
+      expert_rows(R, st[i1].u, np, P.T, q0, q1);
+      if (q1 - h_lo > P.h_rows) break;
+      h_hi = q1;
+      ++i1;
+    }
+    quantise_h<BITS>(P, h_lo, h_hi, hq, CT);
+    named_sync(1, CT);
+#pragma unroll 1
+    for (int i = i0; i < i1; ++i) {
+      if (!aborted(S) && (i - n_gu) % CW == warp) {
+        if (mbar_wait_warp(&S->full[i % kNB], (i / kNB) & 1, deadline))
+          process_dn<BITS, DBPL>(st[i], ring, P, R, np, hq, h_lo, zs);
+        else
+          set_abort(S, P.status, 6);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S->empty[i % kNB]);
+    }
+    named_sync(1, CT);
+    i0 = i1;
+  }
+  if (tid == 0) MOE_TRACE(8)
+  if (aborted(S)) return;
+
+  // combine: y[t, r] = sum_j gate[t,j] z[(t,j)][r] + z_shared[t][r] (+ x)
+  const int nr = r1 - r0;
+  for (int i = tid; i < P.T * nr; i += CT) {
+    const int t = i / nr, rr = i % nr;
+    float acc = 0.f;
+    for (int j = 0; j < P.k; ++j) {
+      const int p = R.pair_pos[t * P.k + j];
+      acc = fmaf(R.pair_gate[p], zs[p * P.rpc + rr], acc);
+    }
+    if (P.has_shared) acc += zs[(np + t) * P.rpc + rr];
+    const size_t o = static_cast<size_t>(t) * P.d + r0 + rr;
+    if (P.residual) acc += bf16_bits_to_float(P.x[o]);
+    if (P.out_f32) static_cast<float*>(P.y)[o] = acc;
+    else static_cast<__nv_bfloat16*>(P.y)[o] = __float2bfloat16_rn(acc);
+  }
+  named_sync(1, CT);
+  if (tid == 0) {
+    MOE_TRACE(9)
+    if (trace != nullptr) trace[15] = clock64();
+  }
+#undef MOE_TRACE
+}
+
+// ------------------------------------------------------------------ host side
+namespace {
+
+struct RowGeom {
+  int lpr, bpl;
+};
+
+RowGeom row_geom(int K) {
+  const int nb = K / kBlock;
+  int lpr = 1;
+  while (lpr < 32 && nb % (lpr * 2) == 0) lpr *= 2;
+  return RowGeom{lpr, nb / lpr};
+}
+
+size_t align_up(size_t n, size_t a) { return (n + a - 1) / a * a; }
+
+constexpr int kSmemMax = 227 * 1024;
+
+typedef void (*DLKernel)(const DLParams);
+
+template <int BITS, bool ROUTE>
+DLKernel pick(int gbpl, int dbpl) {
+  if (gbpl == 2 && dbpl == 3) return decode_layer_kernel<BITS, 2, 3, ROUTE>;
+  if (gbpl == 1 && dbpl == 1) return decode_layer_kernel<BITS, 1, 1, ROUTE>;
+  if (gbpl == 2 && dbpl == 2) return decode_layer_kernel<BITS, 2, 2, ROUTE>;
+  if (gbpl == 2 && dbpl == 1) return decode_layer_kernel<BITS, 2, 1, ROUTE>;
+  if (gbpl == 1 && dbpl == 3) return decode_layer_kernel<BITS, 1, 3, ROUTE>;
+  if (gbpl == 4 && dbpl == 3) return decode_layer_kernel<BITS, 4, 3, ROUTE>;
+  return nullptr;
+}
+
+DLKernel pick_kernel(int bits, bool route, int gbpl, int dbpl) {
+  if (bits == 2) return route ? pick<2, true>(gbpl, dbpl) : pick<2, false>(gbpl, dbpl);
+  return route ? pick<3, true>(gbpl, dbpl) : pick<3, false>(gbpl, dbpl);
+}
+
+}  // namespace
+
+bool decode_geometry_ok(int d, int f) {
+  return pick_kernel(2, true, row_geom(d).bpl, row_geom(f).bpl) != nullptr;
+}
+
+cudaError_t decode_init(const Ctx& ctx) {
+  (void)ctx;
+  const int combos[6][2] = {{2, 3}, {1, 1}, {2, 2}, {2, 1}, {1, 3}, {4, 3}};
+  for (int bits = 2; bits <= 3; ++bits)
+    for (int r = 0; r < 2; ++r)
+      for (const auto& c : combos) {
+        const cudaError_t e = cudaFuncSetAttribute(pick_kernel(bits, r != 0, c[0], c[1]),
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax);
+        if (e != cudaSuccess) return e;
+      }
+  return cudaSuccess;
+}
+
+cudaError_t launch_decode_layer(const Ctx& ctx, const moe_layer_cfg& c, const DecodeArgs& a, cudaStream_t s) {
+  const RowGeom gg = row_geom(c.d), gd = row_geom(c.f);
+  if (a.route && c.E > 512) return cudaErrorNotSupported;  // fused top-k holds 16 logits per lane
+  DLKernel kern = pick_kernel(c.bits, a.route, gg.bpl, gd.bpl);
+  if (kern == nullptr) return cudaErrorNotSupported;
+  const int G = ctx.num_sms;
+  const int CW = consumer_warps(c.bits);
+  const int T = a.T, np = T * c.k;
+  DLParams P{};
+  P.x = a.x;
+  P.T = T;
+  P.d = c.d;
+  P.f = c.f;
+  P.E = c.E;
+  P.k = c.k;
+  P.renorm = c.renorm;
+  P.residual = c.residual;
+  P.has_shared = a.shared != nullptr;
+  P.out_f32 = c.out_fp32;
+  P.wr = a.wr;
+  P.bias = a.bias;
+  P.logits = a.logits;
+  P.idx = a.idx;
+  P.gate = a.gate;
+  P.slot_of = a.slot_of;
+  P.n_slots = a.n_slots;
+  P.g = *a.g;
+  P.pool = a.pool;
+  P.stride = a.stride;
+  P.shared = a.shared;
+  P.lay = a.lay;
+  P.h = a.h;
+  P.y = a.y;
+  P.status = ctx.d_status;
+  P.gbar = ctx.d_gbar;
+  P.timeout_ns = ctx.timeout_ns;
+  P.trace = ctx.d_trace;
+  P.gu_lpr = gg.lpr;
+  P.dn_lpr = gd.lpr;
+  P.gu_row = c.d * c.bits / 8;
+  P.gu_sc = c.d / kBlock * 2;
+  P.dn_row = c.f * c.bits / 8;
+  P.dn_sc = c.f / kBlock * 2;
+  P.gu_chan = CW;
+  // output rows per CTA: a multiple of the smallest row count whose code and
+  // scale bytes are both multiples of 16 (bulk-copy granularity)
+  int gran = 1;
+  while ((gran * P.dn_row) % 16 != 0 || (gran * P.dn_sc) % 16 != 0) gran *= 2;
+  P.rpc = static_cast<int>(align_up((c.d + G - 1) / G, gran));
+  P.wr_rows = (c.E + G - 1) / G;
+  const int n_uniq_max = np < c.E ? np : c.E;
+  const int sh_ch = (c.f + G - 1) / G;
+  P.max_stages = (sh_ch + CW - 1) / CW + 1 +
+                 static_cast<int>((static_cast<long long>(n_uniq_max) * c.f + G - 1) / G + CW - 1) / CW +
+                 n_uniq_max + 2 + n_uniq_max + 2;
+  const size_t qw = c.bits == 3 ? 34 : 18;  // words per quantised block
+  size_t o = align_up(sizeof(DLShared), 128);
+  P.sm_stages = static_cast<int>(o);
+  o = align_up(o + static_cast<size_t>(P.max_stages) * sizeof(StageRec), 128);
+  P.sm_route = static_cast<int>(o);
+  o = align_up(o + (9 * static_cast<size_t>(np) + 1) * 4, 128);
+  P.sm_zs = static_cast<int>(o);
+  o = align_up(o + static_cast<size_t>(np + T) * P.rpc * 4, 128);  // z rows [np + T][rpc]
+  P.sm_xq = static_cast<int>(o);
+  o = align_up(o + static_cast<size_t>(T) * qw * (c.d / kBlock) * 4, 128);
+  P.sm_wr = static_cast<int>(o);
+  if (a.route) o = align_up(o + static_cast<size_t>(P.wr_rows) * c.d * 4, 128);
+  // quantised h rows for the down phase: every row if they fit in 48 KB, else
+  // as many as fit (at least the T rows one expert can have)
+  const int n_rows_all = np + (P.has_shared ? T : 0);
+  const size_t h_row_bytes = qw * (c.f / kBlock) * 4;
+  const int h_cap = static_cast<int>((48 * 1024) / h_row_bytes);
+  P.h_rows = n_rows_all < h_cap ? n_rows_all : (h_cap > T ? h_cap : T);
+  P.sm_hq = static_cast<int>(o);
+  o = align_up(o + static_cast<size_t>(P.h_rows) * h_row_bytes, 128);
+  P.sm_ring = static_cast<int>(o);
+  const long long ring = static_cast<long long>(kSmemMax) - static_cast<long long>(o);
+  const long long gu_stage = 2LL * CW * (P.gu_row + P.gu_sc);
+  const long long dn_stage = static_cast<long long>(P.rpc) * (P.dn_row + P.dn_sc);
+  if (ring < 2 * (gu_stage > dn_stage ? gu_stage : dn_stage)) return cudaErrorNotSupported;
+  P.ring_bytes = static_cast<int>(ring / kStageAlign * kStageAlign);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(G);
+  cfg.blockDim = dim3((CW + 1) * 32);
+  cfg.dynamicSmemBytes = kSmemMax;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, P);
+}
+
+}  // namespace moe

@@ -1,6 +1,7 @@
 // C ABI of libmoe: argument checks, workspace carving and kernel launches.
 // Every compute entry point is asynchronous on the caller's stream and
 // allocates nothing; see include/moe.h for the contract of each call.
+#include <cstdlib>
 #include <new>
 
 #include "moe_internal.cuh"
@@ -89,14 +90,22 @@ static bool aligned(const void* p, size_t a) {
   return (reinterpret_cast<uintptr_t>(p) % a) == 0;
 }
 
-static moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ECUDA; }
+static thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+static moe_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  g_last_cuda_error = e;
+  return MOE_ECUDA;
+}
 
 // Makes the context's device current for this host thread (kernels launch on
 // the runtime's current device).
 static bool use_device(const moe_ctx* ctx) {
   int cur = -1;
-  if (cudaGetDevice(&cur) != cudaSuccess) return false;
-  return cur == ctx->c.device || cudaSetDevice(ctx->c.device) == cudaSuccess;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e == cudaSuccess && cur != ctx->c.device) e = cudaSetDevice(ctx->c.device);
+  if (e != cudaSuccess) g_last_cuda_error = e;
+  return e == cudaSuccess;
 }
 
 static moe_expert_layout layout_of(const moe_layer_cfg& c) {
@@ -174,13 +183,27 @@ static moe_status run_ffn(moe_ctx* ctx, const moe_layer_cfg* cfg, int bits, cons
   a.stride = stride;
   a.shared = cfg->n_shared ? shared : nullptr;
   a.lay = layout_of(*cfg);
-  a.h = reinterpret_cast<float*>(static_cast<char*>(ws) + w.h);
+  a.h = static_cast<char*>(ws) + w.h;
   a.y = y;
   a.status = ctx->c.d_status;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (z_rows == nullptr) {
     if (T > MOE_DECODE_MAX_T || y == nullptr || !aligned(y, 16)) return MOE_EINVAL;
-    return from_cuda(launch_ffn_decode(ctx->c, *cfg, a, s));
+    DecodeArgs d{};
+    d.route = false;
+    d.x = a.x;
+    d.T = T;
+    d.n_slots = 0x7fffffff;
+    d.g = &g;
+    d.pool = pool;
+    d.stride = stride;
+    d.shared = a.shared;
+    d.lay = a.lay;
+    d.h = reinterpret_cast<float*>(a.h);
+    d.y = y;
+    const cudaError_t e = launch_decode_layer(ctx->c, *cfg, d, s);
+    if (e == cudaErrorNotSupported) return MOE_EUNSUPPORTED;
+    return from_cuda(e);
   }
   if (!aligned(z_rows, 16)) return MOE_EINVAL;
   const cudaError_t e = launch_ffn_prefill(ctx->c, *cfg, a, ws, z_rows, s);
@@ -203,11 +226,25 @@ moe_status moe_ctx_create(int device, moe_ctx** out) {
   if (cudaSetDevice(device) != cudaSuccess ||
       cudaDeviceGetAttribute(&ctx->c.num_sms, cudaDevAttrMultiProcessorCount, ctx->c.device) !=
           cudaSuccess ||
-      cudaMalloc(&ctx->c.d_status, 16) != cudaSuccess) {
+      cudaMalloc(&ctx->c.d_status, 64) != cudaSuccess) {
     delete ctx;
     return MOE_ECUDA;
   }
-  if (cudaMemset(ctx->c.d_status, 0, 16) != cudaSuccess || router_init(ctx->c) != cudaSuccess ||
+  ctx->c.d_gbar = reinterpret_cast<unsigned long long*>(ctx->c.d_status + 8);
+  // limit of every device-side wait (default 200 ms): MOE_TIMEOUT_US overrides it
+  if (const char* t = getenv("MOE_TIMEOUT_US")) {
+    const long long us = atoll(t);
+    if (us > 0) ctx->c.timeout_ns = static_cast<unsigned long long>(us) * 1000ull;
+  }
+  if (getenv("MOE_TRACE") != nullptr) {
+    const size_t n = static_cast<size_t>(kTraceCtas) * kTraceSlots * sizeof(unsigned long long);
+    if (cudaMalloc(&ctx->c.d_trace, n) != cudaSuccess || cudaMemset(ctx->c.d_trace, 0, n) != cudaSuccess) {
+      cudaFree(ctx->c.d_status);
+      delete ctx;
+      return MOE_ECUDA;
+    }
+  }
+  if (cudaMemset(ctx->c.d_status, 0, 64) != cudaSuccess || router_init(ctx->c) != cudaSuccess ||
       decode_init(ctx->c) != cudaSuccess || prefill_init(ctx->c) != cudaSuccess) {
     cudaFree(ctx->c.d_status);
     delete ctx;
@@ -220,9 +257,12 @@ moe_status moe_ctx_create(int device, moe_ctx** out) {
 void moe_ctx_destroy(moe_ctx* ctx) {
   if (ctx == nullptr) return;
   use_device(ctx);
+  if (ctx->c.d_trace != nullptr) cudaFree(ctx->c.d_trace);
   cudaFree(ctx->c.d_status);
   delete ctx;
 }
+
+const char* moe_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
 
 const char* moe_status_string(moe_status s) {
   switch (s) {
@@ -246,9 +286,25 @@ moe_status moe_check_device_status(moe_ctx* ctx, moe_stream stream) {
       cudaStreamSynchronize(s) != cudaSuccess)
     return MOE_ECUDA;
   if (h[0] == 0) return MOE_OK;
-  if (cudaMemsetAsync(ctx->c.d_status, 0, 16, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+  // clear the status word and the decode kernel's grid-barrier words (an
+  // interrupted barrier leaves them mid-episode)
+  if (cudaMemsetAsync(ctx->c.d_status, 0, 64, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
     return MOE_ECUDA;
   return h[0] == kDevTimeout ? MOE_ETIMEOUT : MOE_EDEVICE;
+}
+
+moe_status moe_trace_fetch(moe_ctx* ctx, unsigned long long* host, int n, moe_stream stream) {
+  if (ctx == nullptr || host == nullptr || n < 0) return MOE_EINVAL;
+  if (ctx->c.d_trace == nullptr) return MOE_EINVAL;
+  if (!use_device(ctx)) return MOE_ECUDA;
+  const int cap = kTraceCtas * kTraceSlots;
+  const size_t bytes = static_cast<size_t>(n < cap ? n : cap) * sizeof(unsigned long long);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(host, ctx->c.d_trace, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemsetAsync(ctx->c.d_trace, 0, static_cast<size_t>(cap) * sizeof(unsigned long long), s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return from_cuda(cudaGetLastError());
+  return MOE_OK;
 }
 
 moe_status moe_expert_layout_get(const moe_layer_cfg* cfg, moe_expert_layout* out) {
@@ -365,15 +421,40 @@ moe_status moe_layer_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, const void*
   float* logits = reinterpret_cast<float*>(b + w.logits);
   int32_t* idx = reinterpret_cast<int32_t*>(b + w.idx);
   float* gate = reinterpret_cast<float*>(b + w.gate);
+  if (T <= MOE_DECODE_MAX_T && cfg->E <= 512) {
+    // one fused kernel: router, top-k, grouping, experts and combine
+    const GroupPtrs g = group_ptrs(*cfg, T, ws);
+    DecodeArgs d{};
+    d.route = true;
+    d.x = static_cast<const uint16_t*>(x);
+    d.T = T;
+    d.wr = w_router;
+    d.bias = logit_bias;
+    d.logits = logits;
+    d.idx = idx;
+    d.gate = gate;
+    d.slot_of = slot_of;
+    d.n_slots = n_slots;
+    d.g = &g;
+    d.pool = slot_pool;
+    d.stride = slot_stride;
+    d.shared = cfg->n_shared ? shared_expert : nullptr;
+    d.lay = layout_of(*cfg);
+    d.h = reinterpret_cast<float*>(b + w.h);
+    d.y = y;
+    const cudaError_t e = launch_decode_layer(ctx->c, *cfg, d, static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported) return MOE_EUNSUPPORTED;
+    return from_cuda(e);
+  }
   if ((st = moe_router_topk(ctx, cfg, x, w_router, logit_bias, T, logits, idx, gate, stream)) != MOE_OK)
     return st;
   moe_grouping g;
   if ((st = moe_group_tokens(ctx, cfg, idx, gate, T, slot_of, n_slots, ws, ws_bytes, &g, stream)) !=
       MOE_OK)
     return st;
-  if (T <= MOE_DECODE_MAX_T)
-    return run_ffn(ctx, cfg, cfg->bits, x, &g, slot_pool, slot_stride, shared_expert, ws, ws_bytes,
-                   nullptr, y, stream);
+  if (T <= MOE_DECODE_MAX_T)  // E > 512: separate router / grouping kernels, fused expert kernel
+    return run_ffn(ctx, cfg, cfg->bits, x, &g, slot_pool, slot_stride, shared_expert, ws, ws_bytes, nullptr, y,
+                   stream);
   float* z = reinterpret_cast<float*>(b + w.z);
   if ((st = run_ffn(ctx, cfg, cfg->bits, x, &g, slot_pool, slot_stride, shared_expert, ws, ws_bytes, z,
                     nullptr, stream)) != MOE_OK)

@@ -27,8 +27,13 @@ constexpr int kDevTimeout = 3;
 struct Ctx {
   int device = 0;
   int num_sms = 0;
-  int* d_status = nullptr;  // [4] ints: code, detail, spare, spare
+  int* d_status = nullptr;     // [4] ints: code, detail, spare, spare
+  unsigned long long* d_gbar = nullptr;  // grid-barrier arrival counter of the decode kernel
+  unsigned long long timeout_ns = 200ull * 1000 * 1000;  // limit of every device-side wait
+  unsigned long long* d_trace = nullptr;  // phase timestamps (MOE_TRACE), kTraceSlots per CTA
 };
+constexpr int kTraceSlots = 32;
+constexpr int kTraceCtas = 1024;
 
 // ---------------------------------------------------------------- workspace
 
@@ -93,7 +98,30 @@ cudaError_t launch_group(const Ctx& ctx, const moe_layer_cfg& c, const int32_t* 
                          const float* gate, int T, const int32_t* slot_of, int n_slots,
                          const GroupPtrs& g, cudaStream_t s);
 
-// ffn_decode.cu
+// decode_layer.cu
+struct DecodeArgs {
+  bool route;               // true: router + top-k + grouping run inside the kernel
+  const uint16_t* x;        // [T, d] bf16
+  int T;
+  const float* wr;          // route: [E, d]
+  const float* bias;        // route: [T, E] or null
+  float* logits;            // route: [T, E] (workspace)
+  int32_t* idx;             // route: [T, k]
+  float* gate;              // route: [T, k]
+  const int32_t* slot_of;   // route: [E]
+  int n_slots;
+  const GroupPtrs* g;       // grouping (written when route, read otherwise)
+  const uint8_t* pool;
+  size_t stride;
+  const uint8_t* shared;    // record or null
+  moe_expert_layout lay;
+  float* h;                 // fp32 [n_rows, f]
+  void* y;
+};
+cudaError_t launch_decode_layer(const Ctx& ctx, const moe_layer_cfg& c, const DecodeArgs& a, cudaStream_t s);
+bool decode_geometry_ok(int d, int f);
+
+// FFN arguments of the prefill path
 struct FfnArgs {
   const uint16_t* x;        // [T, d] bf16
   int T;
@@ -102,13 +130,10 @@ struct FfnArgs {
   size_t stride;
   const uint8_t* shared;    // record or null
   moe_expert_layout lay;
-  float* h;                 // decode: fp32 [n_rows, f]
+  void* h;
   void* y;
   int* status;
 };
-cudaError_t launch_ffn_decode(const Ctx& ctx, const moe_layer_cfg& c, const FfnArgs& a,
-                              cudaStream_t s);
-bool decode_geometry_ok(int d, int f);
 
 // ffn_prefill.cu
 cudaError_t launch_ffn_prefill(const Ctx& ctx, const moe_layer_cfg& c, const FfnArgs& a,

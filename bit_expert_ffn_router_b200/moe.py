@@ -21,7 +21,10 @@ DECODE_MAX_T = 8
 class MoeError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {status_string(status)} ({status})")
+        msg = f"{what}: {status_string(status)} ({status})"
+        if status == ECUDA:
+            msg += f" [{load_library().moe_last_cuda_error().decode()}]"
+        super().__init__(msg)
 
 
 class _Cfg(ctypes.Structure):
@@ -70,7 +73,9 @@ _SIGS = {
     "moe_ctx_create": (_I, [_I, ctypes.POINTER(ctypes.c_void_p)]),
     "moe_ctx_destroy": (None, [_P]),
     "moe_status_string": (ctypes.c_char_p, [_I]),
+    "moe_last_cuda_error": (ctypes.c_char_p, []),
     "moe_check_device_status": (_I, [_P, _S]),
+    "moe_trace_fetch": (_I, [_P, ctypes.c_void_p, _I, _S]),
     "moe_expert_layout_get": (_I, [ctypes.POINTER(_Cfg), ctypes.POINTER(_Layout)]),
     "moe_workspace_bytes": (_Z, [ctypes.POINTER(_Cfg), _I]),
     "moe_router_topk": (_I, [_P, ctypes.POINTER(_Cfg), _P, _P, _P, _I, _P, _P, _P, _S]),
@@ -199,6 +204,13 @@ class Context:
 
     def check_device_status(self, stream=None) -> int:
         return self.lib.moe_check_device_status(self.h, _stream(stream))
+
+    def trace_fetch(self, n_ctas: int, stream=None):
+        """Phase timestamps of the last decode-layer launches (MOE_TRACE set at creation)."""
+        import numpy as np
+        buf = np.zeros((n_ctas, 32), dtype=np.uint64)
+        _check(self.lib.moe_trace_fetch(self.h, buf.ctypes.data, buf.size, _stream(stream)), "moe_trace_fetch")
+        return buf
 
 
 # ------------------------------------------------------------------ buffers

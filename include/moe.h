@@ -134,10 +134,21 @@ MOE_API moe_status moe_ctx_create(int device, moe_ctx** out);
 MOE_API void moe_ctx_destroy(moe_ctx* ctx);
 MOE_API const char* moe_status_string(moe_status s);
 
+/* Text of the last CUDA runtime error a call on this host thread turned into
+ * MOE_ECUDA ("no error" if none). Diagnostic only. */
+MOE_API const char* moe_last_cuda_error(void);
+
 /* Synchronises `stream`, reads and clears the device status word. Returns
  * MOE_OK, MOE_EDEVICE (bad expert or slot index seen by a kernel) or
  * MOE_ETIMEOUT (a bounded wait ran out). */
 MOE_API moe_status moe_check_device_status(moe_ctx* ctx, moe_stream stream);
+
+/* Diagnostics: when the environment variable MOE_TRACE is set at context
+ * creation, the decode-layer kernel records the global-timer value (ns) at
+ * its phase boundaries, 32 slots per CTA. This copies up to n values (CTA
+ * major) into host memory, synchronising `stream`, and clears the record.
+ * Returns MOE_EINVAL if tracing is off. */
+MOE_API moe_status moe_trace_fetch(moe_ctx* ctx, unsigned long long* host, int n, moe_stream stream);
 
 /* ---- sizes -------------------------------------------------------------- */
 

@@ -49,7 +49,7 @@ def _fp32_logit_cases():
     big = g.integers(-4, 5, size=(300, 512)).astype(np.float32)
     big[:50] = g.standard_normal((50, 512)).astype(np.float32)
     return [(M.TINY, small), (M.FULL, big), (M.FULL.replace(E=1024, k=32), g.standard_normal((33, 1024)).astype(np.float32)),
-            (M.FULL.replace(E=40, k=40), g.integers(0, 3, size=(9, 40)).astype(np.float32))]
+            (M.FULL.replace(E=40, k=32), g.integers(0, 3, size=(9, 40)).astype(np.float32))]
 
 
 @pytest.mark.parametrize("case", range(4))
@@ -232,3 +232,24 @@ def test_host_argument_errors():
     assert c.layer_forward_status(**{**args, "x": dv["x"].view(torch.uint8)[2:]}) == M.EINVAL  # misaligned
     assert c.layer_forward_status(**{**args, "shared": None}) == M.EINVAL
     assert c.check_device_status() == M.OK
+
+
+def test_device_wait_timeout_is_reported_and_context_recovers(monkeypatch):
+    """A 1 us wait limit makes the decode kernel's waits run out: the call
+    reports MOE_ETIMEOUT through the status word, and the context (after
+    moe_check_device_status clears it) computes correct results again."""
+    L = H.Layer(M.FULL, 1, seed=70, zipf=True)
+    dv = L.device()
+    monkeypatch.setenv("MOE_TIMEOUT_US", "1")
+    short = M.Context(torch.cuda.current_device())
+    monkeypatch.delenv("MOE_TIMEOUT_US")
+    ws = M.workspace(M.FULL, 1)
+    y = L.out_tensor()
+    st = short.layer_forward_status(M.FULL, dv["x"], 1, dv["wr"], dv["bias"], dv["slot_of"], L.n_slots, dv["pool"],
+                                    dv["stride"], dv["shared"], ws, y)
+    assert st == M.OK  # the launch itself is fine
+    assert short.check_device_status() == M.ETIMEOUT
+    assert short.check_device_status() == M.OK
+    short.close()
+    y2, _ = L.forward()
+    H.assert_close_rows(H.y_as_f64(y2), L.oracle()["y"])
