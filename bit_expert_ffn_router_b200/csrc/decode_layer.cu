@@ -177,6 +177,30 @@ __device__ int push_dn(StageRec* st, int n, int u, int r0, int r1, const DLParam
   return n;
 }
 
+// Routed stage list: this CTA's share of the nu*f routed gate/up channels,
+// then the down slices: routed experts in order, shared last, so that the h
+// rows they read are one ascending range. Stages [0, n_sh) (the shared
+// expert's gate/up) are already in place.
+__device__ void build_routed_list(StageRec* st, DLShared* S, int n_sh, int nu, int b, int G, int r0, int r1,
+                                  const DLParams& P) {
+  int n = n_sh;
+  const long long tot = static_cast<long long>(nu) * P.f;
+  long long c = tot * b / G;
+  const long long c1 = tot * (b + 1) / G;
+  while (c < c1) {
+    const int u = static_cast<int>(c / P.f);
+    const long long ub = static_cast<long long>(u) * P.f;
+    const int ce = static_cast<int>(min(c1, ub + P.f) - ub);
+    n = push_gu(st, n, u, static_cast<int>(c - ub), ce, P);
+    c = ub + ce;
+  }
+  S->n_gu = n;
+  for (int u = 0; u < nu; ++u) n = push_dn(st, n, u, r0, r1, P);
+  if (P.has_shared) n = push_dn(st, n, kShared, r0, r1, P);
+  S->n_st = n;
+  S->n_uniq = nu;
+}
+
 // ------------------------------------------------------------------ producer
 struct Ring {
   int head;       // end of the newest live stage
@@ -208,13 +232,16 @@ __device__ bool ring_pop(DLShared* S, StageRec* st, Ring& rg, uint64_t deadline)
   return true;
 }
 
-__device__ bool ring_issue(DLShared* S, StageRec* st, Ring& rg, int i, uint8_t* ring, int cap,
-                           const DLParams& P, const RouteSmem& R, uint64_t deadline) {
+// Reserves ring space for stage i (the producer's lane 0), freeing older
+// stages as needed but never one at index >= pop_limit (reserved in the
+// current batch, not issued yet). Returns 1 on success, 2 if the stage must
+// wait for the next batch, 0 on timeout or abort.
+__device__ int ring_alloc(DLShared* S, StageRec* st, Ring& rg, int i, int cap, int pop_limit, uint64_t deadline) {
   StageRec& s = st[i];
   const int need = (s.bytes + kStageAlign - 1) / kStageAlign * kStageAlign;
   int start = -1;
   while (true) {
-    if (aborted(S)) return false;
+    if (aborted(S)) return 0;
     if (rg.tail == rg.issued) {
       rg.head = 0;
       start = 0;
@@ -230,55 +257,54 @@ __device__ bool ring_issue(DLShared* S, StageRec* st, Ring& rg, int i, uint8_t* 
         break;
       }
     }
-    if (!ring_pop(S, st, rg, deadline)) return false;
+    if (rg.tail >= pop_limit) return 2;
+    if (!ring_pop(S, st, rg, deadline)) return 0;
   }
   s.off = start;
   rg.head = start + need;
+  rg.issued = i + 1;
+  return 1;
+}
+
+// Arms stage i's mbarrier and issues its two bulk copies (codes, scales).
+// Any lane may issue any reserved stage: copies issued from several lanes
+// at once overlap their issue latency.
+__device__ void stage_issue(DLShared* S, const StageRec& s, int i, uint8_t* ring, const DLParams& P,
+                            const RouteSmem& R) {
   const uint8_t* rec = expert_record(P, R, s.u);
-  uint8_t* dst = ring + start;
+  uint8_t* dst = ring + s.off;
   uint64_t* bar = &S->full[i % kNB];
   mbar_arrive_expect_tx(bar, static_cast<uint32_t>(s.bytes));
-  if (s.type == kStGU) {
-    const int rows = 2 * (s.b - s.a);
-    const int row_b = s.code_bytes / rows;
-    const int sc_b = (s.bytes - s.code_bytes) / rows;
-    bulk_g2s(dst, rec + P.lay.gu_codes + static_cast<size_t>(2 * s.a) * row_b, s.code_bytes, bar);
-    bulk_g2s(dst + s.code_bytes, rec + P.lay.gu_scales + static_cast<size_t>(2 * s.a) * sc_b,
-             s.bytes - s.code_bytes, bar);
-  } else {
-    const int rows = s.b - s.a;
-    const int row_b = s.code_bytes / rows;
-    const int sc_b = (s.bytes - s.code_bytes) / rows;
-    bulk_g2s(dst, rec + P.lay.dn_codes + static_cast<size_t>(s.a) * row_b, s.code_bytes, bar);
-    bulk_g2s(dst + s.code_bytes, rec + P.lay.dn_scales + static_cast<size_t>(s.a) * sc_b,
-             s.bytes - s.code_bytes, bar);
-  }
-  rg.issued = i + 1;
-  return true;
+  const int rows = s.type == kStGU ? 2 * (s.b - s.a) : s.b - s.a;
+  const int first = s.type == kStGU ? 2 * s.a : s.a;
+  const int row_b = s.code_bytes / rows;
+  const int sc_b = (s.bytes - s.code_bytes) / rows;
+  const size_t oc = s.type == kStGU ? P.lay.gu_codes : P.lay.dn_codes;
+  const size_t os = s.type == kStGU ? P.lay.gu_scales : P.lay.dn_scales;
+  bulk_g2s(dst, rec + oc + static_cast<size_t>(first) * row_b, s.code_bytes, bar);
+  bulk_g2s(dst + s.code_bytes, rec + os + static_cast<size_t>(first) * sc_b, s.bytes - s.code_bytes, bar);
 }
 
 // ------------------------------------------------------------------ consumers
-// Quantises the T token rows of x (bf16, global) into the gate/up layout.
+// Quantises the T token rows of x (bf16, global) into the gate/up layout,
+// four lanes per 32-value block. Loops run in whole warps (shuffles).
 template <int BITS>
 __device__ void quantise_x(const DLParams& P, int* xq, int nct) {
   const int nb = P.d / kBlock, bpl = nb / P.gu_lpr;
   const int words = QV<BITS>::kWords * nb;
-  for (int job = threadIdx.x; job < P.T * nb; job += nct) {
-    const int t = job / nb, blk = job % nb;
-    const uint4* src = reinterpret_cast<const uint4*>(P.x + static_cast<size_t>(t) * P.d + blk * kBlock);
-    float v[32];
+  const int jobs = P.T * nb;
+  const int q = threadIdx.x & 3;
+#pragma unroll 1
+  for (int base = threadIdx.x & ~31; base < jobs * 4; base += nct) {
+    const int job = (base + (threadIdx.x & 31)) >> 2;
+    const bool live = job < jobs;
+    const int t = live ? job / nb : 0, blk = live ? job % nb : 0;
+    const uint16_t* src = P.x + static_cast<size_t>(t) * P.d + blk * kBlock + q;
+    float v[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 q = __ldcg(src + i);
-      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
-        v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
-      }
-    }
+    for (int k = 0; k < 8; ++k) v[k] = live ? bf16_bits_to_float(__ldcg(src + 4 * k)) : 0.f;
     const int gl = blk / bpl, bb = blk % bpl;
-    quant_block<BITS>(v, xq + t * words, nb, bb * P.gu_lpr + gl);
+    quant_quad<BITS>(v, xq + t * words, nb, bb * P.gu_lpr + gl, q, live);
   }
 }
 
@@ -287,20 +313,19 @@ template <int BITS>
 __device__ void quantise_h(const DLParams& P, int lo, int hi, int* hq, int nct) {
   const int nb = P.f / kBlock, bpl = nb / P.dn_lpr;
   const int words = QV<BITS>::kWords * nb;
-  for (int job = threadIdx.x; job < (hi - lo) * nb; job += nct) {
-    const int r = job / nb, blk = job % nb;
-    const float4* src = reinterpret_cast<const float4*>(P.h + static_cast<size_t>(lo + r) * P.f + blk * kBlock);
-    float v[32];
+  const int jobs = (hi - lo) * nb;
+  const int q = threadIdx.x & 3;
+#pragma unroll 1
+  for (int base = threadIdx.x & ~31; base < jobs * 4; base += nct) {
+    const int job = (base + (threadIdx.x & 31)) >> 2;
+    const bool live = job < jobs;
+    const int r = live ? job / nb : 0, blk = live ? job % nb : 0;
+    const float* src = P.h + static_cast<size_t>(lo + r) * P.f + blk * kBlock + q;
+    float v[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 q = __ldcg(src + i);
-      v[4 * i] = q.x;
-      v[4 * i + 1] = q.y;
-      v[4 * i + 2] = q.z;
-      v[4 * i + 3] = q.w;
-    }
+    for (int k = 0; k < 8; ++k) v[k] = live ? __ldcg(src + 4 * k) : 0.f;
     const int gl = blk / bpl, bb = blk % bpl;
-    quant_block<BITS>(v, hq + r * words, nb, bb * P.dn_lpr + gl);
+    quant_quad<BITS>(v, hq + r * words, nb, bb * P.dn_lpr + gl, q, live);
   }
 }
 
@@ -597,10 +622,11 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
 
   if (warp == CW) {
     // ------------------------------------------------------------ producer
-    if (lane != 0) return;
+    // lane 0 reserves ring space for up to 32 stages at a time, then every
+    // lane issues one reserved stage
     Ring rg{0, 0, 0};
     bool ok = true, wr_issued = false;
-    if (ROUTE && e1 > e0) {
+    if (ROUTE && e1 > e0 && lane == 0) {
       const uint32_t bytes = static_cast<uint32_t>((e1 - e0) * P.d * 4);
       mbar_arrive_expect_tx(&S->wr_bar, bytes);
       bulk_g2s(wrs, P.wr + static_cast<size_t>(e0) * P.d, bytes, &S->wr_bar);
@@ -608,26 +634,81 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
     }
     const int n_sh = S->n_sh;
     int n_st = n_sh;
-    for (int i = 0; ok; ++i) {
-      if (i == n_sh) {
-        if (!mbar_wait(&S->list_bar, 0, deadline)) {
+    if (!ROUTE) {
+      // the grouping is already in global memory (written by an earlier
+      // kernel): build the whole stage list now and stream every row at once
+      grid_dep_wait();
+      const int np = P.T * P.k;
+      const int nu = min(max(__ldcg(P.g.n_uniq), 0), min(np, P.E));
+      for (int u = lane; u < nu; u += 32) {
+        int slot = __ldcg(P.g.uniq_slot + u);
+        if (slot < 0 || slot >= P.n_slots) {
+          report(P.status, kDevBadSlot, u);
+          slot = 0;
+        }
+        R.uniq_slot[u] = slot;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        build_routed_list(st, S, n_sh, nu, b, G, r0, r1, P);
+        mbar_arrive(&S->list_bar);
+      }
+      __syncwarp();
+    }
+    bool listed = !ROUTE;
+    int i = 0;
+    while (ok) {
+      if (i == n_sh && !listed) {
+        int got = 1;
+        if (lane == 0) got = mbar_wait(&S->list_bar, 0, deadline) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) {
           ok = false;
           break;
         }
-        MOE_TRACE(12)
-        n_st = S->n_st;
+        listed = true;
+        if (lane == 0) MOE_TRACE(12)
       }
-      if (i >= n_st) break;
-      ok = ring_issue(S, st, rg, i, ring, P.ring_bytes, P, R, deadline);
+      if (listed) n_st = S->n_st;
+      const int end = listed ? n_st : n_sh;
+      if (i >= end) {
+        if (listed) break;
+        continue;
+      }
+      int batch = 0, okl = 1;
+      if (lane == 0) {
+        const int want = min(32, end - i);
+        while (batch < want) {
+          const int r = ring_alloc(S, st, rg, i + batch, P.ring_bytes, i, deadline);
+          if (r == 0) okl = 0;
+          if (r != 1) break;
+          ++batch;
+        }
+      }
+      okl = __shfl_sync(0xffffffffu, okl, 0);
+      batch = __shfl_sync(0xffffffffu, batch, 0);
+      if (!okl) {
+        ok = false;
+        break;
+      }
+      __syncwarp();
+      if (lane < batch) stage_issue(S, st[i + lane], i + lane, ring, P, R);
+      __syncwarp();
+      i += batch;
     }
-    MOE_TRACE(13)
+    if (lane == 0) MOE_TRACE(13)
     if (!ok) {
-      if (!aborted(S)) set_abort(S, P.status, 10);
-      // every issued copy must land before the CTA may exit; copies finish
-      // in microseconds, the 100 ms bound only guards against the impossible
-      const uint64_t d2 = global_timer_ns() + 100000000ull;
-      for (int j = rg.tail; j < rg.issued; ++j) mbar_wait(&S->full[j % kNB], (j / kNB) & 1, d2);
-      if (wr_issued) mbar_wait(&S->wr_bar, 0, d2);
+      // stages below i were issued (those reserved in a failed batch were not)
+      rg.tail = __shfl_sync(0xffffffffu, rg.tail, 0);
+      rg.issued = i;
+      if (lane == 0) {
+        if (!aborted(S)) set_abort(S, P.status, 10);
+        // every issued copy must land before the CTA may exit; copies finish
+        // in microseconds, the 100 ms bound only guards against the impossible
+        const uint64_t d2 = global_timer_ns() + 100000000ull;
+        for (int j = rg.tail; j < rg.issued; ++j) mbar_wait(&S->full[j % kNB], (j / kNB) & 1, d2);
+        if (wr_issued) mbar_wait(&S->wr_bar, 0, d2);
+      }
     }
     return;
   }
@@ -673,47 +754,19 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
         group_in_smem(P, R, S, np, CT);
         if (b == 0) publish_grouping(P, R, S->n_uniq, np, CT);
       } else {
-        // grouping written by moe_group_tokens
-        const int nu = min(max(__ldcg(P.g.n_uniq), 0), min(np, P.E));
+        // grouping written by moe_group_tokens; the producer has read the
+        // slots and built the stage list
+        const int nu_g = min(max(__ldcg(P.g.n_uniq), 0), min(np, P.E));
         for (int p = tid; p < np; p += CT) {
           R.pair_token[p] = min(max(__ldcg(P.g.pair_token + p), 0), P.T - 1);
           R.pair_gate[p] = __ldcg(P.g.pair_gate + p);
           R.pair_pos[p] = min(max(__ldcg(P.g.pair_pos + p), 0), np - 1);
         }
-        for (int u = tid; u <= nu; u += CT) {
-          R.uniq_off[u] = min(max(__ldcg(P.g.uniq_offset + u), 0), np);
-          if (u < nu) {
-            int slot = __ldcg(P.g.uniq_slot + u);
-            if (slot < 0 || slot >= P.n_slots) {
-              report(P.status, kDevBadSlot, u);
-              slot = 0;
-            }
-            R.uniq_slot[u] = slot;
-          }
-        }
-        if (tid == 0) S->n_uniq = nu;
-        named_sync(1, CT);
+        for (int u = tid; u <= nu_g; u += CT) R.uniq_off[u] = min(max(__ldcg(P.g.uniq_offset + u), 0), np);
+        if (!mbar_wait_warp(&S->list_bar, 0, deadline)) set_abort(S, P.status, 7);
       }
-      // routed stage list: this CTA's share of the n_uniq*f routed gate/up
-      // channels, then the down slices: routed experts in order, shared last,
-      // so that the h rows they read are one ascending range
-      if (tid == 0) {
-        const int nu = S->n_uniq;
-        int n = n_sh;
-        const long long tot = static_cast<long long>(nu) * P.f;
-        long long c = tot * b / G;
-        const long long c1 = tot * (b + 1) / G;
-        while (c < c1) {
-          const int u = static_cast<int>(c / P.f);
-          const long long ub = static_cast<long long>(u) * P.f;
-          const int ce = static_cast<int>(min(c1, ub + P.f) - ub);
-          n = push_gu(st, n, u, static_cast<int>(c - ub), ce, P);
-          c = ub + ce;
-        }
-        S->n_gu = n;
-        for (int u = 0; u < nu; ++u) n = push_dn(st, n, u, r0, r1, P);
-        if (P.has_shared) n = push_dn(st, n, kShared, r0, r1, P);
-        S->n_st = n;
+      if (ROUTE && tid == 0) {
+        build_routed_list(st, S, n_sh, S->n_uniq, b, G, r0, r1, P);
         mbar_arrive(&S->list_bar);
       }
       named_sync(1, CT);
@@ -758,13 +811,18 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
     }
     quantise_h<BITS>(P, h_lo, h_hi, hq, CT);
     named_sync(1, CT);
+    if (tid == 0) MOE_TRACE(24)
 #pragma unroll 1
     for (int i = i0; i < i1; ++i) {
       if (!aborted(S) && (i - n_gu) % CW == warp) {
-        if (mbar_wait_warp(&S->full[i % kNB], (i / kNB) & 1, deadline))
+        if (trace != nullptr && warp == 1 && lane == 0) trace[25] = global_timer_ns();
+        const bool got = mbar_wait_warp(&S->full[i % kNB], (i / kNB) & 1, deadline);
+        if (trace != nullptr && warp == 1 && lane == 0) trace[26] = global_timer_ns();
+        if (got)
           process_dn<BITS, DBPL>(st[i], ring, P, R, np, hq, h_lo, zs);
         else
           set_abort(S, P.status, 6);
+        if (trace != nullptr && warp == 1 && lane == 0) trace[27] = global_timer_ns();
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&S->empty[i % kNB]);

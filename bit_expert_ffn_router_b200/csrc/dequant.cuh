@@ -89,6 +89,46 @@ __device__ __forceinline__ void quant_block(const float* v, int* vec, int nb, in
   vec[(QV<BITS>::kSX + 1) * nb + col] = sum;
 }
 
+// The same, spread over an aligned group of 4 lanes: lane q of the group
+// holds v[k] = block value q + 4k (k = 0..7). Every int16 pair a lane stores
+// is made of its own values; the block max and sum come from 2 shuffles.
+// All 32 lanes of the warp must call it (dummy groups pass zeros).
+template <int BITS>
+__device__ __forceinline__ void quant_quad(const float* v, int* vec, int nb, int col, int q, bool store) {
+  float m = fmaxf(fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))),
+                  fmaxf(fmaxf(fabsf(v[4]), fabsf(v[5])), fmaxf(fabsf(v[6]), fabsf(v[7]))));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  const float inv = m > 0.f ? 32767.f / m : 0.f;
+  constexpr float kMagic = 12582912.f;  // 1.5 * 2^23
+  int r[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) r[k] = __float_as_int(fmaf(v[k], inv, kMagic));
+  unsigned us = (static_cast<unsigned>(r[0]) + static_cast<unsigned>(r[1])) +
+                (static_cast<unsigned>(r[2]) + static_cast<unsigned>(r[3])) +
+                ((static_cast<unsigned>(r[4]) + static_cast<unsigned>(r[5])) +
+                 (static_cast<unsigned>(r[6]) + static_cast<unsigned>(r[7])));
+  us += __shfl_xor_sync(0xffffffffu, us, 1);
+  us += __shfl_xor_sync(0xffffffffu, us, 2);
+  if (!store) return;
+  // words j = 0, 1: values (16j+q, 16j+q+4) and (16j+q+8, 16j+q+12)
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    vec[(8 * j + q) * nb + col] = static_cast<int>(__byte_perm(r[4 * j], r[4 * j + 1], 0x5410));
+    vec[(8 * j + 4 + q) * nb + col] = static_cast<int>(__byte_perm(r[4 * j + 2], r[4 * j + 3], 0x5410));
+  }
+  if (BITS == 3) {  // high-plane pairs (t, t+8), (t+16, t+24) for t = q, q+4
+    vec[(16 + q) * nb + col] = static_cast<int>(__byte_perm(r[0], r[2], 0x5410));
+    vec[(16 + q + 4) * nb + col] = static_cast<int>(__byte_perm(r[1], r[3], 0x5410));
+    vec[(24 + q) * nb + col] = static_cast<int>(__byte_perm(r[4], r[6], 0x5410));
+    vec[(24 + q + 4) * nb + col] = static_cast<int>(__byte_perm(r[5], r[7], 0x5410));
+  }
+  if (q == 0) {
+    vec[QV<BITS>::kSX * nb + col] = __float_as_int(m * (1.f / 32767.f));
+    vec[(QV<BITS>::kSX + 1) * nb + col] = static_cast<int>(us - 32u * 0x4B400000u);
+  }
+}
+
 // One block of a quantised vector, in registers.
 template <int BITS>
 struct XR {
