@@ -12,7 +12,8 @@ One step = one pass of all 48 layers; the 48 layers' weights (~1 GB touched
 per step) do not fit in the 126 MB L2, so every layer reads its weights from
 HBM.
 
---workload prefill: one layer at T=8192 (81,920 token-expert pairs).
+--workload prefill: one full-size layer at T=8192 (81,920 token-expert pairs,
+Zipf-skewed over 512 experts), the prefill chunk of the pages.
 
 Prints one JSON line (rank 0). --impl reference times the fp64 CPU oracle on
 a bounded sample of the same workload instead.
@@ -236,6 +237,181 @@ class DecodeStack:
         return float(np.mean(ms)), float(np.mean(bytes_))
 
 
+KERNELS_PER_LAYER_PREFILL = 9  # router GEMM, top-k, 3 grouping, x gather, 2 grouped GEMMs, combine
+
+
+class PrefillLayer:
+    """One full-size layer at T tokens (prefill chunk): 512 experts in a slot
+    pool behind a shuffled slot table, Zipf routing, bf16 output."""
+
+    def __init__(self, T=8192, bits=2, seed=SEED):
+        import torch
+        from bit_expert_ffn_router_b200 import moe as M
+        from bit_expert_ffn_router_b200 import synth
+        self.M, self.torch = M, torch
+        self.T = T
+        self.cfg = M.FULL.replace(bits=bits, out_fp32=0)
+        cfg = self.cfg
+        self.lay = M.expert_layout(cfg)
+        self.stride = self.lay["bytes"]
+        self.n_slots = cfg.E
+        dev = "cuda"
+        self.pool = torch.empty(self.n_slots, self.stride, dtype=torch.uint8, device=dev)
+        synth.fill_random_bytes_(self.pool, seed + 21)
+        self.shared = torch.empty(1, self.stride, dtype=torch.uint8, device=dev)
+        synth.fill_random_bytes_(self.shared, seed + 22)
+        for name, seedoff in (("gu_scales", 23), ("dn_scales", 24)):
+            lo = self.lay[name]
+            n = (2 * cfg.f * (cfg.d // 32) if name == "gu_scales" else cfg.d * (cfg.f // 32)) * 2
+            synth.fill_scales_(self.pool[:, lo:lo + n], seed + seedoff)
+            synth.fill_scales_(self.shared[:, lo:lo + n], seed + seedoff + 1)
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed + 25)
+        self.wr = torch.randn(cfg.E, cfg.d, generator=g, device=dev) * 0.02
+        self.slot_of = torch.from_numpy(synth.rng(seed + 26).permutation(cfg.E).astype(np.int32)).to(dev)
+        self.sets = synth.zipf_sets(T, cfg.E, cfg.k, seed)
+        self.bias = torch.from_numpy(synth.bias_from_sets(self.sets, cfg.E)).to(dev)
+        self.x_host = synth.activations(T, cfg.d, seed + 27)
+        self.x = torch.from_numpy(self.x_host.view(np.int16)).to(dev).view(torch.bfloat16)
+        self.y = torch.empty(T, cfg.d, dtype=torch.bfloat16, device=dev)
+        self.ws = M.workspace(cfg, T)
+        self.ctx = M.Context(torch.cuda.current_device())
+        counts = np.bincount(np.asarray(self.sets).reshape(-1), minlength=cfg.E)
+        self.load = {"max": int(counts.max()), "median": float(np.median(counts)), "min": int(counts.min()),
+                     "experts_lt16": int((counts < 16).sum()), "experts_ge128": int((counts >= 128).sum())}
+        self.flops = 6 * cfg.d * cfg.f * (T * cfg.k + T * cfg.n_shared)
+        self.graph = None
+
+    def step(self):
+        self.ctx.layer_forward(self.cfg, self.x, self.T, self.wr, self.bias, self.slot_of, self.n_slots, self.pool,
+                               self.stride, self.shared[0], self.ws, self.y)
+        return self.y
+
+    def capture(self):
+        torch = self.torch
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.step()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.step()
+        torch.cuda.synchronize()
+
+    def time_parts(self, reps=5):
+        """CUDA-event time of each entry point of the unfused path (ms)."""
+        torch, M, cfg, T = self.torch, self.M, self.cfg, self.T
+        st = torch.cuda.current_stream()
+        logits = torch.empty(T, cfg.E, device="cuda")
+        idx = torch.empty(T, cfg.k, dtype=torch.int32, device="cuda")
+        gate = torch.empty(T, cfg.k, device="cuda")
+        ws = M.workspace(cfg, T)
+        z = torch.empty(T * cfg.k + T, cfg.d, device="cuda")
+        parts = {"router_topk": [], "group": [], "expert_ffn": [], "combine": []}
+        g = None
+        for r in range(reps + 1):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            ev[0].record(st)
+            self.ctx.router_topk(cfg, self.x, self.wr, self.bias, T, logits, idx, gate)
+            ev[1].record(st)
+            g = self.ctx.group_tokens(cfg, idx, gate, T, self.slot_of, self.n_slots, ws)
+            ev[2].record(st)
+            self.ctx.expert_ffn(cfg, self.x, g, self.pool, self.stride, self.shared[0], ws, z_rows=z)
+            ev[3].record(st)
+            self.ctx.combine(cfg, g, z, self.x, T, self.y)
+            ev[4].record(st)
+            torch.cuda.synchronize()
+            if r > 0:
+                for i, k in enumerate(parts):
+                    parts[k].append(ev[i].elapsed_time(ev[i + 1]))
+        return {k: float(np.median(v)) for k, v in parts.items()}
+
+
+def run_prefill(args):
+    import torch
+    world, rank, local = dist_setup()
+    hbm, tf, tf_s, peak_kind = peaks()
+    pl = PrefillLayer(T=args.tokens if args.tokens > 8 else 8192, bits=args.bits)
+    pl.capture()
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        pl.graph.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            pl.graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_max = allreduce_max(e0.elapsed_time(e1), world)
+    ms_step = ms_max / args.steps
+    value = pl.T * args.steps * world / (ms_max / 1e3)
+
+    parts = pl.time_parts()
+    ffn_ms = parts["expert_ffn"]
+    achieved = pl.flops / (ffn_ms / 1e3) / 1e12
+
+    xh = torch.from_numpy(pl.x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    for _ in range(2):
+        pl.x.copy_(xh, non_blocking=True)
+        yh.copy_(pl.step(), non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, args.steps // 4)
+    e2.record(stream)
+    for _ in range(n_e2e):
+        pl.x.copy_(xh, non_blocking=True)
+        yh.copy_(pl.step(), non_blocking=True)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = allreduce_max(e2.elapsed_time(e3), world)
+    e2e_value = pl.T * n_e2e * world / (e2e_ms / 1e3)
+
+    res = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": f"tokens/s (one MoE layer, prefill chunk T={pl.T})",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": f"u{args.bits} codes -> f16 x f16 tcgen05, f32 accumulate",
+        "data": "synthetic (seeded; random-init weights of the stated shapes)",
+        "config": {
+            "workload": f"prefill layer d=2048 f=768 E=512 top-10 + 1 shared, T={pl.T} "
+                        f"({pl.T * pl.cfg.k} pairs), {args.bits}-bit block-32 fp16-scale, Zipf(1.1) routing",
+            "global_batch": pl.T * world, "seq_len": pl.T, "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (0.76-1.06 GB of expert weights per layer)",
+            "expert_load": pl.load, "parts_ms": {k: round(v, 4) for k, v in parts.items()},
+            "useful_gflop": round(pl.flops / 1e9, 1),
+        },
+        "roofline": {
+            "kernel": "prefill expert FFN (x gather + gate/up and down tcgen05 grouped GEMMs), useful FLOPs",
+            "bound": "tensor", "achieved": round(achieved, 1), "peak": tf, "unit": "TFLOP/s",
+            "frac": round(achieved / tf, 4), "peak_source": f"{peak_kind} bf16 burst (fp16 has the same dense rate)",
+            "traffic": None, "avg_launch_us": round(ffn_ms * 1e3, 2), "flops_per_launch": pl.flops,
+        },
+        "e2e": {"value": round(e2e_value, 1), "unit": f"tokens/s (one MoE layer, prefill chunk T={pl.T})",
+                "h2d_bytes_per_step": pl.T * pl.cfg.d * 2, "d2h_bytes_per_step": pl.T * pl.cfg.d * 2,
+                "how": "pinned host x -> moe_layer_forward -> pinned host y (bf16), CUDA events"},
+        "gpu_launches": KERNELS_PER_LAYER_PREFILL * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline_prefill(pl, args.cpu_tokens)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_setup()
@@ -372,12 +548,40 @@ def cpu_baseline(st, n_layers):
             "sample": f"{n_layers} of 48 layers at T={st.T} (fp64 numpy oracle, {dt:.1f} s), scaled to 48 layers"}
 
 
+def prefill_oracle_inputs(pl, tokens):
+    cfg = pl.cfg
+    sel = np.unique(np.asarray(pl.sets)[tokens].reshape(-1))
+    slot_of = pl.slot_of.cpu().numpy()
+    recs = {int(e): pl.pool[int(slot_of[e])].cpu().numpy() for e in sel}
+    return (pl.x_host[tokens], pl.wr.cpu().numpy(), pl.bias.cpu().numpy()[tokens], recs,
+            pl.shared[0].cpu().numpy())
+
+
+def cpu_baseline_prefill(pl, n_tokens):
+    """The fp64 oracle, as it stands, on the first n_tokens of the chunk."""
+    from oracle import moe_oracle as O
+    import threadpoolctl
+    cfg = pl.cfg
+    x, wr, bias, recs, shared = prefill_oracle_inputs(pl, np.arange(n_tokens))
+    t0 = time.perf_counter()
+    cache = O.ExpertCache(lambda e: O.sections_from_record(recs[e], cfg.d, cfg.f, cfg.bits), cfg.d, cfg.f, cfg.bits)
+    sh = O.expert_weights(O.sections_from_record(shared, cfg.d, cfg.f, cfg.bits), cfg.d, cfg.f, cfg.bits)
+    O.layer_forward(x, wr, cfg.k, cache, sh, bias=bias)
+    dt = time.perf_counter() - t0
+    cores = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
+    return {"value": round(n_tokens / dt, 3), "unit": f"tokens/s (one MoE layer, prefill chunk T={pl.T})",
+            "cores": cores, "kind": "oracle",
+            "sample": f"first {n_tokens} of {pl.T} tokens of the chunk (fp64 numpy oracle, {dt:.1f} s)"}
+
+
 def run_reference(args):
     """The oracle as the reference arm: rank 0 only, a bounded sample per step."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    if args.workload == "prefill":
+        return run_reference_prefill(args, world)
     from oracle import moe_oracle as O
     from bit_expert_ffn_router_b200 import synth
     import threadpoolctl
@@ -422,6 +626,43 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_reference_prefill(args, world):
+    """Reference arm of the prefill workload: the oracle on a bounded token sample per step."""
+    from oracle import moe_oracle as O
+    from bit_expert_ffn_router_b200 import synth
+    import threadpoolctl
+    d, f, E, k, bits, T = 2048, 768, 512, 10, args.bits, 8192
+    n = 4  # tokens per step: keeps --steps 50 --warmup 5 within a few minutes
+    sets = synth.zipf_sets(T, E, k, SEED)[:n]
+    bias = synth.bias_from_sets(sets, E)
+    wr = synth.router_weights(E, d, SEED + 1)
+    x = synth.activations(T, d, SEED + 27)[:n]
+    sel = np.unique(np.asarray(sets).reshape(-1))
+    secs = {int(e): synth.expert_sections(d, f, bits, SEED + 100 + int(e)) for e in sel}
+    shared = synth.expert_sections(d, f, bits, SEED + 99)
+    times = []
+    for step in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        cache = O.ExpertCache(lambda e: secs[e], d, f, bits)
+        O.layer_forward(x, wr, k, cache, O.expert_weights(shared, d, f, bits), bias=bias)
+        if step >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    value = n / float(np.mean(times))
+    cores = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
+    unit = f"tokens/s (one MoE layer, prefill chunk T={T})"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(float(np.mean(times)) * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"prefill layer d=2048 f=768 E=512 top-10 + 1 shared, T={T}, {bits}-bit "
+                               f"(oracle on {n} tokens per step)", "global_batch": n, "seq_len": T,
+                   "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 3), "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": f"{n} of {T} tokens per step"},
+        "e2e": {"value": round(value, 3), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -432,11 +673,15 @@ def main():
     ap.add_argument("--bits", type=int, default=2)
     ap.add_argument("--cpu-layers", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"])
+    ap.add_argument("--cpu-tokens", type=int, default=32, help="prefill: oracle sample size")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "prefill":
+        run_prefill(args)
     else:
         run_ours(args)
 

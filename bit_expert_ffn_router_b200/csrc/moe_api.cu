@@ -48,7 +48,8 @@ WsLayout ws_layout(const moe_layer_cfg& c, int T) {
   const size_t h16 = (static_cast<size_t>(w.n_rows) + kTileN) * c.f * 2;
   w.h = take(h32 > h16 ? h32 : h16);
   w.z = take(T > MOE_DECODE_MAX_T ? static_cast<size_t>(w.n_rows) * c.d * 4 : 0);
-  w.x16 = take(T > MOE_DECODE_MAX_T ? Tz * c.d * 2 : 0);
+  // x gathered into pair order as fp16 (prefill grouped GEMM operand)
+  w.x16 = take(static_cast<size_t>(w.n_rows) * c.d * 2);
   w.total = o;
   return w;
 }

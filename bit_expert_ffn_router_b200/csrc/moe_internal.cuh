@@ -139,6 +139,7 @@ struct FfnArgs {
 cudaError_t launch_ffn_prefill(const Ctx& ctx, const moe_layer_cfg& c, const FfnArgs& a,
                                void* ws, float* z_rows, cudaStream_t s);
 cudaError_t prefill_init(const Ctx& ctx);
+bool prefill_geometry_ok(int d, int f);
 
 // combine.cu
 cudaError_t launch_combine(const Ctx& ctx, const moe_layer_cfg& c, const int32_t* pair_pos,
