@@ -166,7 +166,8 @@ class DecodeStack:
         g = torch.Generator(device=dev)
         g.manual_seed(seed + 15)
         self.wr = torch.randn(layers, cfg.E, cfg.d, generator=g, device=dev) * 0.02
-        self.slot_of = torch.from_numpy(synth.hot_slot_table(layers, cfg.E, HOT, seed)).to(dev)
+        hot = HOT * layers // LAYERS  # the hot share of the pool stays 4,500 / 24,576
+        self.slot_of = torch.from_numpy(synth.hot_slot_table(layers, cfg.E, hot, seed)).to(dev)
         bias = np.stack([synth.bias_from_sets(synth.zipf_sets(T, cfg.E, cfg.k, seed + 1000 * l), cfg.E)
                          for l in range(layers)])
         self.bias = torch.from_numpy(bias).to(dev)
@@ -416,7 +417,7 @@ def run_ours(args):
     import torch
     world, rank, local = dist_setup()
     hbm, tf, tf_s, peak_kind = peaks()
-    st = DecodeStack(T=args.tokens, bits=args.bits)
+    st = DecodeStack(T=args.tokens, bits=args.bits, layers=args.layers)
     st.capture()
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
@@ -436,7 +437,7 @@ def run_ours(args):
     ms_max = allreduce_max(ms, world)
     ms_step = ms_max / args.steps
     tokens = st.T * args.steps * world
-    value = tokens / (ms_max / 1e3)
+    value = tokens / (ms_max / 1e3 * LAYERS / st.L)  # per 48-layer stack (st.L < 48 only when profiling)
 
     # expert kernels alone (events around each decode expert FFN call, cold weights)
     ffn_ms, ffn_bytes = st.time_expert_ffn()
@@ -461,7 +462,7 @@ def run_ours(args):
     e3.record(stream)
     torch.cuda.synchronize()
     e2e_ms = allreduce_max(e2.elapsed_time(e3), world)
-    e2e_value = st.T * n_e2e * world / (e2e_ms / 1e3)
+    e2e_value = st.T * n_e2e * world / (e2e_ms / 1e3 * LAYERS / st.L)
 
     layer_us = ms_step * 1e3 / st.L
     expert_gbs_layer = st.expert_bytes_step / (ms_step / 1e3) / 1e9
@@ -480,7 +481,7 @@ def run_ours(args):
         "data": "synthetic (seeded; random-init weights of the stated shapes)",
         "config": {
             "workload": f"decode layer d=2048 f=768 E=512 top-10 + 1 shared, T={st.T}, "
-                        f"{args.bits}-bit block-32 fp16-scale, Zipf(1.1) routing; 48 distinct layers per step",
+                        f"{args.bits}-bit block-32 fp16-scale, Zipf(1.1) routing; {st.L} distinct layers per step",
             "global_batch": st.T * world, "seq_len": 1, "parallelism": f"replicas x{world}",
             "l2": "inputs larger than L2 (48 layers, ~1 GB touched per step)",
             "layer_us": round(layer_us, 3),
@@ -504,7 +505,7 @@ def run_ours(args):
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(st, args.cpu_layers)
+        res["cpu_baseline"] = cpu_baseline(st, min(args.cpu_layers, st.L))
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:
@@ -674,6 +675,8 @@ def main():
     ap.add_argument("--cpu-layers", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill"])
+    ap.add_argument("--layers", type=int, default=LAYERS,
+                    help="decode: layers in the stack (fewer only to profile a small case)")
     ap.add_argument("--cpu-tokens", type=int, default=32, help="prefill: oracle sample size")
     args = ap.parse_args()
     if args.warmup < 3:
