@@ -6,10 +6,6 @@
 
 #include "moe_internal.cuh"
 
-struct moe_ctx {
-  moe::Ctx c;
-};
-
 namespace moe {
 
 static size_t align_up(size_t n, size_t a) { return (n + a - 1) / a * a; }

@@ -35,6 +35,15 @@ struct Ctx {
 constexpr int kTraceSlots = 32;
 constexpr int kTraceCtas = 1024;
 
+}  // namespace moe
+
+// The opaque context handle of the C ABI.
+struct moe_ctx {
+  moe::Ctx c;
+};
+
+namespace moe {
+
 // ---------------------------------------------------------------- workspace
 
 struct WsLayout {

@@ -89,6 +89,7 @@ _SIGS = {
     "moe_combine": (_I, [_P, ctypes.POINTER(_Cfg), ctypes.POINTER(Grouping), _P, _P, _I, _P, _S]),
     "moe_layer_forward": (_I, [_P, ctypes.POINTER(_Cfg), _P, _I, _P, _P, _P, _I, _P, _Z, _P, _P, _Z, _P,
                                _S]),
+    "moe_layer_forward_static": (_I, [_P, ctypes.POINTER(_Cfg), _P, _I, _P, _P, _P, _I, _P, _Z, _P, _P, _S]),
 }
 
 _lib = None
@@ -171,6 +172,13 @@ class Context:
                                           _ptr(slot_of), n_slots, _ptr(pool), stride, _ptr(shared), _ptr(ws),
                                           0 if ws is None else ws.numel() * ws.element_size(), _ptr(y),
                                           _stream(stream))
+
+    def layer_forward_static_status(self, cfg, x, T, w_router, bias, slot_of, n_slots, pool, stride, shared, y,
+                                    stream=None):
+        """moe_layer_forward with the library's static scratch (no workspace argument)."""
+        return self.lib.moe_layer_forward_static(self.h, ctypes.byref(cfg.c()), _ptr(x), T, _ptr(w_router),
+                                                 _ptr(bias), _ptr(slot_of), n_slots, _ptr(pool), stride,
+                                                 _ptr(shared), _ptr(y), _stream(stream))
 
     # -- checked wrappers ---------------------------------------------------------
     def router_topk(self, cfg, x, w_router, bias, T, logits, idx, gate, stream=None):

@@ -219,6 +219,34 @@ MOE_API moe_status moe_layer_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, con
                              size_t slot_stride, const uint8_t* shared_expert, void* ws,
                              size_t ws_bytes, void* y, moe_stream stream);
 
+/* moe_layer_forward without a workspace argument: the step's scratch is a
+ * static device array of MOE_STATIC_SCRATCH_BYTES inside the library image,
+ * reserved on each device when the library's module loads there, so the call
+ * allocates nothing. The pages have no counterpart; this serves callers that
+ * own no device allocator (a plain C host linking only this library) and
+ * decode loops that must not call cudaMalloc, which can synchronise the
+ * device.
+ *   - Arguments and results as moe_layer_forward, minus ws / ws_bytes.
+ *   - Limit: moe_workspace_bytes(cfg, T) must be <= MOE_STATIC_SCRATCH_BYTES,
+ *     else MOE_ENOSPACE and nothing runs. The full-size layer (d=2048,
+ *     f=768, E=512, k=10) needs about 0.72 MB at T = 8, so every decode
+ *     batch fits; at that size prefill chunks above about a dozen tokens
+ *     do not.
+ *   - Nothing in the scratch needs to start at zero.
+ *   - There is ONE scratch per device, shared by every context and stream:
+ *     calls that overlap in time on one device (two streams, two host
+ *     threads) race on it and give wrong results. Serialise them, e.g. on
+ *     one stream.
+ *   - The first call on a device does a one-time set-up (it looks up the
+ *     array's device address with that device current); make that first
+ *     call before any stream capture begins. */
+#define MOE_STATIC_SCRATCH_BYTES (2u << 20)
+MOE_API moe_status moe_layer_forward_static(moe_ctx* ctx, const moe_layer_cfg* cfg, const void* x, int T,
+                                    const float* w_router, const float* logit_bias,
+                                    const int32_t* slot_of, int n_slots, const uint8_t* slot_pool,
+                                    size_t slot_stride, const uint8_t* shared_expert, void* y,
+                                    moe_stream stream);
+
 #ifdef __cplusplus
 }
 #endif
