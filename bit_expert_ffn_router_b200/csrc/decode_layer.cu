@@ -58,7 +58,10 @@ struct DLParams {
   size_t stride;
   const uint8_t* shared;
   moe_expert_layout lay;
-  float* h;
+  float* h;                  // kRep copies of [n_rows, f], h_rep floats apart
+  size_t h_rep;
+  float* logits_rep;         // route: kRep copies of [T, E]
+  int32_t* slot_rep;         // route: kRep copies of [E]
   void* y;
   int* status;
   unsigned long long* gbar;  // grid-barrier arrival counter
@@ -289,7 +292,7 @@ __device__ void stage_issue(DLShared* S, const StageRec& s, int i, uint8_t* ring
 // Quantises the T token rows of x (bf16, global) into the gate/up layout,
 // four lanes per 32-value block. Loops run in whole warps (shuffles).
 template <int BITS>
-__device__ void quantise_x(const DLParams& P, int* xq, int nct) {
+__device__ void quantise_x(const DLParams& P, int* xq, uint16_t* xs, int nct) {
   const int nb = P.d / kBlock, bpl = nb / P.gu_lpr;
   const int words = QV<BITS>::kWords * nb;
   const int jobs = P.T * nb;
@@ -299,10 +302,14 @@ __device__ void quantise_x(const DLParams& P, int* xq, int nct) {
     const int job = (base + (threadIdx.x & 31)) >> 2;
     const bool live = job < jobs;
     const int t = live ? job / nb : 0, blk = live ? job % nb : 0;
-    const uint16_t* src = P.x + static_cast<size_t>(t) * P.d + blk * kBlock + q;
+    const size_t at = static_cast<size_t>(t) * P.d + blk * kBlock + q;
     float v[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = live ? bf16_bits_to_float(__ldcg(src + 4 * k)) : 0.f;
+    for (int k = 0; k < 8; ++k) {
+      const uint16_t bits = live ? __ldcg(P.x + at + 4 * k) : uint16_t(0);
+      if (live) xs[at + 4 * k] = bits;
+      v[k] = bf16_bits_to_float(bits);
+    }
     const int gl = blk / bpl, bb = blk % bpl;
     quant_quad<BITS>(v, xq + t * words, nb, bb * P.gu_lpr + gl, q, live);
   }
@@ -320,7 +327,7 @@ __device__ void quantise_h(const DLParams& P, int lo, int hi, int* hq, int nct) 
     const int job = (base + (threadIdx.x & 31)) >> 2;
     const bool live = job < jobs;
     const int r = live ? job / nb : 0, blk = live ? job % nb : 0;
-    const float* src = P.h + static_cast<size_t>(lo + r) * P.f + blk * kBlock + q;
+    const float* src = P.h + (blockIdx.x % kRep) * P.h_rep + static_cast<size_t>(lo + r) * P.f + blk * kBlock + q;
     float v[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) v[k] = live ? __ldcg(src + 4 * k) : 0.f;
@@ -356,7 +363,10 @@ __device__ __forceinline__ void process_gu(const StageRec& s, const uint8_t* rin
     if (active) v = row_dot2<BITS, BPL>(cg, sg, cg + row_b, sg + sc_n, P.d, gl, xr);
     v.x = group_sum(v.x, lpr);
     v.y = group_sum(v.y, lpr);
-    if (lane == 0) P.h[static_cast<size_t>(p) * P.f + c] = v.x / (1.f + expf(-v.x)) * v.y;
+    float hv = 0.f;
+    if (lane == 0) hv = v.x / (1.f + expf(-v.x)) * v.y;
+    hv = __shfl_sync(0xffffffffu, hv, 0);
+    if (lane < kRep) P.h[lane * P.h_rep + static_cast<size_t>(p) * P.f + c] = hv;
   }
 }
 
@@ -417,7 +427,7 @@ __device__ void group_in_smem(const DLParams& P, const RouteSmem& R, DLShared* S
       if (first) {
         const int u = base + __popc(m & ((1u << tid) - 1u));
         const int e = R.sorted_e[i];
-        int slot = P.slot_of[e];
+        int slot = __ldcg(P.slot_rep + (blockIdx.x % kRep) * P.E + e);
         if (slot < 0 || slot >= P.n_slots) {
           report(P.status, kDevBadSlot, e);
           slot = 0;
@@ -490,18 +500,76 @@ __device__ __forceinline__ float key_value(uint32_t k) {
   return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
 }
 
-__device__ void topk_warp(const DLParams& P, const RouteSmem& R, int t) {
+//
+// Fast path: the k-th largest of the 32 lane maxima (a bitonic sort across
+// the lanes) is a lower bound L of the k-th largest key, since those k lane
+// maxima are k distinct values. When at most 32 keys reach L, they are
+// compacted into `scratch` (32 words per warp) and each is ranked against the
+// others in one pass; otherwise k rounds of warp max select them.
+__device__ void topk_warp(const DLParams& P, const RouteSmem& R, int t, unsigned long long* scratch,
+                          unsigned long long* tr) {
   constexpr int VPL = 16;
   const int lane = threadIdx.x & 31;
-  const float* row = P.logits + static_cast<size_t>(t) * P.E;
+  const float* row = P.logits_rep + (static_cast<size_t>(blockIdx.x % kRep) * P.T + t) * P.E;
   uint32_t key[VPL];
 #pragma unroll
   for (int v = 0; v < VPL; ++v) {
     const int e = v * 32 + lane;
     key[v] = e < P.E ? order_key(__ldcg(row + e)) : 0u;
   }
+  if (tr != nullptr && lane == 0) {
+    uint32_t any = 0u;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) any |= key[v];
+    tr[28] = global_timer_ns() + (any & 0u);
+  }
   uint32_t mine_key = 0u;
   int mine_e = 0;
+  uint32_t lmax = 0u;
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) lmax = max(lmax, key[v]);
+  uint32_t srt = lmax;  // bitonic sort of the lane maxima, descending
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const uint32_t o = __shfl_xor_sync(0xffffffffu, srt, stride);
+      const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0 || size == 32);
+      srt = keep_max ? max(srt, o) : min(srt, o);
+    }
+  }
+  const uint32_t L = __shfl_sync(0xffffffffu, srt, P.k - 1);
+  int cnt = 0;
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) cnt += (L > 0u && key[v] >= L) ? 1 : 0;
+  const int C = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(cnt)));
+  if (L > 0u && C <= 32) {
+    int pos = cnt;  // exclusive prefix of cnt over the lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, pos, o);
+      if (lane >= o) pos += n;
+    }
+    pos -= cnt;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v)
+      if (key[v] >= L)  // larger word = larger key, then lower expert index
+        scratch[pos++] = (static_cast<unsigned long long>(key[v]) << 32) |
+                         (0xffffffffu - static_cast<uint32_t>(v * 32 + lane));
+    __syncwarp();
+    const unsigned long long mine = lane < C ? scratch[lane] : 0ull;
+    int rank = 0;
+    for (int j = 0; j < C; ++j) rank += scratch[j] > mine ? 1 : 0;
+    __syncwarp();
+    if (lane < C && rank < P.k) scratch[rank] = mine;
+    __syncwarp();
+    if (lane < P.k) {
+      const unsigned long long sel = scratch[lane];
+      mine_key = static_cast<uint32_t>(sel >> 32);
+      mine_e = static_cast<int>(0xffffffffu - static_cast<uint32_t>(sel & 0xffffffffu));
+    }
+    __syncwarp();
+  } else {
 #pragma unroll 1
   for (int j = 0; j < P.k; ++j) {
     uint32_t lm = 0u;
@@ -523,6 +591,8 @@ __device__ void topk_warp(const DLParams& P, const RouteSmem& R, int t) {
       mine_e = e;
     }
   }
+  }
+  if (tr != nullptr && lane == 0) tr[29] = global_timer_ns() + (mine_key & 0u);
   const bool sel = lane < P.k;
   const float lj = sel ? key_value(mine_key) : 0.f;
   const float l0 = __shfl_sync(0xffffffffu, lj, 0);
@@ -541,13 +611,19 @@ __device__ void topk_warp(const DLParams& P, const RouteSmem& R, int t) {
   }
 }
 
-// Router rows [e0, e1) of this CTA for every token: lanes read W_r (shared
-// memory) and x (global, bf16) in interleaved 4-column groups.
-__device__ void router_rows(const DLParams& P, const float* wrs, int e0, int e1, int cw) {
+// Router rows [e0, e1) of this CTA for every token: lanes read W_r and x
+// (both in shared memory) in interleaved 4-column groups. Every logit and
+// the rows' slots are written kRep times (one copy per group of readers).
+__device__ void router_rows(const DLParams& P, const float* wrs, const uint16_t* xs, int e0, int e1, int cw) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int n4 = P.d / 4;
+  if (warp == 0)
+    for (int i = lane; i < (e1 - e0) * kRep; i += 32) {
+      const int e = e0 + i / kRep, r = i % kRep;
+      P.slot_rep[r * P.E + e] = P.slot_of[e];
+    }
   for (int t = 0; t < P.T; ++t) {
-    const uint2* x2 = reinterpret_cast<const uint2*>(P.x + static_cast<size_t>(t) * P.d);
+    const uint2* x2 = reinterpret_cast<const uint2*>(xs + static_cast<size_t>(t) * P.d);
 #pragma unroll 1
     for (int e = e0 + warp; e < e1; e += cw) {
       const float4* w4 = reinterpret_cast<const float4*>(wrs + static_cast<size_t>(e - e0) * P.d);
@@ -555,16 +631,16 @@ __device__ void router_rows(const DLParams& P, const float* wrs, int e0, int e1,
 #pragma unroll 4
       for (int c4 = lane; c4 < n4; c4 += 32) {
         const float4 w = w4[c4];
-        const uint2 xb = __ldcg(x2 + c4);
+        const uint2 xb = x2[c4];
         acc = fmaf(w.x, __uint_as_float(xb.x << 16), acc);
         acc = fmaf(w.y, __uint_as_float(xb.x & 0xffff0000u), acc);
         acc = fmaf(w.z, __uint_as_float(xb.y << 16), acc);
         acc = fmaf(w.w, __uint_as_float(xb.y & 0xffff0000u), acc);
       }
       acc = warp_sum(acc);
-      if (lane == 0) {
+      if (lane < kRep) {
         const size_t o = static_cast<size_t>(t) * P.E + e;
-        P.logits[o] = P.bias ? acc + P.bias[o] : acc;
+        P.logits_rep[lane * static_cast<size_t>(P.T) * P.E + o] = P.bias ? acc + P.bias[o] : acc;
       }
     }
   }
@@ -586,6 +662,7 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
   int* xq = reinterpret_cast<int*>(smem + P.sm_xq);
   float* wrs = reinterpret_cast<float*>(smem + P.sm_wr);
   int* hq = reinterpret_cast<int*>(smem + P.sm_hq);
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + P.sm_hq);  // raw x for the router (before hq is used)
   uint8_t* ring = reinterpret_cast<uint8_t*>(smem + P.sm_ring);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -687,6 +764,7 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
       }
       okl = __shfl_sync(0xffffffffu, okl, 0);
       batch = __shfl_sync(0xffffffffu, batch, 0);
+      if (lane == 0 && i == n_sh) MOE_TRACE(16)
       if (!okl) {
         ok = false;
         break;
@@ -694,6 +772,7 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
       __syncwarp();
       if (lane < batch) stage_issue(S, st[i + lane], i + lane, ring, P, R);
       __syncwarp();
+      if (lane == 0 && i == n_sh) MOE_TRACE(17)
       i += batch;
     }
     if (lane == 0) MOE_TRACE(13)
@@ -716,13 +795,13 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
   // -------------------------------------------------------------- consumers
   const int tid = threadIdx.x;
   grid_dep_wait();  // x (and the workspace) may come from the previous kernel
-  quantise_x<BITS>(P, xq, CT);
+  quantise_x<BITS>(P, xq, xs, CT);
   named_sync(1, CT);
   if (tid == 0) MOE_TRACE(1)
 
   if (ROUTE) {
     if (e1 > e0 && !mbar_wait_warp(&S->wr_bar, 0, deadline)) set_abort(S, P.status, 1);
-    if (!aborted(S)) router_rows(P, wrs, e0, e1, CW);
+    if (!aborted(S)) router_rows(P, wrs, xs, e0, e1, CW);
     named_sync(1, CT);
     if (tid == 0) MOE_TRACE(2)
     if (tid == 0 && !aborted(S)) S->bar_target = gbar_arrive(P.gbar, G);
@@ -743,7 +822,9 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
         named_sync(1, CT);
         if (tid == 0) MOE_TRACE(4)
         if (!aborted(S))
-          for (int t = warp; t < P.T; t += CW) topk_warp(P, R, t);
+          for (int t = warp; t < P.T; t += CW)
+            topk_warp(P, R, t, reinterpret_cast<unsigned long long*>(smem + P.sm_hq) + warp * 32,
+                      t == 0 ? trace : nullptr);
         named_sync(1, CT);
         if (tid == 0) MOE_TRACE(10)
         if (b == 0)
@@ -775,10 +856,13 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
     }
     if (i >= n_gu) break;
     if (!aborted(S) && warp < st[i].b - st[i].a) {
-      if (mbar_wait_warp(&S->full[i % kNB], (i / kNB) & 1, deadline))
+      if (mbar_wait_warp(&S->full[i % kNB], (i / kNB) & 1, deadline)) {
+        if (tid == 0 && i == n_sh) MOE_TRACE(18)
         process_gu<BITS, GBPL>(st[i], ring, P, R, np, xq, cur_t, xr);
-      else
+        if (tid == 0 && i == n_gu - 1) MOE_TRACE(19)
+      } else {
         set_abort(S, P.status, 4);
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&S->empty[i % kNB]);
@@ -795,6 +879,7 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
   named_sync(1, CT);
   if (tid == 0) MOE_TRACE(7)
   grid_dep_launch();
+  if (tid == 0) MOE_TRACE(11)
 
   // down stages, in chunks whose h rows fit the quantised staging area
 #pragma unroll 1
@@ -943,6 +1028,9 @@ cudaError_t launch_decode_layer(const Ctx& ctx, const moe_layer_cfg& c, const De
   P.shared = a.shared;
   P.lay = a.lay;
   P.h = a.h;
+  P.h_rep = static_cast<size_t>(np + (c.n_shared ? T : 0)) * c.f;
+  P.logits_rep = a.logits_rep;
+  P.slot_rep = a.slot_rep;
   P.y = a.y;
   P.status = ctx.d_status;
   P.gbar = ctx.d_gbar;
@@ -984,8 +1072,13 @@ cudaError_t launch_decode_layer(const Ctx& ctx, const moe_layer_cfg& c, const De
   const size_t h_row_bytes = qw * (c.f / kBlock) * 4;
   const int h_cap = static_cast<int>((48 * 1024) / h_row_bytes);
   P.h_rows = n_rows_all < h_cap ? n_rows_all : (h_cap > T ? h_cap : T);
-  P.sm_hq = static_cast<int>(o);
-  o = align_up(o + static_cast<size_t>(P.h_rows) * h_row_bytes, 128);
+  P.sm_hq = static_cast<int>(o);  // also holds the raw x [T, d] bf16 before the down phase
+  const size_t hq_bytes = static_cast<size_t>(P.h_rows) * h_row_bytes;
+  const size_t xs_bytes = static_cast<size_t>(T) * c.d * 2;
+  const size_t tk_bytes = static_cast<size_t>(CW) * 32 * 8;  // top-k scratch (after the router, before hq)
+  size_t region = hq_bytes > xs_bytes ? hq_bytes : xs_bytes;
+  region = region > tk_bytes ? region : tk_bytes;
+  o = align_up(o + region, 128);
   P.sm_ring = static_cast<int>(o);
   const long long ring = static_cast<long long>(kSmemMax) - static_cast<long long>(o);
   const long long gu_stage = 2LL * CW * (P.gu_row + P.gu_sc);

@@ -12,16 +12,31 @@
 //   down:    D[128 output rows, N pairs] = W_d[rows, f] * H[pairs, f]^T,
 //            epilogue z = gate * D -> fp32 rows in pair order
 //
-// One persistent CTA per SM, ten warps:
-//   warp 0     TMA producer: packed codes (3-D tensor maps over the whole
-//              expert pool), fp16 scales (one bulk copy per tile) and the
-//              activation tile (128B-swizzled, K-major);
-//   warp 1     TMEM allocation and the single-thread tcgen05.mma issue;
-//   warps 2-5  dequantisation: each thread owns one weight row and writes
-//              s * (q - 2^(b-1)) as fp16 straight into the 128B-swizzled
-//              K-major layout the tensor core reads;
-//   warps 6-9  epilogue: tcgen05.ld of the fp32 accumulators (two TMEM
-//              buffers, so the next tile's MMAs overlap this tile's stores).
+// One persistent CTA per SM, fifteen warps:
+//   warp 0      activation producer: the 128B-swizzled K-major activation
+//               tile by TMA, a box of 16 to 128 rows sized to the item's N;
+//   warp 14     weight producer: packed codes (3-D tensor maps over the
+//               whole expert pool) and fp16 scales (one bulk copy per work
+//               item), running ahead of the activations as far as its own
+//               ring allows;
+//   warp 1      TMEM allocation and the single-thread tcgen05.mma issue;
+//   warps 2-9   dequantisation, two teams of four warps taking alternate
+//               64-wide K stages: each thread owns one weight row and writes
+//               s * (q - 2^(b-1)) as fp16 straight into the 128B-swizzled
+//               K-major layout the tensor core reads;
+//   warps 10-13 epilogue: tcgen05.ld of the fp32 accumulators (two TMEM
+//               buffers, so the next item's MMAs overlap this item's stores).
+//
+// K order. A 32-bit word of 2-bit codes holds a 16-code group; shifting it by
+// 2i and masking 0x00030003 yields codes i and i+8 in the two halves of one
+// fp16x2 register. The dequantiser stores that pair as K positions 2i, 2i+1,
+// i.e. inside every aligned group of 16 the K order is
+//     position 2i <- index i,   position 2i+1 <- index i+8.
+// A dot product does not depend on the order of its terms, so the activation
+// operands are stored in the same order (the x gather and the gate/up
+// epilogue's h writes permute within each group of 16) and the result is the
+// plain contraction. Groups never straddle a 32-weight scale block.
+//
 // Operands are fp16 on both sides (A and B of one kind::f16 MMA share a
 // type): 2-bit weights are exact in fp16, 3-bit ones round at 2^-12
 // relative, bf16 activations convert exactly in fp16's normal range.
@@ -38,19 +53,20 @@ namespace {
 constexpr int kBM = 128;            // weight rows per tile (MMA M)
 constexpr int kBN = kTileN;         // pairs per tile (MMA N, max)
 constexpr int kBK = 64;             // K per pipeline stage (one 128-byte swizzle row of fp16)
-constexpr int kChunk = 128;         // codes per code-chunk load (two stages)
-constexpr int kKPerChunk = kChunk / kBK;
-constexpr int kStages = 4;          // A/B ring depth
-constexpr int kCStages = 4;         // code-chunk ring depth
-constexpr int kThreads = 320;
+constexpr int kChunk = 128;         // codes per code-chunk load: one stage for each dequant team
+constexpr int kAStages = 4;         // dequantised weight ring
+constexpr int kBStages = 5;         // activation ring
+constexpr int kCStages = 4;         // code-chunk ring
+constexpr int kDqThreads = 128;     // threads per dequant team (one per weight row)
+constexpr int kThreads = 15 * 32;
 constexpr int kTmemCols = 2 * kBN;  // two accumulator buffers
 constexpr int kMaxKDim = 2048;      // largest reduction size (scale staging holds 128 x K/16 bytes)
 
 struct PrefillSmem {
   // byte offsets from the 1024-aligned base of dynamic shared memory
-  static constexpr int kA = 0;                                     // kStages x 16 KB, 128B-swizzled
-  static constexpr int kB = kA + kStages * kBM * kBK * 2;          // kStages x 16 KB, 128B-swizzled
-  static constexpr int kCodeLo = kB + kStages * kBN * kBK * 2;     // kCStages x (128 rows x 32 B)
+  static constexpr int kA = 0;                                     // kAStages x 16 KB, 128B-swizzled
+  static constexpr int kB = kA + kAStages * kBM * kBK * 2;         // kBStages x 16 KB, 128B-swizzled
+  static constexpr int kCodeLo = kB + kBStages * kBN * kBK * 2;    // kCStages x (128 rows x 32 B)
   static constexpr int kCodeHi = kCodeLo + kCStages * kBM * (kChunk / 4);  // kCStages x (128 x 16 B)
   static constexpr int kScale = kCodeHi + kCStages * kBM * (kChunk / 8);   // 2 x (128 rows x K/16 B)
   static constexpr int kScaleBuf = kBM * (kMaxKDim / kBlock) * 2;
@@ -59,39 +75,39 @@ struct PrefillSmem {
   static constexpr int kBytes = kBar + 1024;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base
 };
+static_assert(PrefillSmem::kAlloc <= 227 * 1024, "shared memory budget");
 
 struct Bars {
-  uint64_t ab_full_a[kStages];   // dequant -> MMA (count 128)
-  uint64_t ab_full_b[kStages];   // TMA -> MMA (tx)
-  uint64_t ab_empty[kStages];    // MMA commit -> producer, dequant
-  uint64_t c_full[kCStages];     // TMA -> dequant (tx)
-  uint64_t c_empty[kCStages];    // dequant -> producer (count 128)
-  uint64_t s_full[2];            // bulk copy -> dequant (tx)
-  uint64_t s_empty[2];           // dequant -> producer (count 128)
-  uint64_t d_full[2];            // MMA commit -> epilogue
-  uint64_t d_empty[2];           // epilogue -> MMA (count 128)
-  uint64_t mma_done;             // final MMA commit, waited on before TMEM is freed
+  uint64_t a_full[kAStages];    // dequant team -> MMA (count 128)
+  uint64_t a_empty[kAStages];   // MMA commit -> dequant team
+  uint64_t b_full[kBStages];    // TMA -> MMA (tx)
+  uint64_t b_empty[kBStages];   // MMA commit -> producer
+  uint64_t c_full[kCStages];    // TMA -> dequant (tx)
+  uint64_t c_empty[kCStages];   // both dequant teams -> producer (count 256)
+  uint64_t s_full[2];           // bulk copy -> dequant (tx)
+  uint64_t s_empty[2];          // both dequant teams -> producer (count 256)
+  uint64_t d_full[2];           // MMA commit -> epilogue
+  uint64_t d_empty[2];          // epilogue -> MMA (count 128)
+  uint64_t mma_done;            // final MMA commit, waited on before TMEM is freed
   uint32_t tmem_base;
   int abort_flag;
 };
 static_assert(sizeof(Bars) <= 1024, "barrier block");
 
 struct GemmParams {
-  const int32_t* tile_offset;    // [E+2]
-  const int32_t* expert_offset;  // [E+1]
-  const int32_t* expert_count;   // [E]
-  const int32_t* pair_slot;      // [n_pairs]
-  const float* pair_gate;        // [n_pairs]
-  const uint8_t* pool;           // scale sections are read with plain bulk copies
-  const uint8_t* shared;         // shared-expert record (or null)
+  const int4* tile_info;        // per token tile: {expert (E = shared), first row, rows, slot}
+  const int32_t* tile_offset;   // [E+2]; tile_offset[E+1] = number of token tiles
+  const float* pair_gate;       // [n_pairs]
+  const uint8_t* pool;          // scale sections are read with plain bulk copies
+  const uint8_t* shared;        // shared-expert record (or null)
   size_t stride;
-  size_t scale_off;              // section offset of this matrix's scales inside a record
-  int E, T, n_pairs;
-  int K, m_tiles;                // reduction size, weight-row tiles per expert
-  int hi_col0;                   // byte column of the high plane in a code row (3-bit)
-  int sc_row_bytes;              // fp16 scale bytes per weight row (K/16)
-  void* out;                     // gate/up: h fp16 [n_rows, f]; down: z fp32 [n_rows, d]
-  int ld_out;                    // elements per output row
+  size_t scale_off;             // section offset of this matrix's scales inside a record
+  int E, n_pairs;
+  int K, m_tiles;               // reduction size, weight-row tiles per expert
+  int hi_col0;                  // byte column of the high plane in a code row (3-bit)
+  int sc_row_bytes;             // fp16 scale bytes per weight row (K/16)
+  void* out;                    // gate/up: h fp16 [n_rows, f]; down: z fp32 [n_rows, d]
+  int ld_out;                   // elements per output row
   int* status;
   unsigned long long timeout_ns;
 };
@@ -180,98 +196,82 @@ __device__ __forceinline__ bool wait_bar(Bars* B, uint64_t* bar, uint32_t parity
   return false;
 }
 
-// ------------------------------------------------------------------ work decoding
-struct Item {
-  int expert;  // 0..E-1 routed, E shared
-  int row0;    // first sorted row of the tile
-  int rows;    // valid rows (1..kBN)
-  int slot;    // pool slot (routed experts)
-  int m;       // weight-row tile
-};
-
-// Work item w = token tile * m_tiles + weight-row tile; consecutive items
-// share a token tile, so CTAs running side by side read the same activation
-// rows from L2 and different weight tiles.
-__device__ __forceinline__ Item decode_item(const GemmParams& P, int w) {
-  const int tile = w / P.m_tiles;
-  Item it;
-  it.m = w - tile * P.m_tiles;
-  int lo = 0, hi = P.E;  // last extended expert x with tile_offset[x] <= tile
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(P.tile_offset + mid) <= tile) lo = mid;
-    else hi = mid - 1;
-  }
-  it.expert = lo;
-  const int ti = tile - __ldg(P.tile_offset + lo);
-  const int base = lo < P.E ? __ldg(P.expert_offset + lo) : P.n_pairs;
-  const int cnt = lo < P.E ? __ldg(P.expert_count + lo) : P.T;
-  it.row0 = base + ti * kBN;
-  it.rows = min(kBN, cnt - ti * kBN);
-  it.slot = lo < P.E ? __ldg(P.pair_slot + it.row0) : 0;
-  return it;
-}
+// ------------------------------------------------------------------ K-order permutation
+// Position of index i inside its group of 16 (inverse of: position 2i <- i,
+// position 2i+1 <- i+8).
+__host__ __device__ __forceinline__ int k_position(int i) { return i < 8 ? 2 * i : 2 * i - 15; }
 
 // ------------------------------------------------------------------ dequantisation of one K stage
-// Thread r writes row r of the A tile: 64 weights s * (q - 2^(BITS-1)) as
-// fp16, 16-byte chunk j of the row at chunk position j ^ (r % 8) (the
-// 128-byte swizzle the descriptor names).
+// Row r of the A tile: 64 weights s * (q - 2^(BITS-1)) as fp16 in the
+// permuted K order, 16-byte chunk j of the row at chunk position j ^ (r % 8)
+// (the 128-byte swizzle the descriptor names).
 template <int BITS>
 __device__ __forceinline__ void dequant_stage(uint8_t* a_tile, const uint8_t* lo, const uint8_t* hi,
-                                              const uint16_t* sc, int r) {
-  const uint4 w = *reinterpret_cast<const uint4*>(lo);  // 64 two-bit codes
+                                              uint32_t s01, int r) {
+  const uint4 w = *reinterpret_cast<const uint4*>(lo);  // 64 two-bit codes: four groups of 16
   const uint32_t wl[4] = {w.x, w.y, w.z, w.w};
-  uint2 hw = make_uint2(0u, 0u);
-  if (BITS == 3) hw = *reinterpret_cast<const uint2*>(hi);  // their 64 high bits
-  const uint32_t hb[2] = {hw.x, hw.y};
-  const __half2 s0 = __half2half2(__ushort_as_half(sc[0]));
-  const __half2 s1 = __half2half2(__ushort_as_half(sc[1]));
+  uint32_t hq[4] = {0u, 0u, 0u, 0u};
+  if (BITS == 3) {
+    // the groups' high bits, spread so that index i lands at bit 2+i and
+    // index i+8 at bit 18+i
+    const uint2 hv = *reinterpret_cast<const uint2*>(hi);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t h16 = ((q < 2 ? hv.x : hv.y) >> (16 * (q & 1))) & 0xffffu;
+      hq[q] = ((h16 & 0xffu) | ((h16 & 0xff00u) << 8)) << 2;
+    }
+  }
+  const __half2 s0 = __half2half2(__ushort_as_half(static_cast<unsigned short>(s01 & 0xffffu)));
+  const __half2 s1 = __half2half2(__ushort_as_half(static_cast<unsigned short>(s01 >> 16)));
   // 0x6400 | q is the fp16 number 1024 + q; subtracting 1024 + 2^(BITS-1) is exact
   const __half2 off = __float2half2_rn(1024.f + static_cast<float>(1 << (BITS - 1)));
   uint8_t* row = a_tile + r * 128;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {  // weights 8j .. 8j+7
-    const uint32_t wd = wl[j >> 1] >> (16 * (j & 1));
-    uint32_t hbits = 0;
-    if (BITS == 3) hbits = (hb[j >> 2] >> (8 * (j & 3))) & 0xffu;
-    uint32_t out[4];
+  for (int q = 0; q < 4; ++q) {
+    const __half2 s = q < 2 ? s0 : s1;
+    uint32_t out[8];
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {  // weights 8j+2p (low half), 8j+2p+1 (high half)
-      uint32_t q = ((wd >> (4 * p)) & 0x3u) | (((wd >> (4 * p + 2)) & 0x3u) << 16);
-      if (BITS == 3) q |= (((hbits >> (2 * p)) & 1u) << 2) | (((hbits >> (2 * p + 1)) & 1u) << 18);
-      q |= 0x64006400u;
-      const __half2 v = __hsub2(*reinterpret_cast<const __half2*>(&q), off);
-      const __half2 y = __hmul2(v, (j < 4) ? s0 : s1);
-      out[p] = *reinterpret_cast<const uint32_t*>(&y);
+    for (int i = 0; i < 8; ++i) {
+      uint32_t v = (wl[q] >> (2 * i)) & 0x00030003u;
+      if (BITS == 3) v |= (hq[q] >> i) & 0x00040004u;
+      v |= 0x64006400u;
+      const __half2 y = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&v), off), s);
+      out[i] = *reinterpret_cast<const uint32_t*>(&y);
     }
-    *reinterpret_cast<uint4*>(row + ((j ^ (r & 7)) * 16)) = make_uint4(out[0], out[1], out[2], out[3]);
+    *reinterpret_cast<uint4*>(row + (((2 * q) ^ (r & 7)) * 16)) = make_uint4(out[0], out[1], out[2], out[3]);
+    *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ (r & 7)) * 16)) = make_uint4(out[4], out[5], out[6], out[7]);
   }
 }
 
 // ------------------------------------------------------------------ the kernel
 template <int BITS, bool DOWN>
 __global__ void __launch_bounds__(kThreads, 1)
-grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB, const __grid_constant__ CUtensorMap tLo,
-                    const __grid_constant__ CUtensorMap tHi, const __grid_constant__ CUtensorMap tLoS,
-                    const __grid_constant__ CUtensorMap tHiS, const GemmParams P) {
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB16, const __grid_constant__ CUtensorMap tB32,
+                    const __grid_constant__ CUtensorMap tB64, const __grid_constant__ CUtensorMap tB128,
+                    const __grid_constant__ CUtensorMap tLo, const __grid_constant__ CUtensorMap tHi,
+                    const __grid_constant__ CUtensorMap tLoS, const __grid_constant__ CUtensorMap tHiS,
+                    const GemmParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* B = reinterpret_cast<Bars*>(smem + PrefillSmem::kBar);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&B->ab_full_a[i], 128);
-      mbar_init(&B->ab_full_b[i], 1);
-      mbar_init(&B->ab_empty[i], 1);
+    for (int i = 0; i < kAStages; ++i) {
+      mbar_init(&B->a_full[i], kDqThreads);
+      mbar_init(&B->a_empty[i], 1);
+    }
+    for (int i = 0; i < kBStages; ++i) {
+      mbar_init(&B->b_full[i], 1);
+      mbar_init(&B->b_empty[i], 1);
     }
     for (int i = 0; i < kCStages; ++i) {
       mbar_init(&B->c_full[i], 1);
-      mbar_init(&B->c_empty[i], 128);
+      mbar_init(&B->c_empty[i], 2 * kDqThreads);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&B->s_full[i], 1);
-      mbar_init(&B->s_empty[i], 128);
+      mbar_init(&B->s_empty[i], 2 * kDqThreads);
       mbar_init(&B->d_full[i], 1);
       mbar_init(&B->d_empty[i], 128);
     }
@@ -293,59 +293,76 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB, const __grid_constan
   // everything below reads the grouping (and, for the down pass, h) written
   // by the kernels before this one
   grid_dep_wait();
-  const uint64_t deadline = P.timeout_ns;  // limit of each wait
+  const uint64_t limit = P.timeout_ns;  // limit of each wait
   const int total = __ldg(P.tile_offset + P.E + 1) * P.m_tiles;
   const int ks_per_item = P.K / kBK;
   const int chunks_per_item = P.K / kChunk;
   const uint32_t code_tx = kBM * (kChunk / 4) + (BITS == 3 ? kBM * (kChunk / 8) : 0);
   const uint32_t scale_tx = kBM * P.sc_row_bytes;
+  const int G = gridDim.x;
 
   if (warp == 0) {
-    // ---------------------------------------------------------- producer
+    // ---------------------------------------------------------- activation producer
     if (lane == 0) {
-      int g = 0, gc = 0, it = 0;
-      for (int w = blockIdx.x; w < total && !aborted(B); w += gridDim.x, ++it) {
-        const Item I = decode_item(P, w);
-        const bool sh = I.expert >= P.E;
+      int g = 0;
+      int4 next = blockIdx.x < total ? __ldg(P.tile_info + blockIdx.x / P.m_tiles) : make_int4(0, 0, 0, 0);
+      bool ok = true;
+      for (int w = blockIdx.x; w < total && ok && !aborted(B); w += G) {
+        const int4 info = next;  // {expert, row0, rows, slot}
+        if (w + G < total) next = __ldg(P.tile_info + (w + G) / P.m_tiles);
+        const int box = info.z <= 16 ? 16 : info.z <= 32 ? 32 : info.z <= 64 ? 64 : 128;
+        const CUtensorMap* mB = box == 16 ? &tB16 : box == 32 ? &tB32 : box == 64 ? &tB64 : &tB128;
+        const uint32_t b_tx = static_cast<uint32_t>(box) * kBK * 2;
+        for (int k = 0; k < ks_per_item; ++k, ++g) {
+          const int st = g % kBStages;
+          if (g >= kBStages && !wait_bar(B, &B->b_empty[st], ((g / kBStages) - 1) & 1, limit, P.status, 3)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&B->b_full[st], b_tx);
+          tma_load_2d(smem + PrefillSmem::kB + st * kBN * kBK * 2, mB, k * kBK, info.y, &B->b_full[st]);
+        }
+      }
+      // every copy this thread issued lands before the CTA may exit (bounded wait)
+      const uint64_t drain = global_timer_ns() + P.timeout_ns;
+      for (int n = max(0, g - kBStages); n < g; ++n) mbar_wait(&B->b_full[n % kBStages], (n / kBStages) & 1, drain);
+    }
+  } else if (warp == 14) {
+    // ---------------------------------------------------------- weight producer
+    if (lane == 0) {
+      int gc = 0, it = 0;
+      int4 next = blockIdx.x < total ? __ldg(P.tile_info + blockIdx.x / P.m_tiles) : make_int4(0, 0, 0, 0);
+      for (int w = blockIdx.x; w < total && !aborted(B); w += G, ++it) {
+        const int4 info = next;
+        if (w + G < total) next = __ldg(P.tile_info + (w + G) / P.m_tiles);
+        const int m = w % P.m_tiles;
+        const bool sh = info.x >= P.E;
         const CUtensorMap* mLo = sh ? &tLoS : &tLo;
         const CUtensorMap* mHi = sh ? &tHiS : &tHi;
-        const int slot = sh ? 0 : I.slot;
+        const int slot = sh ? 0 : info.w;
         const uint8_t* rec = sh ? P.shared : P.pool + static_cast<size_t>(slot) * P.stride;
         const int sb = it & 1;
-        if (it >= 2 && !wait_bar(B, &B->s_empty[sb], ((it >> 1) - 1) & 1, deadline, P.status, 1)) break;
+        if (it >= 2 && !wait_bar(B, &B->s_empty[sb], ((it >> 1) - 1) & 1, limit, P.status, 1)) break;
         mbar_arrive_expect_tx(&B->s_full[sb], scale_tx);
         bulk_g2s(smem + PrefillSmem::kScale + sb * PrefillSmem::kScaleBuf,
-                 rec + P.scale_off + static_cast<size_t>(I.m) * scale_tx, scale_tx, &B->s_full[sb]);
+                 rec + P.scale_off + static_cast<size_t>(m) * scale_tx, scale_tx, &B->s_full[sb]);
         bool ok = true;
-        for (int c = 0; c < chunks_per_item && ok; ++c, ++gc) {
+        for (int c = 0; c < chunks_per_item; ++c, ++gc) {
           const int cs = gc % kCStages;
-          if (gc >= kCStages && !wait_bar(B, &B->c_empty[cs], ((gc / kCStages) - 1) & 1, deadline, P.status, 2)) {
+          if (gc >= kCStages && !wait_bar(B, &B->c_empty[cs], ((gc / kCStages) - 1) & 1, limit, P.status, 2)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&B->c_full[cs], code_tx);
-          tma_load_3d(smem + PrefillSmem::kCodeLo + cs * kBM * (kChunk / 4), mLo, c * (kChunk / 4), I.m * kBM, slot,
+          tma_load_3d(smem + PrefillSmem::kCodeLo + cs * kBM * (kChunk / 4), mLo, c * (kChunk / 4), m * kBM, slot,
                       &B->c_full[cs]);
           if (BITS == 3)
             tma_load_3d(smem + PrefillSmem::kCodeHi + cs * kBM * (kChunk / 8), mHi, P.hi_col0 + c * (kChunk / 8),
-                        I.m * kBM, slot, &B->c_full[cs]);
-          for (int k = 0; k < kKPerChunk; ++k, ++g) {
-            const int st = g % kStages;
-            if (g >= kStages && !wait_bar(B, &B->ab_empty[st], ((g / kStages) - 1) & 1, deadline, P.status, 3)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(&B->ab_full_b[st], kBN * kBK * 2);
-            tma_load_2d(smem + PrefillSmem::kB + st * kBN * kBK * 2, &tB, (c * kKPerChunk + k) * kBK, I.row0,
-                        &B->ab_full_b[st]);
-          }
+                        m * kBM, slot, &B->c_full[cs]);
         }
         if (!ok) break;
       }
-      // Every copy this thread issued lands before the CTA may exit: wait
-      // (bounded) for the last phase armed on each ring slot.
       const uint64_t drain = global_timer_ns() + P.timeout_ns;
-      for (int n = max(0, g - kStages); n < g; ++n) mbar_wait(&B->ab_full_b[n % kStages], (n / kStages) & 1, drain);
       for (int n = max(0, gc - kCStages); n < gc; ++n) mbar_wait(&B->c_full[n % kCStages], (n / kCStages) & 1, drain);
       for (int n = max(0, it - 2); n < it; ++n) mbar_wait(&B->s_full[n & 1], (n >> 1) & 1, drain);
     }
@@ -353,30 +370,32 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB, const __grid_constan
     // ---------------------------------------------------------- MMA issue
     if (lane == 0) {
       int g = 0, it = 0;
-      for (int w = blockIdx.x; w < total && !aborted(B); w += gridDim.x, ++it) {
-        const Item I = decode_item(P, w);
-        const int n = (I.rows + 15) / 16 * 16;
+      int4 next = blockIdx.x < total ? __ldg(P.tile_info + blockIdx.x / P.m_tiles) : make_int4(0, 0, 0, 0);
+      for (int w = blockIdx.x; w < total && !aborted(B); w += G, ++it) {
+        const int4 info = next;
+        if (w + G < total) next = __ldg(P.tile_info + (w + G) / P.m_tiles);
+        const int n = (info.z + 15) / 16 * 16;
         const uint32_t idesc = instr_desc(n);
         const int acc = it & 1;
-        if (it >= 2 && !wait_bar(B, &B->d_empty[acc], ((it >> 1) - 1) & 1, deadline, P.status, 4)) break;
+        if (it >= 2 && !wait_bar(B, &B->d_empty[acc], ((it >> 1) - 1) & 1, limit, P.status, 4)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kBN);
         bool ok = true;
         for (int k = 0; k < ks_per_item; ++k, ++g) {
-          const int st = g % kStages;
-          const uint32_t ph = (g / kStages) & 1;
-          if (!wait_bar(B, &B->ab_full_a[st], ph, deadline, P.status, 5) ||
-              !wait_bar(B, &B->ab_full_b[st], ph, deadline, P.status, 6)) {
+          const int sa = g % kAStages, sbb = g % kBStages;
+          if (!wait_bar(B, &B->a_full[sa], (g / kAStages) & 1, limit, P.status, 5) ||
+              !wait_bar(B, &B->b_full[sbb], (g / kBStages) & 1, limit, P.status, 6)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t da = smem_desc(smem + PrefillSmem::kA + st * kBM * kBK * 2);
-          const uint64_t db = smem_desc(smem + PrefillSmem::kB + st * kBN * kBK * 2);
+          const uint64_t da = smem_desc(smem + PrefillSmem::kA + sa * kBM * kBK * 2);
+          const uint64_t db = smem_desc(smem + PrefillSmem::kB + sbb * kBN * kBK * 2);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)  // K = 16 per MMA: 32 bytes = 2 descriptor units
             tc_mma(d_tmem, da + 2 * kk, db + 2 * kk, idesc, (k > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(&B->ab_empty[st]);
+          tc_commit(&B->a_empty[sa]);
+          tc_commit(&B->b_empty[sbb]);
         }
         if (!ok) break;
         tc_commit(&B->d_full[acc]);
@@ -385,73 +404,79 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB, const __grid_constan
       tc_commit(&B->mma_done);
       mbar_wait(&B->mma_done, 0, global_timer_ns() + P.timeout_ns);
     }
-  } else if (warp < 6) {
+  } else if (warp >= 2 && warp < 10) {
     // ---------------------------------------------------------- dequantisation
-    const int r = threadIdx.x - 64;  // weight row of the tile
+    const int team = (warp - 2) >> 2;          // stages 2c + team of code chunk c
+    const int r = (threadIdx.x - 64) & 127;    // weight row of the tile
     int g = 0, gc = 0, it = 0;
-    for (int w = blockIdx.x; w < total && !aborted(B); w += gridDim.x, ++it) {
+    for (int w = blockIdx.x; w < total && !aborted(B); w += G, ++it) {
       const int sb = it & 1;
-      if (!wait_bar(B, &B->s_full[sb], (it >> 1) & 1, deadline, P.status, 7)) break;
-      const uint16_t* sc = reinterpret_cast<const uint16_t*>(smem + PrefillSmem::kScale + sb * PrefillSmem::kScaleBuf) +
-                           r * (P.sc_row_bytes / 2);
+      if (!wait_bar(B, &B->s_full[sb], (it >> 1) & 1, limit, P.status, 7)) break;
+      const uint8_t* sc = smem + PrefillSmem::kScale + sb * PrefillSmem::kScaleBuf + r * P.sc_row_bytes;
       bool ok = true;
-      for (int c = 0; c < chunks_per_item && ok; ++c, ++gc) {
+      for (int c = 0; c < chunks_per_item; ++c, ++gc, g += kChunk / kBK) {
         const int cs = gc % kCStages;
-        if (!wait_bar(B, &B->c_full[cs], (gc / kCStages) & 1, deadline, P.status, 8)) {
+        if (!wait_bar(B, &B->c_full[cs], (gc / kCStages) & 1, limit, P.status, 8)) {
           ok = false;
           break;
         }
-        const uint8_t* lo = smem + PrefillSmem::kCodeLo + cs * kBM * (kChunk / 4) + r * (kChunk / 4);
-        const uint8_t* hi = smem + PrefillSmem::kCodeHi + cs * kBM * (kChunk / 8) + r * (kChunk / 8);
-        for (int k = 0; k < kKPerChunk; ++k, ++g) {
-          const int st = g % kStages;
-          if (g >= kStages && !wait_bar(B, &B->ab_empty[st], ((g / kStages) - 1) & 1, deadline, P.status, 9)) {
-            ok = false;
-            break;
-          }
-          const int kb = (c * kKPerChunk + k) * (kBK / kBlock);  // first scale block of the stage
-          dequant_stage<BITS>(smem + PrefillSmem::kA + st * kBM * kBK * 2, lo + k * (kBK / 4), hi + k * (kBK / 8),
-                              sc + kb, r);
-          fence_proxy_async();  // generic-proxy writes -> visible to the tensor core
-          mbar_arrive(&B->ab_full_a[st]);
+        const int gt = g + team;  // this team's stage
+        const int st = gt % kAStages;
+        if (gt >= kAStages && !wait_bar(B, &B->a_empty[st], ((gt / kAStages) - 1) & 1, limit, P.status, 9)) {
+          ok = false;
+          break;
         }
+        // scales of blocks 4c + 2*team and 4c + 2*team + 1
+        const uint32_t s01 = *reinterpret_cast<const uint32_t*>(sc + 8 * c + 4 * team);
+        dequant_stage<BITS>(smem + PrefillSmem::kA + st * kBM * kBK * 2,
+                            smem + PrefillSmem::kCodeLo + cs * kBM * (kChunk / 4) + r * (kChunk / 4) + team * 16,
+                            smem + PrefillSmem::kCodeHi + cs * kBM * (kChunk / 8) + r * (kChunk / 8) + team * 8, s01,
+                            r);
+        fence_proxy_async();  // generic-proxy writes -> visible to the tensor core
+        mbar_arrive(&B->a_full[st]);
         mbar_arrive(&B->c_empty[cs]);
       }
       if (!ok) break;
       mbar_arrive(&B->s_empty[sb]);
     }
-  } else {
+  } else if (warp >= 10 && warp < 14) {
     // ---------------------------------------------------------- epilogue
     const int q = warp & 3;            // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;       // accumulator lane = weight row of the tile
-    const int et = threadIdx.x - 192;  // 0..127 among the epilogue threads
+    const int et = threadIdx.x - 320;  // 0..127 among the epilogue threads
     int it = 0;
-    for (int w = blockIdx.x; w < total && !aborted(B); w += gridDim.x, ++it) {
-      const Item I = decode_item(P, w);
+    int4 next = blockIdx.x < total ? __ldg(P.tile_info + blockIdx.x / P.m_tiles) : make_int4(0, 0, 0, 0);
+    for (int w = blockIdx.x; w < total && !aborted(B); w += G, ++it) {
+      const int4 info = next;
+      if (w + G < total) next = __ldg(P.tile_info + (w + G) / P.m_tiles);
+      const int m = w % P.m_tiles, row0 = info.y, rows = info.z;
       const int acc = it & 1;
-      if (!wait_bar(B, &B->d_full[acc], (it >> 1) & 1, deadline, P.status, 10)) break;
+      if (!wait_bar(B, &B->d_full[acc], (it >> 1) & 1, limit, P.status, 10)) break;
       tc_fence_after();
       const uint32_t base = tmem + static_cast<uint32_t>(acc * kBN) + (static_cast<uint32_t>(q * 32) << 16);
       if (!DOWN) {
-        // channel m*64 + r/2: gate on the even lane, up on the odd one
+        // channel m*64 + r/2 (gate on the even lane, up on the odd one),
+        // stored at its permuted position inside its group of 16
+        const int lc = r >> 1;
+        const int lp = (lc & ~15) | k_position(lc & 15);
         __half* hs = reinterpret_cast<__half*>(smem + PrefillSmem::kStage);  // [kBN pairs][64 channels]
-        for (int c0 = 0; c0 < I.rows; c0 += 16) {
+        for (int c0 = 0; c0 < rows; c0 += 16) {
           float v[16];
           tmem_ld16(base + c0, v);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float u = __shfl_xor_sync(0xffffffffu, v[i], 1);
-            if ((lane & 1) == 0 && c0 + i < I.rows)
-              hs[(c0 + i) * 64 + (r >> 1)] = __float2half_rn(v[i] / (1.f + expf(-v[i])) * u);
+            if ((lane & 1) == 0 && c0 + i < rows)
+              hs[(c0 + i) * 64 + lp] = __float2half_rn(v[i] / (1.f + expf(-v[i])) * u);
           }
         }
         tc_fence_before();
         mbar_arrive(&B->d_empty[acc]);
         named_sync(2, 128);
         __half* out = static_cast<__half*>(P.out);
-        for (int e = et; e < I.rows * 8; e += 128) {  // 128 bytes (64 channels) per pair row
+        for (int e = et; e < rows * 8; e += 128) {  // 128 bytes (64 channels) per pair row
           const int row = e >> 3, ch = (e & 7) * 8;
-          *reinterpret_cast<uint4*>(out + static_cast<size_t>(I.row0 + row) * P.ld_out + I.m * 64 + ch) =
+          *reinterpret_cast<uint4*>(out + static_cast<size_t>(row0 + row) * P.ld_out + m * 64 + ch) =
               *reinterpret_cast<const uint4*>(hs + row * 64 + ch);
         }
         named_sync(2, 128);
@@ -459,21 +484,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB, const __grid_constan
         // output dim m*128 + r, 32 pairs at a time through the staging tile
         float* zs = reinterpret_cast<float*>(smem + PrefillSmem::kStage);  // [32 pairs][128 dims]
         float* out = static_cast<float*>(P.out);
-        for (int c0 = 0; c0 < I.rows; c0 += 32) {
+        for (int c0 = 0; c0 < rows; c0 += 32) {
           float v[32];
           tmem_ld16(base + c0, v);
           tmem_ld16(base + c0 + 16, v + 16);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const int p = I.row0 + c0 + i;
-            const float gt = (c0 + i < I.rows && p < P.n_pairs) ? __ldg(P.pair_gate + p) : 1.f;
+            const int p = row0 + c0 + i;
+            const float gt = (c0 + i < rows && p < P.n_pairs) ? __ldg(P.pair_gate + p) : 1.f;
             zs[i * 128 + r] = gt * v[i];
           }
           named_sync(2, 128);
-          const int nrow = min(32, I.rows - c0);
+          const int nrow = min(32, rows - c0);
           for (int e = et; e < nrow * 32; e += 128) {
             const int row = e >> 5, col = (e & 31) * 4;
-            *reinterpret_cast<float4*>(out + static_cast<size_t>(I.row0 + c0 + row) * P.ld_out + I.m * kBM + col) =
+            *reinterpret_cast<float4*>(out + static_cast<size_t>(row0 + c0 + row) * P.ld_out + m * kBM + col) =
                 *reinterpret_cast<const float4*>(zs + row * 128 + col);
           }
           named_sync(2, 128);
@@ -494,7 +519,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB, const __grid_constan
 
 // ------------------------------------------------------------------ x gather (bf16 -> fp16 rows in pair order)
 // Row r < n_pairs is token pair_token[r]; rows n_pairs .. n_rows-1 are the
-// shared expert's rows, token r - n_pairs.
+// shared expert's rows, token r - n_pairs. Inside every group of 16 columns
+// the row is stored in the permuted K order: position 2i <- column i,
+// position 2i+1 <- column i+8.
 __global__ void __launch_bounds__(256) gather_x_kernel(const uint16_t* __restrict__ x,
                                                        const int32_t* __restrict__ pair_token, int n_pairs,
                                                        int n_rows, int d, __half* __restrict__ xg) {
@@ -503,17 +530,37 @@ __global__ void __launch_bounds__(256) gather_x_kernel(const uint16_t* __restric
   const int t = r < n_pairs ? __ldg(pair_token + r) : r - n_pairs;
   const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
   uint4* dst = reinterpret_cast<uint4*>(xg + static_cast<size_t>(r) * d);
-  for (int i = threadIdx.x; i < d / 8; i += blockDim.x) {
-    const uint4 v = __ldg(src + i);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
+  for (int gi = threadIdx.x; gi < d / 16; gi += blockDim.x) {
+    const uint4 a = __ldg(src + 2 * gi), b = __ldg(src + 2 * gi + 1);  // columns 16gi .. +7, +8 .. +15
+    const uint32_t lo[4] = {a.x, a.y, a.z, a.w}, hi[4] = {b.x, b.y, b.z, b.w};
+    uint32_t o[8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const __half2 h = __floats2half2_rn(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u));
-      o[j] = *reinterpret_cast<const uint32_t*>(&h);
+    for (int i = 0; i < 8; ++i) {  // (column i, column i+8) as one fp16 pair
+      const uint32_t xi = (i & 1) ? (lo[i >> 1] & 0xffff0000u) : (lo[i >> 1] << 16);
+      const uint32_t xj = (i & 1) ? (hi[i >> 1] & 0xffff0000u) : (hi[i >> 1] << 16);
+      const __half2 h = __floats2half2_rn(__uint_as_float(xi), __uint_as_float(xj));
+      o[i] = *reinterpret_cast<const uint32_t*>(&h);
     }
-    dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[2 * gi] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[2 * gi + 1] = make_uint4(o[4], o[5], o[6], o[7]);
   }
+}
+
+// Token-tile table: for every extended expert x (routed 0..E-1, shared = E)
+// and each of its ceil(n_x / 128) token tiles, {x, first sorted row, rows,
+// pool slot}, at index tile_offset[x] + i.
+__global__ void __launch_bounds__(256) tile_table_kernel(const int32_t* __restrict__ tile_offset,
+                                                         const int32_t* __restrict__ expert_offset,
+                                                         const int32_t* __restrict__ expert_count,
+                                                         const int32_t* __restrict__ pair_slot, int E, int T,
+                                                         int n_pairs, int has_shared, int4* __restrict__ info) {
+  const int x = blockIdx.x * blockDim.x + threadIdx.x;
+  if (x > E) return;
+  const int n = x < E ? expert_count[x] : (has_shared ? T : 0);
+  const int base = x < E ? expert_offset[x] : n_pairs;
+  const int slot = (x < E && n > 0) ? pair_slot[base] : 0;
+  const int t0 = tile_offset[x];
+  for (int i = 0; i * kBN < n; ++i) info[t0 + i] = make_int4(x, base + i * kBN, min(kBN, n - i * kBN), slot);
 }
 
 // ------------------------------------------------------------------ tensor maps (host)
@@ -546,12 +593,12 @@ bool map_codes(CUtensorMap* m, const uint8_t* base, size_t row_bytes, int rows, 
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2-D fp16 activation tensor [rows][K], boxes of 64 x 128 with the 128-byte
-// swizzle; rows past the end read as zeros.
-bool map_act(CUtensorMap* m, const __half* base, int K, int rows) {
+// 2-D fp16 activation tensor [rows][K], boxes of 64 x box_rows with the
+// 128-byte swizzle; rows past the end read as zeros.
+bool map_act(CUtensorMap* m, const __half* base, int K, int rows, int box_rows) {
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kBN)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t es[2] = {1u, 1u};
   return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -565,12 +612,13 @@ cudaError_t run_pass(const Ctx& ctx, const FfnArgs& a, GemmParams P, const __hal
                      size_t codes_off, size_t scales_off, cudaStream_t s) {
   const size_t row_b = static_cast<size_t>(K) * BITS / 8;
   const uint8_t* shr = a.shared != nullptr ? a.shared : a.pool;  // keeps the shared maps well formed
-  CUtensorMap maps[5];
-  bool ok = map_act(&maps[0], act, K, n_rows);
-  ok = ok && map_codes(&maps[1], a.pool + codes_off, row_b, rows, a.stride, kMapSlots, kChunk / 4);
-  ok = ok && map_codes(&maps[2], a.pool + codes_off, row_b, rows, a.stride, kMapSlots, kChunk / 8);
-  ok = ok && map_codes(&maps[3], shr + codes_off, row_b, rows, a.stride, 1, kChunk / 4);
-  ok = ok && map_codes(&maps[4], shr + codes_off, row_b, rows, a.stride, 1, kChunk / 8);
+  CUtensorMap maps[8];
+  bool ok = true;
+  for (int i = 0; i < 4; ++i) ok = ok && map_act(&maps[i], act, K, n_rows, 16 << i);
+  ok = ok && map_codes(&maps[4], a.pool + codes_off, row_b, rows, a.stride, kMapSlots, kChunk / 4);
+  ok = ok && map_codes(&maps[5], a.pool + codes_off, row_b, rows, a.stride, kMapSlots, kChunk / 8);
+  ok = ok && map_codes(&maps[6], shr + codes_off, row_b, rows, a.stride, 1, kChunk / 4);
+  ok = ok && map_codes(&maps[7], shr + codes_off, row_b, rows, a.stride, 1, kChunk / 8);
   if (!ok) return cudaErrorInvalidValue;
   P.K = K;
   P.m_tiles = rows / kBM;
@@ -588,23 +636,21 @@ cudaError_t run_pass(const Ctx& ctx, const FfnArgs& a, GemmParams P, const __hal
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<BITS, DOWN>, maps[0], maps[1], maps[2], maps[3], maps[4], P);
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<BITS, DOWN>, maps[0], maps[1], maps[2], maps[3], maps[4],
+                            maps[5], maps[6], maps[7], P);
 }
 
 template <int BITS>
-cudaError_t run_ffn(const Ctx& ctx, const moe_layer_cfg& c, const FfnArgs& a, __half* xg, __half* h16,
-                    float* z_rows, int n_pairs, int n_rows, cudaStream_t s) {
+cudaError_t run_ffn(const Ctx& ctx, const moe_layer_cfg& c, const FfnArgs& a, const int4* info, __half* xg,
+                    __half* h16, float* z_rows, int n_pairs, int n_rows, cudaStream_t s) {
   GemmParams P{};
+  P.tile_info = info;
   P.tile_offset = a.g->tile_offset;
-  P.expert_offset = a.g->expert_offset;
-  P.expert_count = a.g->expert_count;
-  P.pair_slot = a.g->pair_slot;
   P.pair_gate = a.g->pair_gate;
   P.pool = a.pool;
   P.shared = a.shared;
   P.stride = a.stride;
   P.E = c.E;
-  P.T = a.T;
   P.n_pairs = n_pairs;
   P.status = a.status;
   P.timeout_ns = ctx.timeout_ns;
@@ -648,11 +694,16 @@ cudaError_t launch_ffn_prefill(const Ctx& ctx, const moe_layer_cfg& c, const Ffn
   char* b = static_cast<char*>(ws);
   __half* xg = reinterpret_cast<__half*>(b + w.x16);
   __half* h16 = reinterpret_cast<__half*>(b + w.h);
+  int4* info = reinterpret_cast<int4*>(b + w.tile_info);
 
-  gather_x_kernel<<<w.n_rows, 256, 0, s>>>(a.x, a.g->pair_token, w.n_pairs, w.n_rows, c.d, xg);
+  tile_table_kernel<<<(c.E + 1 + 255) / 256, 256, 0, s>>>(a.g->tile_offset, a.g->expert_offset, a.g->expert_count,
+                                                           a.g->pair_slot, c.E, a.T, w.n_pairs, a.shared != nullptr,
+                                                           info);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  return c.bits == 2 ? run_ffn<2>(ctx, c, a, xg, h16, z_rows, w.n_pairs, w.n_rows, s)
-                     : run_ffn<3>(ctx, c, a, xg, h16, z_rows, w.n_pairs, w.n_rows, s);
+  gather_x_kernel<<<w.n_rows, 128, 0, s>>>(a.x, a.g->pair_token, w.n_pairs, w.n_rows, c.d, xg);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return c.bits == 2 ? run_ffn<2>(ctx, c, a, info, xg, h16, z_rows, w.n_pairs, w.n_rows, s)
+                     : run_ffn<3>(ctx, c, a, info, xg, h16, z_rows, w.n_pairs, w.n_rows, s);
 }
 
 }  // namespace moe

@@ -18,6 +18,10 @@ constexpr int kMaxE = 1024;           // experts per layer
 constexpr int kMaxK = 32;             // experts per token
 constexpr int kGroupChunk = 512;      // pairs per chunk in the multi-CTA grouping
 constexpr int kTileN = 128;           // tokens per tile of the prefill grouped GEMM
+// Copies of the small arrays every CTA of the decode kernel reads (logits,
+// slots, h): CTA b reads copy b % kRep, so each cache line has ~148/kRep
+// readers instead of all of them.
+constexpr int kRep = 8;
 
 // Device status word codes (word 0 holds the first error seen).
 constexpr int kDevBadExpert = 1;
@@ -51,7 +55,9 @@ struct WsLayout {
   size_t expert_count, expert_offset, pair_token, pair_j, pair_gate, pair_slot, pair_pos;
   size_t uniq_expert, uniq_slot, uniq_offset, n_uniq;
   size_t chunk_hist, tile_offset;
+  size_t logits_rep, slot_rep;  // decode path: kRep copies of [T, E] logits and [E] slots
   size_t h, z, x16;
+  size_t tile_info;              // prefill: int4 per token tile
   size_t total;
   int n_pairs, n_rows, n_chunks, n_uniq_max;
 };
@@ -124,7 +130,9 @@ struct DecodeArgs {
   size_t stride;
   const uint8_t* shared;    // record or null
   moe_expert_layout lay;
-  float* h;                 // fp32 [n_rows, f]
+  float* h;                 // fp32 [kRep][n_rows, f]
+  float* logits_rep;        // route: [kRep][T, E]
+  int32_t* slot_rep;        // route: [kRep][E]
   void* y;
 };
 cudaError_t launch_decode_layer(const Ctx& ctx, const moe_layer_cfg& c, const DecodeArgs& a, cudaStream_t s);

@@ -16,7 +16,7 @@
 namespace {
 
 // Largest workspace the static variant serves (moe_workspace_bytes(cfg, T)):
-// the full-size layer (d=2048, f=768, E=512, k=10) needs about 0.72 MB at
+// the full-size layer (d=2048, f=768, E=512, k=10) needs about 2.7 MB at
 // T = 8.
 constexpr size_t kStaticScratchBytes = MOE_STATIC_SCRATCH_BYTES;
 static_assert(kStaticScratchBytes % 256 == 0, "scratch size");

@@ -229,8 +229,8 @@ MOE_API moe_status moe_layer_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, con
  *   - Arguments and results as moe_layer_forward, minus ws / ws_bytes.
  *   - Limit: moe_workspace_bytes(cfg, T) must be <= MOE_STATIC_SCRATCH_BYTES,
  *     else MOE_ENOSPACE and nothing runs. The full-size layer (d=2048,
- *     f=768, E=512, k=10) needs about 0.72 MB at T = 8, so every decode
- *     batch fits; at that size prefill chunks above about a dozen tokens
+ *     f=768, E=512, k=10) needs about 2.7 MB at T = 8, so every decode
+ *     batch fits; at that size prefill chunks above about two dozen tokens
  *     do not.
  *   - Nothing in the scratch needs to start at zero.
  *   - There is ONE scratch per device, shared by every context and stream:
@@ -240,7 +240,7 @@ MOE_API moe_status moe_layer_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, con
  *   - The first call on a device does a one-time set-up (it looks up the
  *     array's device address with that device current); make that first
  *     call before any stream capture begins. */
-#define MOE_STATIC_SCRATCH_BYTES (2u << 20)
+#define MOE_STATIC_SCRATCH_BYTES (4u << 20)
 MOE_API moe_status moe_layer_forward_static(moe_ctx* ctx, const moe_layer_cfg* cfg, const void* x, int T,
                                     const float* w_router, const float* logit_bias,
                                     const int32_t* slot_of, int n_slots, const uint8_t* slot_pool,

@@ -38,7 +38,7 @@ def test_static_scratch_matches_workspace_path(cfg, T, zipf):
 
 def test_static_scratch_rejects_workspaces_beyond_its_size():
     T = 64  # the full-size layer needs ~11 MB of scratch here
-    assert M.workspace_bytes(M.FULL, T) > 2 << 20
+    assert M.workspace_bytes(M.FULL, T) > 4 << 20
     L = H.Layer(M.FULL, T, seed=32)
     y = L.out_tensor()
     assert _static(L, M.FULL, y) == M.ENOSPACE
