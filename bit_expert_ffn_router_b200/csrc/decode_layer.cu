@@ -289,8 +289,16 @@ __device__ void stage_issue(DLShared* S, const StageRec& s, int i, uint8_t* ring
 }
 
 // ------------------------------------------------------------------ consumers
+// The quantisers below walk their jobs in warp-sized steps, kQD steps at a
+// time: all loads of a group are issued before any value is used, so a group
+// costs about one memory round trip (at T = 1 one group covers all h rows a
+// CTA needs). A step past the end is skipped as a whole (the test is uniform
+// across the warp); inside the last step, idle lanes read a clamped, valid
+// address, so no single load carries a guard.
+constexpr int kQD = 3;
+
 // Quantises the T token rows of x (bf16, global) into the gate/up layout,
-// four lanes per 32-value block. Loops run in whole warps (shuffles).
+// four lanes per 32-value block, and keeps the raw rows in xs for the router.
 template <int BITS>
 __device__ void quantise_x(const DLParams& P, int* xq, uint16_t* xs, int nct) {
   const int nb = P.d / kBlock, bpl = nb / P.gu_lpr;
@@ -298,41 +306,68 @@ __device__ void quantise_x(const DLParams& P, int* xq, uint16_t* xs, int nct) {
   const int jobs = P.T * nb;
   const int q = threadIdx.x & 3;
 #pragma unroll 1
-  for (int base = threadIdx.x & ~31; base < jobs * 4; base += nct) {
-    const int job = (base + (threadIdx.x & 31)) >> 2;
-    const bool live = job < jobs;
-    const int t = live ? job / nb : 0, blk = live ? job % nb : 0;
-    const size_t at = static_cast<size_t>(t) * P.d + blk * kBlock + q;
-    float v[8];
+  for (int base0 = threadIdx.x & ~31; base0 < jobs * 4; base0 += kQD * nct) {
+    uint16_t bits[kQD][8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint16_t bits = live ? __ldcg(P.x + at + 4 * k) : uint16_t(0);
-      if (live) xs[at + 4 * k] = bits;
-      v[k] = bf16_bits_to_float(bits);
+    for (int g = 0; g < kQD; ++g) {
+      if (base0 + g * nct >= jobs * 4) break;
+      const int job = min((base0 + g * nct + (threadIdx.x & 31)) >> 2, jobs - 1);
+      const size_t a = static_cast<size_t>(job / nb) * P.d + (job % nb) * kBlock + q;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) bits[g][k] = __ldcg(P.x + a + 4 * k);
     }
-    const int gl = blk / bpl, bb = blk % bpl;
-    quant_quad<BITS>(v, xq + t * words, nb, bb * P.gu_lpr + gl, q, live);
+#pragma unroll
+    for (int g = 0; g < kQD; ++g) {
+      const int base = base0 + g * nct;  // warp-uniform
+      if (base >= jobs * 4) break;
+      const int job = (base + (threadIdx.x & 31)) >> 2;
+      const bool live = job < jobs;
+      const int t = live ? job / nb : 0, blk = live ? job % nb : 0;
+      const size_t at = static_cast<size_t>(t) * P.d + blk * kBlock + q;
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (live) xs[at + 4 * k] = bits[g][k];
+        v[k] = live ? bf16_bits_to_float(bits[g][k]) : 0.f;
+      }
+      const int gl = blk / bpl, bb = blk % bpl;
+      quant_quad<BITS>(v, xq + t * words, nb, bb * P.gu_lpr + gl, q, live);
+    }
   }
 }
 
-// Quantises h rows [lo, hi) (fp32, global) into the down layout.
+// Quantises h rows [lo, hi) (fp32, global; this CTA's copy) into the down layout.
 template <int BITS>
 __device__ void quantise_h(const DLParams& P, int lo, int hi, int* hq, int nct) {
   const int nb = P.f / kBlock, bpl = nb / P.dn_lpr;
   const int words = QV<BITS>::kWords * nb;
   const int jobs = (hi - lo) * nb;
   const int q = threadIdx.x & 3;
+  const float* hb = P.h + (blockIdx.x % kRep) * P.h_rep;
 #pragma unroll 1
-  for (int base = threadIdx.x & ~31; base < jobs * 4; base += nct) {
-    const int job = (base + (threadIdx.x & 31)) >> 2;
-    const bool live = job < jobs;
-    const int r = live ? job / nb : 0, blk = live ? job % nb : 0;
-    const float* src = P.h + (blockIdx.x % kRep) * P.h_rep + static_cast<size_t>(lo + r) * P.f + blk * kBlock + q;
-    float v[8];
+  for (int base0 = threadIdx.x & ~31; base0 < jobs * 4; base0 += kQD * nct) {
+    float vals[kQD][8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = live ? __ldcg(src + 4 * k) : 0.f;
-    const int gl = blk / bpl, bb = blk % bpl;
-    quant_quad<BITS>(v, hq + r * words, nb, bb * P.dn_lpr + gl, q, live);
+    for (int g = 0; g < kQD; ++g) {
+      if (base0 + g * nct >= jobs * 4) break;
+      const int job = min((base0 + g * nct + (threadIdx.x & 31)) >> 2, jobs - 1);
+      const float* src = hb + static_cast<size_t>(lo + job / nb) * P.f + (job % nb) * kBlock + q;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) vals[g][k] = __ldcg(src + 4 * k);
+    }
+#pragma unroll
+    for (int g = 0; g < kQD; ++g) {
+      const int base = base0 + g * nct;  // warp-uniform
+      if (base >= jobs * 4) break;
+      const int job = (base + (threadIdx.x & 31)) >> 2;
+      const bool live = job < jobs;
+      const int r = live ? job / nb : 0, blk = live ? job % nb : 0;
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = live ? vals[g][k] : 0.f;
+      const int gl = blk / bpl, bb = blk % bpl;
+      quant_quad<BITS>(v, hq + r * words, nb, bb * P.dn_lpr + gl, q, live);
+    }
   }
 }
 
@@ -511,12 +546,14 @@ __device__ void topk_warp(const DLParams& P, const RouteSmem& R, int t, unsigned
   constexpr int VPL = 16;
   const int lane = threadIdx.x & 31;
   const float* row = P.logits_rep + (static_cast<size_t>(blockIdx.x % kRep) * P.T + t) * P.E;
+  // every load is issued before any is used: the index is clamped into the
+  // row, so the loads need no guard and their latencies overlap
+  float lv[VPL];
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) lv[v] = __ldcg(row + min(v * 32 + lane, P.E - 1));
   uint32_t key[VPL];
 #pragma unroll
-  for (int v = 0; v < VPL; ++v) {
-    const int e = v * 32 + lane;
-    key[v] = e < P.E ? order_key(__ldcg(row + e)) : 0u;
-  }
+  for (int v = 0; v < VPL; ++v) key[v] = v * 32 + lane < P.E ? order_key(lv[v]) : 0u;
   if (tr != nullptr && lane == 0) {
     uint32_t any = 0u;
 #pragma unroll
@@ -601,7 +638,7 @@ __device__ void topk_warp(const DLParams& P, const RouteSmem& R, int t, unsigned
   if (P.renorm) {
     denom = warp_sum(ex);
   } else {
-    float s = 0.f;
+    float s = 0.f;  // full-softmax denominator (re-read: keeps the logits out of registers above)
     for (int e = lane; e < P.E; e += 32) s += expf(__ldcg(row + e) - l0);
     denom = warp_sum(s);
   }
@@ -627,6 +664,8 @@ __device__ void router_rows(const DLParams& P, const float* wrs, const uint16_t*
 #pragma unroll 1
     for (int e = e0 + warp; e < e1; e += cw) {
       const float4* w4 = reinterpret_cast<const float4*>(wrs + static_cast<size_t>(e - e0) * P.d);
+      const size_t o = static_cast<size_t>(t) * P.E + e;
+      const float bv = P.bias != nullptr ? __ldcg(P.bias + o) : 0.f;  // in flight during the dot product
       float acc = 0.f;
 #pragma unroll 4
       for (int c4 = lane; c4 < n4; c4 += 32) {
@@ -638,10 +677,7 @@ __device__ void router_rows(const DLParams& P, const float* wrs, const uint16_t*
         acc = fmaf(w.w, __uint_as_float(xb.y & 0xffff0000u), acc);
       }
       acc = warp_sum(acc);
-      if (lane < kRep) {
-        const size_t o = static_cast<size_t>(t) * P.E + e;
-        P.logits_rep[lane * static_cast<size_t>(P.T) * P.E + o] = P.bias ? acc + P.bias[o] : acc;
-      }
+      if (lane < kRep) P.logits_rep[lane * static_cast<size_t>(P.T) * P.E + o] = acc + bv;
     }
   }
 }
@@ -816,6 +852,7 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
 #pragma unroll 1
   for (int i = 0;; ++i) {
     if (i == n_sh) {
+      cur_t = -1;  // the cached x row is not needed across the routing step (frees its registers)
       if (tid == 0) MOE_TRACE(3)
       if (ROUTE) {
         if (tid == 0 && !aborted(S) && !gbar_wait(P.gbar, S->bar_target, deadline)) set_abort(S, P.status, 3);

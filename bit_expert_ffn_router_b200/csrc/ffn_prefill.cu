@@ -21,9 +21,11 @@
 //               ring allows;
 //   warp 1      TMEM allocation and the single-thread tcgen05.mma issue;
 //   warps 2-9   dequantisation, two teams of four warps taking alternate
-//               64-wide K stages: each thread owns one weight row and writes
-//               s * (q - 2^(b-1)) as fp16 straight into the 128B-swizzled
-//               K-major layout the tensor core reads;
+//               128-wide K stages: each thread owns one weight row and writes
+//               s * (q - 2^(b-1)) as fp16 straight into tensor memory (its
+//               TMEM lane), where the MMA reads its A operand. The weights
+//               never pass through shared memory, whose bandwidth the
+//               activation tiles and codes already use;
 //   warps 10-13 epilogue: tcgen05.ld of the fp32 accumulators (two TMEM
 //               buffers, so the next item's MMAs overlap this item's stores).
 //
@@ -52,23 +54,24 @@ namespace {
 
 constexpr int kBM = 128;            // weight rows per tile (MMA M)
 constexpr int kBN = kTileN;         // pairs per tile (MMA N, max)
-constexpr int kBK = 64;             // K per pipeline stage (one 128-byte swizzle row of fp16)
-constexpr int kChunk = 128;         // codes per code-chunk load: one stage for each dequant team
-constexpr int kAStages = 4;         // dequantised weight ring
-constexpr int kBStages = 5;         // activation ring
-constexpr int kCStages = 4;         // code-chunk ring
+constexpr int kBK = 128;            // K per pipeline stage: 8 MMAs of K = 16
+constexpr int kSub = 64;            // K per 128-byte swizzle atom of fp16 (two per stage)
+constexpr int kStages = 4;          // ring depth: A stages (TMEM), activation slots, code chunks
 constexpr int kDqThreads = 128;     // threads per dequant team (one per weight row)
 constexpr int kThreads = 15 * 32;
-constexpr int kTmemCols = 2 * kBN;  // two accumulator buffers
+constexpr int kAccCols = 2 * kBN;   // two accumulator buffers (TMEM columns 0..255)
+constexpr int kACols = kBK / 2;     // one A stage: 128 fp16 per lane = 64 columns
+constexpr int kTmemCols = 512;      // accumulators + kStages A stages
+static_assert(kAccCols + kStages * kACols <= kTmemCols, "tensor memory budget");
 constexpr int kMaxKDim = 2048;      // largest reduction size (scale staging holds 128 x K/16 bytes)
 
 struct PrefillSmem {
   // byte offsets from the 1024-aligned base of dynamic shared memory
-  static constexpr int kA = 0;                                     // kAStages x 16 KB, 128B-swizzled
-  static constexpr int kB = kA + kAStages * kBM * kBK * 2;         // kBStages x 16 KB, 128B-swizzled
-  static constexpr int kCodeLo = kB + kBStages * kBN * kBK * 2;    // kCStages x (128 rows x 32 B)
-  static constexpr int kCodeHi = kCodeLo + kCStages * kBM * (kChunk / 4);  // kCStages x (128 x 16 B)
-  static constexpr int kScale = kCodeHi + kCStages * kBM * (kChunk / 8);   // 2 x (128 rows x K/16 B)
+  static constexpr int kSubBytes = kBN * kSub * 2;                 // one swizzled sub-tile: 16 KB
+  static constexpr int kB = 0;                                     // kStages x 2 sub-tiles
+  static constexpr int kCodeLo = kB + kStages * 2 * kSubBytes;     // kStages x (128 rows x 32 B)
+  static constexpr int kCodeHi = kCodeLo + kStages * kBM * (kBK / 4);  // kStages x (128 x 16 B)
+  static constexpr int kScale = kCodeHi + kStages * kBM * (kBK / 8);   // 2 x (128 rows x K/16 B)
   static constexpr int kScaleBuf = kBM * (kMaxKDim / kBlock) * 2;
   static constexpr int kStage = kScale + 2 * kScaleBuf;            // epilogue staging 16 KB
   static constexpr int kBar = kStage + 16384;
@@ -78,12 +81,11 @@ struct PrefillSmem {
 static_assert(PrefillSmem::kAlloc <= 227 * 1024, "shared memory budget");
 
 struct Bars {
-  uint64_t a_full[kAStages];    // dequant team -> MMA (count 128)
-  uint64_t a_empty[kAStages];   // MMA commit -> dequant team
-  uint64_t b_full[kBStages];    // TMA -> MMA (tx)
-  uint64_t b_empty[kBStages];   // MMA commit -> producer
-  uint64_t c_full[kCStages];    // TMA -> dequant (tx)
-  uint64_t c_empty[kCStages];   // both dequant teams -> producer (count 256)
+  uint64_t a_full[kStages];     // dequant team -> MMA (count 128): A stage written to TMEM
+  uint64_t b_full[kStages];     // TMA -> MMA (tx): activation slot landed
+  uint64_t st_empty[kStages];   // MMA commit -> dequant team and activation producer: A stage and slot free
+  uint64_t c_full[kStages];     // TMA -> dequant (tx): code chunk landed
+  uint64_t c_empty[kStages];    // dequant team -> weight producer (count 128)
   uint64_t s_full[2];           // bulk copy -> dequant (tx)
   uint64_t s_empty[2];          // both dequant teams -> producer (count 256)
   uint64_t d_full[2];           // MMA commit -> epilogue
@@ -130,7 +132,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -158,13 +159,30 @@ __device__ __forceinline__ uint32_t instr_desc(int n) {
   return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(kBM >> 4) << 24);
 }
 
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+// tcgen05.mma with A read from tensor memory: row m of A in TMEM lane m,
+// two fp16 K values per 32-bit column (the lower K index in the low half).
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                          uint32_t acc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
+}
+
+// 32 consecutive 32-bit columns of this thread's TMEM lane (the warp's lane
+// quarter), then wait for the stores to complete.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // 32 lanes x 16 consecutive fp32 columns of the warp's TMEM lane quarter.
@@ -196,18 +214,54 @@ __device__ __forceinline__ bool wait_bar(Bars* B, uint64_t* bar, uint32_t parity
   return false;
 }
 
+__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// For waits that are usually already satisfied (the MMA thread's): one
+// non-blocking test, then the bounded wait.
+__device__ __forceinline__ bool wait_fast(Bars* B, uint64_t* bar, uint32_t parity, uint64_t limit, int* status,
+                                          int where) {
+  return mbar_test(bar, parity) || wait_bar(B, bar, parity, limit, status, where);
+}
+
+// The abort flag as lane 0 sees it, the same for the whole warp.
+__device__ __forceinline__ bool aborted_warp(const Bars* B) {
+  return __shfl_sync(0xffffffffu, aborted(B) ? 1 : 0, 0) != 0;
+}
+
+// Warp-wide wait: lane 0 waits, the result is broadcast and the warp
+// synchronises (ordering the other lanes' later accesses after lane 0's
+// observation of the phase). Every lane then takes the same path, which the
+// warp-collective tcgen05.ld / tcgen05.st that follow require.
+__device__ __forceinline__ bool wait_bar_warp(Bars* B, uint64_t* bar, uint32_t parity, uint64_t limit, int* status,
+                                              int where) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = wait_bar(B, bar, parity, limit, status, where) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
 // ------------------------------------------------------------------ K-order permutation
 // Position of index i inside its group of 16 (inverse of: position 2i <- i,
 // position 2i+1 <- i+8).
 __host__ __device__ __forceinline__ int k_position(int i) { return i < 8 ? 2 * i : 2 * i - 15; }
 
 // ------------------------------------------------------------------ dequantisation of one K stage
-// Row r of the A tile: 64 weights s * (q - 2^(BITS-1)) as fp16 in the
-// permuted K order, 16-byte chunk j of the row at chunk position j ^ (r % 8)
-// (the 128-byte swizzle the descriptor names).
+// One weight row's 64 weights s * (q - 2^(BITS-1)) of a K stage as 32 fp16
+// pairs, in the permuted K order: word 8q + i holds (index 16q+i, index
+// 16q+i+8) of the stage.
 template <int BITS>
-__device__ __forceinline__ void dequant_stage(uint8_t* a_tile, const uint8_t* lo, const uint8_t* hi,
-                                              uint32_t s01, int r) {
+__device__ __forceinline__ void dequant_stage(uint32_t* out, const uint8_t* lo, const uint8_t* hi, uint32_t s01) {
   const uint4 w = *reinterpret_cast<const uint4*>(lo);  // 64 two-bit codes: four groups of 16
   const uint32_t wl[4] = {w.x, w.y, w.z, w.w};
   uint32_t hq[4] = {0u, 0u, 0u, 0u};
@@ -225,21 +279,17 @@ __device__ __forceinline__ void dequant_stage(uint8_t* a_tile, const uint8_t* lo
   const __half2 s1 = __half2half2(__ushort_as_half(static_cast<unsigned short>(s01 >> 16)));
   // 0x6400 | q is the fp16 number 1024 + q; subtracting 1024 + 2^(BITS-1) is exact
   const __half2 off = __float2half2_rn(1024.f + static_cast<float>(1 << (BITS - 1)));
-  uint8_t* row = a_tile + r * 128;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const __half2 s = q < 2 ? s0 : s1;
-    uint32_t out[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       uint32_t v = (wl[q] >> (2 * i)) & 0x00030003u;
       if (BITS == 3) v |= (hq[q] >> i) & 0x00040004u;
       v |= 0x64006400u;
       const __half2 y = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&v), off), s);
-      out[i] = *reinterpret_cast<const uint32_t*>(&y);
+      out[8 * q + i] = *reinterpret_cast<const uint32_t*>(&y);
     }
-    *reinterpret_cast<uint4*>(row + (((2 * q) ^ (r & 7)) * 16)) = make_uint4(out[0], out[1], out[2], out[3]);
-    *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ (r & 7)) * 16)) = make_uint4(out[4], out[5], out[6], out[7]);
   }
 }
 
@@ -257,17 +307,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB16, const __grid_const
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kAStages; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&B->a_full[i], kDqThreads);
-      mbar_init(&B->a_empty[i], 1);
-    }
-    for (int i = 0; i < kBStages; ++i) {
       mbar_init(&B->b_full[i], 1);
-      mbar_init(&B->b_empty[i], 1);
-    }
-    for (int i = 0; i < kCStages; ++i) {
+      mbar_init(&B->st_empty[i], 1);
       mbar_init(&B->c_full[i], 1);
-      mbar_init(&B->c_empty[i], 2 * kDqThreads);
+      mbar_init(&B->c_empty[i], kDqThreads);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&B->s_full[i], 1);
@@ -279,7 +324,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB16, const __grid_const
     B->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {  // TMEM: two accumulator buffers of kBN fp32 columns
+  if (warp == 1) {  // TMEM: accumulators and the A stages
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&B->tmem_base)),
                  "r"(kTmemCols)
                  : "memory");
@@ -296,8 +341,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB16, const __grid_const
   const uint64_t limit = P.timeout_ns;  // limit of each wait
   const int total = __ldg(P.tile_offset + P.E + 1) * P.m_tiles;
   const int ks_per_item = P.K / kBK;
-  const int chunks_per_item = P.K / kChunk;
-  const uint32_t code_tx = kBM * (kChunk / 4) + (BITS == 3 ? kBM * (kChunk / 8) : 0);
+  const uint32_t code_tx = kBM * (kBK / 4) + (BITS == 3 ? kBM * (kBK / 8) : 0);
   const uint32_t scale_tx = kBM * P.sc_row_bytes;
   const int G = gridDim.x;
 
@@ -314,23 +358,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB16, const __grid_const
         const CUtensorMap* mB = box == 16 ? &tB16 : box == 32 ? &tB32 : box == 64 ? &tB64 : &tB128;
         const uint32_t b_tx = static_cast<uint32_t>(box) * kBK * 2;
         for (int k = 0; k < ks_per_item; ++k, ++g) {
-          const int st = g % kBStages;
-          if (g >= kBStages && !wait_bar(B, &B->b_empty[st], ((g / kBStages) - 1) & 1, limit, P.status, 3)) {
+          const int st = g % kStages;
+          if (g >= kStages && !wait_bar(B, &B->st_empty[st], ((g / kStages) - 1) & 1, limit, P.status, 3)) {
             ok = false;
             break;
           }
+          uint8_t* slot = smem + PrefillSmem::kB + st * 2 * PrefillSmem::kSubBytes;
           mbar_arrive_expect_tx(&B->b_full[st], b_tx);
-          tma_load_2d(smem + PrefillSmem::kB + st * kBN * kBK * 2, mB, k * kBK, info.y, &B->b_full[st]);
+          tma_load_2d(slot, mB, k * kBK, info.y, &B->b_full[st]);
+          tma_load_2d(slot + PrefillSmem::kSubBytes, mB, k * kBK + kSub, info.y, &B->b_full[st]);
         }
       }
       // every copy this thread issued lands before the CTA may exit (bounded wait)
       const uint64_t drain = global_timer_ns() + P.timeout_ns;
-      for (int n = max(0, g - kBStages); n < g; ++n) mbar_wait(&B->b_full[n % kBStages], (n / kBStages) & 1, drain);
+      for (int n = max(0, g - kStages); n < g; ++n) mbar_wait(&B->b_full[n % kStages], (n / kStages) & 1, drain);
     }
   } else if (warp == 14) {
     // ---------------------------------------------------------- weight producer
     if (lane == 0) {
-      int gc = 0, it = 0;
+      int g = 0, it = 0;
       int4 next = blockIdx.x < total ? __ldg(P.tile_info + blockIdx.x / P.m_tiles) : make_int4(0, 0, 0, 0);
       for (int w = blockIdx.x; w < total && !aborted(B); w += G, ++it) {
         const int4 info = next;
@@ -347,23 +393,23 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB16, const __grid_const
         bulk_g2s(smem + PrefillSmem::kScale + sb * PrefillSmem::kScaleBuf,
                  rec + P.scale_off + static_cast<size_t>(m) * scale_tx, scale_tx, &B->s_full[sb]);
         bool ok = true;
-        for (int c = 0; c < chunks_per_item; ++c, ++gc) {
-          const int cs = gc % kCStages;
-          if (gc >= kCStages && !wait_bar(B, &B->c_empty[cs], ((gc / kCStages) - 1) & 1, limit, P.status, 2)) {
+        for (int k = 0; k < ks_per_item; ++k, ++g) {
+          const int st = g % kStages;
+          if (g >= kStages && !wait_bar(B, &B->c_empty[st], ((g / kStages) - 1) & 1, limit, P.status, 2)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&B->c_full[cs], code_tx);
-          tma_load_3d(smem + PrefillSmem::kCodeLo + cs * kBM * (kChunk / 4), mLo, c * (kChunk / 4), m * kBM, slot,
-                      &B->c_full[cs]);
+          mbar_arrive_expect_tx(&B->c_full[st], code_tx);
+          tma_load_3d(smem + PrefillSmem::kCodeLo + st * kBM * (kBK / 4), mLo, k * (kBK / 4), m * kBM, slot,
+                      &B->c_full[st]);
           if (BITS == 3)
-            tma_load_3d(smem + PrefillSmem::kCodeHi + cs * kBM * (kChunk / 8), mHi, P.hi_col0 + c * (kChunk / 8),
-                        m * kBM, slot, &B->c_full[cs]);
+            tma_load_3d(smem + PrefillSmem::kCodeHi + st * kBM * (kBK / 8), mHi, P.hi_col0 + k * (kBK / 8),
+                        m * kBM, slot, &B->c_full[st]);
         }
         if (!ok) break;
       }
       const uint64_t drain = global_timer_ns() + P.timeout_ns;
-      for (int n = max(0, gc - kCStages); n < gc; ++n) mbar_wait(&B->c_full[n % kCStages], (n / kCStages) & 1, drain);
+      for (int n = max(0, g - kStages); n < g; ++n) mbar_wait(&B->c_full[n % kStages], (n / kStages) & 1, drain);
       for (int n = max(0, it - 2); n < it; ++n) mbar_wait(&B->s_full[n & 1], (n >> 1) & 1, drain);
     }
   } else if (warp == 1) {
@@ -377,25 +423,26 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB16, const __grid_const
         const int n = (info.z + 15) / 16 * 16;
         const uint32_t idesc = instr_desc(n);
         const int acc = it & 1;
-        if (it >= 2 && !wait_bar(B, &B->d_empty[acc], ((it >> 1) - 1) & 1, limit, P.status, 4)) break;
+        if (it >= 2 && !wait_fast(B, &B->d_empty[acc], ((it >> 1) - 1) & 1, limit, P.status, 4)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kBN);
         bool ok = true;
         for (int k = 0; k < ks_per_item; ++k, ++g) {
-          const int sa = g % kAStages, sbb = g % kBStages;
-          if (!wait_bar(B, &B->a_full[sa], (g / kAStages) & 1, limit, P.status, 5) ||
-              !wait_bar(B, &B->b_full[sbb], (g / kBStages) & 1, limit, P.status, 6)) {
+          const int st = g % kStages;
+          const uint32_t ph = (g / kStages) & 1;
+          if (!wait_fast(B, &B->a_full[st], ph, limit, P.status, 5) ||
+              !wait_fast(B, &B->b_full[st], ph, limit, P.status, 6)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t da = smem_desc(smem + PrefillSmem::kA + sa * kBM * kBK * 2);
-          const uint64_t db = smem_desc(smem + PrefillSmem::kB + sbb * kBN * kBK * 2);
+          const uint32_t ta = tmem + static_cast<uint32_t>(kAccCols + st * kACols);
+          const uint8_t* slot = smem + PrefillSmem::kB + st * 2 * PrefillSmem::kSubBytes;
+          const uint64_t db0 = smem_desc(slot), db1 = smem_desc(slot + PrefillSmem::kSubBytes);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)  // K = 16 per MMA: 32 bytes = 2 descriptor units
-            tc_mma(d_tmem, da + 2 * kk, db + 2 * kk, idesc, (k > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(&B->a_empty[sa]);
-          tc_commit(&B->b_empty[sbb]);
+          for (int kk = 0; kk < kBK / 16; ++kk)  // K = 16 per MMA: 8 TMEM columns of A, 32 bytes of B
+            tc_mma_ts(d_tmem, ta + 8 * kk, (kk < 4 ? db0 : db1) + 2 * (kk & 3), idesc, (k > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&B->st_empty[st]);
         }
         if (!ok) break;
         tc_commit(&B->d_full[acc]);
@@ -406,35 +453,36 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB16, const __grid_const
     }
   } else if (warp >= 2 && warp < 10) {
     // ---------------------------------------------------------- dequantisation
-    const int team = (warp - 2) >> 2;          // stages 2c + team of code chunk c
-    const int r = (threadIdx.x - 64) & 127;    // weight row of the tile
-    int g = 0, gc = 0, it = 0;
-    for (int w = blockIdx.x; w < total && !aborted(B); w += G, ++it) {
+    const int team = (warp - 2) >> 2;          // takes the stages g with g % 2 == team
+    const int r = 32 * (warp & 3) + lane;      // weight row of the tile = this thread's TMEM lane
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+    int g = 0, it = 0;
+    for (int w = blockIdx.x; w < total && !aborted_warp(B); w += G, ++it) {
       const int sb = it & 1;
-      if (!wait_bar(B, &B->s_full[sb], (it >> 1) & 1, limit, P.status, 7)) break;
+      if (!wait_bar_warp(B, &B->s_full[sb], (it >> 1) & 1, limit, P.status, 7)) break;
       const uint8_t* sc = smem + PrefillSmem::kScale + sb * PrefillSmem::kScaleBuf + r * P.sc_row_bytes;
       bool ok = true;
-      for (int c = 0; c < chunks_per_item; ++c, ++gc, g += kChunk / kBK) {
-        const int cs = gc % kCStages;
-        if (!wait_bar(B, &B->c_full[cs], (gc / kCStages) & 1, limit, P.status, 8)) {
+      for (int k = 0; k < ks_per_item; ++k, ++g) {
+        if ((g & 1) != team) continue;
+        const int st = g % kStages;
+        if (!wait_bar_warp(B, &B->c_full[st], (g / kStages) & 1, limit, P.status, 8) ||
+            (g >= kStages && !wait_bar_warp(B, &B->st_empty[st], ((g / kStages) - 1) & 1, limit, P.status, 9))) {
           ok = false;
           break;
         }
-        const int gt = g + team;  // this team's stage
-        const int st = gt % kAStages;
-        if (gt >= kAStages && !wait_bar(B, &B->a_empty[st], ((gt / kAStages) - 1) & 1, limit, P.status, 9)) {
-          ok = false;
-          break;
-        }
-        // scales of blocks 4c + 2*team and 4c + 2*team + 1
-        const uint32_t s01 = *reinterpret_cast<const uint32_t*>(sc + 8 * c + 4 * team);
-        dequant_stage<BITS>(smem + PrefillSmem::kA + st * kBM * kBK * 2,
-                            smem + PrefillSmem::kCodeLo + cs * kBM * (kChunk / 4) + r * (kChunk / 4) + team * 16,
-                            smem + PrefillSmem::kCodeHi + cs * kBM * (kChunk / 8) + r * (kChunk / 8) + team * 8, s01,
-                            r);
-        fence_proxy_async();  // generic-proxy writes -> visible to the tensor core
+        tc_fence_after();
+        const uint2 s4 = *reinterpret_cast<const uint2*>(sc + 8 * k);  // scales of the stage's 4 blocks
+        const uint8_t* lo = smem + PrefillSmem::kCodeLo + st * kBM * (kBK / 4) + r * (kBK / 4);
+        const uint8_t* hi = smem + PrefillSmem::kCodeHi + st * kBM * (kBK / 8) + r * (kBK / 8);
+        const uint32_t ta = lane_addr + static_cast<uint32_t>(kAccCols + st * kACols);
+        uint32_t a_half[kACols / 2];
+        dequant_stage<BITS>(a_half, lo, hi, s4.x);  // K 0..63 of the stage
+        tmem_st32(ta, a_half);
+        dequant_stage<BITS>(a_half, lo + 16, hi + 8, s4.y);  // K 64..127
+        tmem_st32(ta + kACols / 2, a_half);
+        tc_fence_before();  // the stores are complete; order them before the arrival
         mbar_arrive(&B->a_full[st]);
-        mbar_arrive(&B->c_empty[cs]);
+        mbar_arrive(&B->c_empty[st]);
       }
       if (!ok) break;
       mbar_arrive(&B->s_empty[sb]);
@@ -446,12 +494,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB16, const __grid_const
     const int et = threadIdx.x - 320;  // 0..127 among the epilogue threads
     int it = 0;
     int4 next = blockIdx.x < total ? __ldg(P.tile_info + blockIdx.x / P.m_tiles) : make_int4(0, 0, 0, 0);
-    for (int w = blockIdx.x; w < total && !aborted(B); w += G, ++it) {
+    for (int w = blockIdx.x; w < total && !aborted_warp(B); w += G, ++it) {
       const int4 info = next;
       if (w + G < total) next = __ldg(P.tile_info + (w + G) / P.m_tiles);
       const int m = w % P.m_tiles, row0 = info.y, rows = info.z;
       const int acc = it & 1;
-      if (!wait_bar(B, &B->d_full[acc], (it >> 1) & 1, limit, P.status, 10)) break;
+      if (!wait_bar_warp(B, &B->d_full[acc], (it >> 1) & 1, limit, P.status, 10)) break;
       tc_fence_after();
       const uint32_t base = tmem + static_cast<uint32_t>(acc * kBN) + (static_cast<uint32_t>(q * 32) << 16);
       if (!DOWN) {
@@ -485,15 +533,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB16, const __grid_const
         float* zs = reinterpret_cast<float*>(smem + PrefillSmem::kStage);  // [32 pairs][128 dims]
         float* out = static_cast<float*>(P.out);
         for (int c0 = 0; c0 < rows; c0 += 32) {
+          // lane i fetches the gate of pair c0 + i (one coalesced load; the
+          // shared expert's rows and rows past the tile take gate 1)
+          const int pl = row0 + c0 + lane;
+          const float g_l = __ldg(P.pair_gate + min(pl, P.n_pairs - 1));
+          const float gate_l = (c0 + lane < rows && pl < P.n_pairs) ? g_l : 1.f;
           float v[32];
           tmem_ld16(base + c0, v);
           tmem_ld16(base + c0 + 16, v + 16);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int p = row0 + c0 + i;
-            const float gt = (c0 + i < rows && p < P.n_pairs) ? __ldg(P.pair_gate + p) : 1.f;
-            zs[i * 128 + r] = gt * v[i];
-          }
+          for (int i = 0; i < 32; ++i) zs[i * 128 + r] = __shfl_sync(0xffffffffu, gate_l, i) * v[i];
           named_sync(2, 128);
           const int nrow = min(32, rows - c0);
           for (int e = et; e < nrow * 32; e += 128) {
@@ -598,7 +647,7 @@ bool map_codes(CUtensorMap* m, const uint8_t* base, size_t row_bytes, int rows, 
 bool map_act(CUtensorMap* m, const __half* base, int K, int rows, int box_rows) {
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kSub), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t es[2] = {1u, 1u};
   return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -614,11 +663,11 @@ cudaError_t run_pass(const Ctx& ctx, const FfnArgs& a, GemmParams P, const __hal
   const uint8_t* shr = a.shared != nullptr ? a.shared : a.pool;  // keeps the shared maps well formed
   CUtensorMap maps[8];
   bool ok = true;
-  for (int i = 0; i < 4; ++i) ok = ok && map_act(&maps[i], act, K, n_rows, 16 << i);
-  ok = ok && map_codes(&maps[4], a.pool + codes_off, row_b, rows, a.stride, kMapSlots, kChunk / 4);
-  ok = ok && map_codes(&maps[5], a.pool + codes_off, row_b, rows, a.stride, kMapSlots, kChunk / 8);
-  ok = ok && map_codes(&maps[6], shr + codes_off, row_b, rows, a.stride, 1, kChunk / 4);
-  ok = ok && map_codes(&maps[7], shr + codes_off, row_b, rows, a.stride, 1, kChunk / 8);
+  for (int i = 0; i < 4; ++i) ok = ok && map_act(&maps[i], act, K, n_rows, 16 << i);  // 64-wide boxes
+  ok = ok && map_codes(&maps[4], a.pool + codes_off, row_b, rows, a.stride, kMapSlots, kBK / 4);
+  ok = ok && map_codes(&maps[5], a.pool + codes_off, row_b, rows, a.stride, kMapSlots, kBK / 8);
+  ok = ok && map_codes(&maps[6], shr + codes_off, row_b, rows, a.stride, 1, kBK / 4);
+  ok = ok && map_codes(&maps[7], shr + codes_off, row_b, rows, a.stride, 1, kBK / 8);
   if (!ok) return cudaErrorInvalidValue;
   P.K = K;
   P.m_tiles = rows / kBM;
@@ -668,8 +717,7 @@ cudaError_t run_ffn(const Ctx& ctx, const moe_layer_cfg& c, const FfnArgs& a, co
 }  // namespace
 
 bool prefill_geometry_ok(int d, int f) {
-  return d % kChunk == 0 && f % kChunk == 0 && d % kBM == 0 && (2 * f) % kBM == 0 && d <= kMaxKDim &&
-         f <= kMaxKDim;
+  return d % kBK == 0 && f % kBK == 0 && d % kBM == 0 && (2 * f) % kBM == 0 && d <= kMaxKDim && f <= kMaxKDim;
 }
 
 cudaError_t prefill_init(const Ctx& ctx) {
