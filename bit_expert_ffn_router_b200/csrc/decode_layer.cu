@@ -338,7 +338,7 @@ __device__ void quantise_x(const DLParams& P, int* xq, uint16_t* xs, int nct) {
 
 // Quantises h rows [lo, hi) (fp32, global; this CTA's copy) into the down layout.
 template <int BITS>
-__device__ void quantise_h(const DLParams& P, int lo, int hi, int* hq, int nct) {
+__device__ void quantise_h(const DLParams& P, int lo, int hi, int* hq, int nct, unsigned long long* tr) {
   const int nb = P.f / kBlock, bpl = nb / P.dn_lpr;
   const int words = QV<BITS>::kWords * nb;
   const int jobs = (hi - lo) * nb;
@@ -365,6 +365,7 @@ __device__ void quantise_h(const DLParams& P, int lo, int hi, int* hq, int nct) 
       float v[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) v[k] = live ? vals[g][k] : 0.f;
+      if (tr != nullptr && g == 0 && threadIdx.x == 0) tr[30] = global_timer_ns() + (__float_as_uint(v[0]) & 0u);
       const int gl = blk / bpl, bb = blk % bpl;
       quant_quad<BITS>(v, hq + r * words, nb, bb * P.dn_lpr + gl, q, live);
     }
@@ -375,7 +376,8 @@ __device__ void quantise_h(const DLParams& P, int lo, int hi, int* hq, int nct) 
 // side) for every token of the stage's expert and writes h.
 template <int BITS, int BPL>
 __device__ __forceinline__ void process_gu(const StageRec& s, const uint8_t* ring, const DLParams& P,
-                                           const RouteSmem& R, int np, const int* xq, int& cur_t, XR<BITS>* xr) {
+                                           const RouteSmem& R, int np, const int* xq, int& cur_t, XR<BITS>* xr,
+                                           unsigned long long* tr = nullptr) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int c = s.a + warp;
   const int lpr = P.gu_lpr, gl = lane % lpr;
@@ -394,14 +396,17 @@ __device__ __forceinline__ void process_gu(const StageRec& s, const uint8_t* rin
       load_xr<BITS, BPL>(xq + t * QV<BITS>::kWords * nb, nb, lpr, gl, xr);
       cur_t = t;
     }
+    if (tr != nullptr && lane == 0) tr[20] = clock64();
     float2 v = make_float2(0.f, 0.f);
     if (active) v = row_dot2<BITS, BPL>(cg, sg, cg + row_b, sg + sc_n, P.d, gl, xr);
-    v.x = group_sum(v.x, lpr);
-    v.y = group_sum(v.y, lpr);
+    if (tr != nullptr && lane == 0) tr[21] = clock64() + (__float_as_uint(v.x) & 0u);
+    v = group_sum2(v, lpr);
+    if (tr != nullptr && lane == 0) tr[22] = clock64() + (__float_as_uint(v.y) & 0u);
     float hv = 0.f;
     if (lane == 0) hv = v.x / (1.f + expf(-v.x)) * v.y;
     hv = __shfl_sync(0xffffffffu, hv, 0);
     if (lane < kRep) P.h[lane * P.h_rep + static_cast<size_t>(p) * P.f + c] = hv;
+    if (tr != nullptr && lane == 0) tr[23] = clock64();
   }
 }
 
@@ -618,11 +623,9 @@ __device__ void topk_warp(const DLParams& P, const RouteSmem& R, int t, unsigned
     for (int v = VPL - 1; v >= 0; --v)
       if (key[v] == M) my = static_cast<uint32_t>(v * 32 + lane);
     const int e = static_cast<int>(__reduce_min_sync(0xffffffffu, lm == M ? my : 0xffffffffu));
-    if ((e & 31) == lane) {
+    // take the chosen value out (a select per element keeps key[] in registers)
 #pragma unroll
-      for (int v = 0; v < VPL; ++v)
-        if (v == (e >> 5)) key[v] = 0u;
-    }
+    for (int v = 0; v < VPL; ++v) key[v] = (v * 32 + lane == e) ? 0u : key[v];
     if (lane == j) {
       mine_key = M;
       mine_e = e;
@@ -768,7 +771,7 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
       }
       __syncwarp();
     }
-    bool listed = !ROUTE;
+    bool listed = !ROUTE, planned = false;
     int i = 0;
     while (ok) {
       if (i == n_sh && !listed) {
@@ -787,6 +790,52 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
       if (i >= end) {
         if (listed) break;
         continue;
+      }
+      if (listed && !planned) {
+        // Once the list is known, every earlier stage has normally been
+        // consumed: free them, and if the rest of the list fits the ring
+        // (and the stage mbarriers), lay it out by a prefix sum over the
+        // stage sizes and issue it at once, one stage per lane.
+        planned = true;
+        int okp = 1;
+        if (lane == 0)
+          while (rg.tail < rg.issued)
+            if (!ring_pop(S, st, rg, deadline)) {
+              okp = 0;
+              break;
+            }
+        okp = __shfl_sync(0xffffffffu, okp, 0);
+        if (!okp) {
+          ok = false;
+          break;
+        }
+        const int cnt = end - i;
+        if (cnt <= 32) {
+          const int need =
+              lane < cnt ? (st[i + lane].bytes + kStageAlign - 1) / kStageAlign * kStageAlign : 0;
+          int incl = need;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n;
+          }
+          const int tot = __shfl_sync(0xffffffffu, incl, 31);
+          if (tot <= P.ring_bytes) {
+            if (lane < cnt) st[i + lane].off = incl - need;
+            if (lane == 0) {
+              rg.head = tot;
+              rg.issued = end;  // rg.tail == i: everything before was freed above
+            }
+            __syncwarp();
+            if (lane == 0 && i == n_sh) MOE_TRACE(16)
+            if (lane < cnt) stage_issue(S, st[i + lane], i + lane, ring, P, R);
+            __syncwarp();
+            if (lane == 0 && i == n_sh) MOE_TRACE(17)
+
+            i = end;
+            continue;
+          }
+        }
       }
       int batch = 0, okl = 1;
       if (lane == 0) {
@@ -895,7 +944,7 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
     if (!aborted(S) && warp < st[i].b - st[i].a) {
       if (mbar_wait_warp(&S->full[i % kNB], (i / kNB) & 1, deadline)) {
         if (tid == 0 && i == n_sh) MOE_TRACE(18)
-        process_gu<BITS, GBPL>(st[i], ring, P, R, np, xq, cur_t, xr);
+        process_gu<BITS, GBPL>(st[i], ring, P, R, np, xq, cur_t, xr, (i == n_sh + 1 && warp == 0) ? trace : nullptr);
         if (tid == 0 && i == n_gu - 1) MOE_TRACE(19)
       } else {
         set_abort(S, P.status, 4);
@@ -931,7 +980,8 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
       h_hi = q1;
       ++i1;
     }
-    quantise_h<BITS>(P, h_lo, h_hi, hq, CT);
+    quantise_h<BITS>(P, h_lo, h_hi, hq, CT, i0 == n_gu ? trace : nullptr);
+    if (tid == 0 && i0 == n_gu) MOE_TRACE(31)
     named_sync(1, CT);
     if (tid == 0) MOE_TRACE(24)
 #pragma unroll 1

@@ -156,27 +156,29 @@ __device__ __forceinline__ void load_xr(const int* __restrict__ vec, int nb, int
 
 // sum_i (q_i - 2^(bits-1)) * xq_i over one block: w0, w1 are the block's two
 // 2-bit-plane words, h its high-plane word (3-bit only).
+// Four independent partial sums keep the dependent dp2a chains short.
 template <int BITS>
 __device__ __forceinline__ int block_dot(uint32_t w0, uint32_t w1, uint32_t h, const XR<BITS>& q) {
-  int acc = 0;
+  int a[4] = {0, 0, 0, 0};
 #pragma unroll
   for (int s = 0; s < 4; ++s) {
     const uint32_t b0 = (w0 >> (2 * s)) & 0x03030303u;
     const uint32_t b1 = (w1 >> (2 * s)) & 0x03030303u;
-    acc = dp2a_lo(q.p[s], b0, acc);
-    acc = dp2a_hi(q.p[4 + s], b0, acc);
-    acc = dp2a_lo(q.p[8 + s], b1, acc);
-    acc = dp2a_hi(q.p[12 + s], b1, acc);
+    a[s] = dp2a_lo(q.p[s], b0, a[s]);
+    a[s] = dp2a_hi(q.p[4 + s], b0, a[s]);
+    a[s] = dp2a_lo(q.p[8 + s], b1, a[s]);
+    a[s] = dp2a_hi(q.p[12 + s], b1, a[s]);
   }
+  int acc = (a[0] + a[1]) + (a[2] + a[3]);
   if (BITS == 3) {
-    int hi = 0;
+    int hi[2] = {0, 0};
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
       const uint32_t bh = (h >> t) & 0x01010101u;
-      hi = dp2a_lo(q.ph[t], bh, hi);
-      hi = dp2a_hi(q.ph[8 + t], bh, hi);
+      hi[t & 1] = dp2a_lo(q.ph[t], bh, hi[t & 1]);
+      hi[t & 1] = dp2a_hi(q.ph[8 + t], bh, hi[t & 1]);
     }
-    acc += 4 * hi;
+    acc += 4 * (hi[0] + hi[1]);
   }
   return acc - (1 << (BITS - 1)) * q.sum;
 }

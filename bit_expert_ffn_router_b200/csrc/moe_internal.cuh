@@ -84,7 +84,22 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // Sum over aligned groups of `width` lanes (width a power of two <= 32).
 __device__ __forceinline__ float group_sum(float v, int width) {
-  for (int o = width >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+    if (o < width) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Two such sums at once (interleaved, so their shuffle latencies overlap).
+__device__ __forceinline__ float2 group_sum2(float2 v, int width) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+    if (o < width) {
+      const float a = __shfl_xor_sync(0xffffffffu, v.x, o);
+      const float b = __shfl_xor_sync(0xffffffffu, v.y, o);
+      v.x += a;
+      v.y += b;
+    }
   return v;
 }
 
