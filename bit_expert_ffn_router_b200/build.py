@@ -16,8 +16,8 @@ OBJDIR = os.path.join(HERE, "_build")
 LIB = os.path.join(LIBDIR, "libmoe.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
-SOURCES = ["moe_api.cu", "router.cu", "group.cu", "decode_layer.cu", "ffn_prefill.cu", "combine.cu",
-           "noalloc.cu"]
+SOURCES = ["moe_api.cu", "router.cu", "router_tc.cu", "group.cu", "decode_layer.cu", "ffn_prefill.cu",
+           "combine.cu", "noalloc.cu"]
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -248,7 +248,7 @@ moe_status moe_ctx_create(int device, moe_ctx** out) {
       return MOE_ECUDA;
     }
   }
-  if (cudaMemset(ctx->c.d_status, 0, 64) != cudaSuccess || router_init(ctx->c) != cudaSuccess ||
+  if (cudaMemset(ctx->c.d_status, 0, 64) != cudaSuccess || router_init(ctx->c) != cudaSuccess || router_tc_init(ctx->c) != cudaSuccess ||
       decode_init(ctx->c) != cudaSuccess || prefill_init(ctx->c) != cudaSuccess) {
     cudaFree(ctx->c.d_status);
     delete ctx;

@@ -138,12 +138,13 @@ router_gemm_kernel(const uint16_t* __restrict__ x, const float* __restrict__ wr,
 cudaError_t launch_router_logits(const Ctx& ctx, const moe_layer_cfg& c, const uint16_t* x,
                                  const float* wr, const float* bias, int T, float* logits,
                                  cudaStream_t s) {
-  (void)ctx;
   if (T <= MOE_DECODE_MAX_T) {
     const size_t smem = static_cast<size_t>(T) * c.d * sizeof(float);
     const dim3 grid((c.E + kRouterWarps - 1) / kRouterWarps);
     router_rows_kernel<MOE_DECODE_MAX_T><<<grid, kRouterWarps * 32, smem, s>>>(x, wr, bias, T, c.d,
                                                                               c.E, logits);
+  } else if (router_tc_ok(c)) {
+    return launch_router_tc(ctx, c, x, wr, bias, T, logits, s);  // tensor cores, bf16 three-part split
   } else {
     const dim3 grid((c.E + kGN - 1) / kGN, (T + kGM - 1) / kGM);
     router_gemm_kernel<<<grid, 256, 0, s>>>(x, wr, bias, T, c.d, c.E, logits);

@@ -21,7 +21,8 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("cfg,T,zipf", [(M.TINY, 4, False), (M.TINY, 1, False), (M.FULL, 1, True),
                                         (M.FULL, 4, True), (M.FULL, 8, False), (M.FULL, 37, True),
-                                        (M.FULL, 1000, False)])
+                                        (M.FULL, 1000, False), (M.TINY, 300, False),
+                                        (M.FULL.replace(E=1024, k=32), 200, False)])
 def test_router_topk_matches_oracle(cfg, T, zipf):
     L = H.Layer(cfg.replace(n_shared=0), T, seed=T, zipf=zipf)
     dv = L.device()
