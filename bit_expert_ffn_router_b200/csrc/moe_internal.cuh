@@ -90,6 +90,22 @@ __device__ __forceinline__ float group_sum(float v, int width) {
   return v;
 }
 
+// Four such sums at once (two float2), interleaved.
+__device__ __forceinline__ void group_sum4(float2& a, float2& b, int width) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+    if (o < width) {
+      const float x0 = __shfl_xor_sync(0xffffffffu, a.x, o);
+      const float x1 = __shfl_xor_sync(0xffffffffu, a.y, o);
+      const float x2 = __shfl_xor_sync(0xffffffffu, b.x, o);
+      const float x3 = __shfl_xor_sync(0xffffffffu, b.y, o);
+      a.x += x0;
+      a.y += x1;
+      b.x += x2;
+      b.y += x3;
+    }
+}
+
 // Two such sums at once (interleaved, so their shuffle latencies overlap).
 __device__ __forceinline__ float2 group_sum2(float2 v, int width) {
 #pragma unroll
@@ -181,5 +197,11 @@ cudaError_t launch_combine(const Ctx& ctx, const moe_layer_cfg& c, const int32_t
 // kernel attribute set-up, once per context
 cudaError_t decode_init(const Ctx& ctx);
 cudaError_t router_init(const Ctx& ctx);
+
+// router_tc.cu: prefill router logits on the tensor cores
+bool router_tc_ok(const moe_layer_cfg& c);
+cudaError_t launch_router_tc(const Ctx& ctx, const moe_layer_cfg& c, const uint16_t* x, const float* wr,
+                             const float* bias, int T, float* logits, cudaStream_t s);
+cudaError_t router_tc_init(const Ctx& ctx);
 
 }  // namespace moe
