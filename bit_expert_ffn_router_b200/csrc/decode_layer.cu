@@ -719,19 +719,20 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
   const int cs1 = static_cast<int>((static_cast<long long>(P.f) * (b + 1)) / G);
   const int r0 = min(b * P.rpc, P.d), r1 = min(r0 + P.rpc, P.d);
 
-  if (threadIdx.x == 0) {
-    if (trace != nullptr) {
-      trace[0] = t_start;
-      trace[14] = clock64();
+  if (warp == 0) {  // lane i initialises stage barrier pair i
+    static_assert(kNB == 32, "one stage barrier pair per lane");
+    mbar_init(&S->full[lane], 1);
+    mbar_init(&S->empty[lane], CW);
+    if (lane == 0) {
+      if (trace != nullptr) {
+        trace[0] = t_start;
+        trace[14] = clock64();
+      }
+      mbar_init(&S->wr_bar, 1);
+      mbar_init(&S->list_bar, 1);
+      S->abort_flag = 0;
+      S->n_sh = P.has_shared ? push_gu(st, 0, kShared, cs0, cs1, P) : 0;
     }
-    for (int i = 0; i < kNB; ++i) {
-      mbar_init(&S->full[i], 1);
-      mbar_init(&S->empty[i], CW);
-    }
-    mbar_init(&S->wr_bar, 1);
-    mbar_init(&S->list_bar, 1);
-    S->abort_flag = 0;
-    S->n_sh = P.has_shared ? push_gu(st, 0, kShared, cs0, cs1, P) : 0;
     fence_mbar_init();
   }
   __syncthreads();

@@ -413,14 +413,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB16, const __grid_const
         const int lc = r >> 1;
         const int lp = (lc & ~15) | k_position(lc & 15);
         __half* hs = reinterpret_cast<__half*>(smem + PrefillSmem::kStage);  // [kBN pairs][64 channels]
+        // the lane pair (gate, up) shares the 16 columns of a chunk: the gate
+        // lane takes columns 0..7, the up lane 8..15 (h is rounded to fp16, so
+        // the fast exponential and division are well inside its precision)
+        const bool up_lane = (lane & 1) != 0;
         for (int c0 = 0; c0 < rows; c0 += 16) {
-          float v[16];
+          float v[16], o[16];
           tmem_ld16(base + c0, v);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float u = __shfl_xor_sync(0xffffffffu, v[i], 1);
-            if ((lane & 1) == 0 && c0 + i < rows)
-              hs[(c0 + i) * 64 + lp] = __float2half_rn(v[i] / (1.f + expf(-v[i])) * u);
+          for (int i = 0; i < 16; ++i) o[i] = __shfl_xor_sync(0xffffffffu, v[i], 1);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float g = up_lane ? o[8 + i] : v[i];
+            const float u = up_lane ? v[8 + i] : o[i];
+            const int col = c0 + (up_lane ? 8 : 0) + i;
+            if (col < rows) hs[col * 64 + lp] = __float2half_rn(__fdividef(g, 1.f + __expf(-g)) * u);
           }
         }
         tc_fence_before();
