@@ -61,7 +61,6 @@ struct DLParams {
   float* h;                  // kRep copies of [n_rows, f], h_rep floats apart
   size_t h_rep;
   float* logits_rep;         // route: kRep copies of [T, E]
-  int32_t* slot_rep;         // route: kRep copies of [E]
   void* y;
   int* status;
   unsigned long long* gbar;  // grid-barrier arrival counter
@@ -118,6 +117,7 @@ struct RouteSmem {
   int32_t* uniq_e;     // [np]
   int32_t* uniq_slot;  // [np]
   int32_t* uniq_off;   // [np + 1]
+  int32_t* slot_s;     // [E] this layer's slot table (routing path)
 };
 
 __device__ __forceinline__ RouteSmem route_smem(char* base, int np) {
@@ -132,6 +132,7 @@ __device__ __forceinline__ RouteSmem route_smem(char* base, int np) {
   r.uniq_e = p + 6 * np;
   r.uniq_slot = p + 7 * np;
   r.uniq_off = p + 8 * np;
+  r.slot_s = p + 9 * np + 1;
   return r;
 }
 
@@ -186,15 +187,16 @@ __device__ int push_dn(StageRec* st, int n, int u, int r0, int r1, const DLParam
 // expert's gate/up) are already in place.
 __device__ void build_routed_list(StageRec* st, DLShared* S, int n_sh, int nu, int b, int G, int r0, int r1,
                                   const DLParams& P) {
+  // 32-bit arithmetic: the launch guarantees nu * f * G < 2^31
   int n = n_sh;
-  const long long tot = static_cast<long long>(nu) * P.f;
-  long long c = tot * b / G;
-  const long long c1 = tot * (b + 1) / G;
+  const int tot = nu * P.f;
+  int c = tot * b / G;
+  const int c1 = tot * (b + 1) / G;
   while (c < c1) {
-    const int u = static_cast<int>(c / P.f);
-    const long long ub = static_cast<long long>(u) * P.f;
-    const int ce = static_cast<int>(min(c1, ub + P.f) - ub);
-    n = push_gu(st, n, u, static_cast<int>(c - ub), ce, P);
+    const int u = c / P.f;
+    const int ub = u * P.f;
+    const int ce = min(c1, ub + P.f) - ub;
+    n = push_gu(st, n, u, c - ub, ce, P);
     c = ub + ce;
   }
   S->n_gu = n;
@@ -467,7 +469,7 @@ __device__ void group_in_smem(const DLParams& P, const RouteSmem& R, DLShared* S
       if (first) {
         const int u = base + __popc(m & ((1u << tid) - 1u));
         const int e = R.sorted_e[i];
-        int slot = __ldcg(P.slot_rep + (blockIdx.x % kRep) * P.E + e);
+        int slot = R.slot_s[e];
         if (slot < 0 || slot >= P.n_slots) {
           report(P.status, kDevBadSlot, e);
           slot = 0;
@@ -652,16 +654,11 @@ __device__ void topk_warp(const DLParams& P, const RouteSmem& R, int t, unsigned
 }
 
 // Router rows [e0, e1) of this CTA for every token: lanes read W_r and x
-// (both in shared memory) in interleaved 4-column groups. Every logit and
-// the rows' slots are written kRep times (one copy per group of readers).
+// (both in shared memory) in interleaved 4-column groups. Every logit is
+// written kRep times (one copy per group of readers).
 __device__ void router_rows(const DLParams& P, const float* wrs, const uint16_t* xs, int e0, int e1, int cw) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int n4 = P.d / 4;
-  if (warp == 0)
-    for (int i = lane; i < (e1 - e0) * kRep; i += 32) {
-      const int e = e0 + i / kRep, r = i % kRep;
-      P.slot_rep[r * P.E + e] = P.slot_of[e];
-    }
   for (int t = 0; t < P.T; ++t) {
     const uint2* x2 = reinterpret_cast<const uint2*>(xs + static_cast<size_t>(t) * P.d);
 #pragma unroll 1
@@ -881,6 +878,14 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
   // -------------------------------------------------------------- consumers
   const int tid = threadIdx.x;
   grid_dep_wait();  // x (and the workspace) may come from the previous kernel
+  // this layer's slot table, fetched now and parked in shared memory after the
+  // router, so that the slot lookup after top-k is a shared-memory read (the
+  // routing path has E <= 2 * CT)
+  int slot_v0 = 0, slot_v1 = 0;
+  if (ROUTE) {
+    if (tid < P.E) slot_v0 = __ldg(P.slot_of + tid);
+    if (tid + CT < P.E) slot_v1 = __ldg(P.slot_of + tid + CT);
+  }
   quantise_x<BITS>(P, xq, xs, CT);
   named_sync(1, CT);
   if (tid == 0) MOE_TRACE(1)
@@ -888,6 +893,8 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
   if (ROUTE) {
     if (e1 > e0 && !mbar_wait_warp(&S->wr_bar, 0, deadline)) set_abort(S, P.status, 1);
     if (!aborted(S)) router_rows(P, wrs, xs, e0, e1, CW);
+    if (tid < P.E) R.slot_s[tid] = slot_v0;
+    if (tid + CT < P.E) R.slot_s[tid + CT] = slot_v1;
     named_sync(1, CT);
     if (tid == 0) MOE_TRACE(2)
     if (tid == 0 && !aborted(S)) S->bar_target = gbar_arrive(P.gbar, G);
@@ -1118,7 +1125,6 @@ cudaError_t launch_decode_layer(const Ctx& ctx, const moe_layer_cfg& c, const De
   P.h = a.h;
   P.h_rep = static_cast<size_t>(np + (c.n_shared ? T : 0)) * c.f;
   P.logits_rep = a.logits_rep;
-  P.slot_rep = a.slot_rep;
   P.y = a.y;
   P.status = ctx.d_status;
   P.gbar = ctx.d_gbar;
@@ -1138,6 +1144,8 @@ cudaError_t launch_decode_layer(const Ctx& ctx, const moe_layer_cfg& c, const De
   P.rpc = static_cast<int>(align_up((c.d + G - 1) / G, gran));
   P.wr_rows = (c.E + G - 1) / G;
   const int n_uniq_max = np < c.E ? np : c.E;
+  // the device-side list arithmetic is 32-bit: nu * f * G must stay below 2^31
+  if (static_cast<long long>(n_uniq_max) * c.f * G >= (1LL << 31)) return cudaErrorNotSupported;
   const int sh_ch = (c.f + G - 1) / G;
   P.max_stages = (sh_ch + CW - 1) / CW + 1 +
                  static_cast<int>((static_cast<long long>(n_uniq_max) * c.f + G - 1) / G + CW - 1) / CW +
@@ -1147,7 +1155,7 @@ cudaError_t launch_decode_layer(const Ctx& ctx, const moe_layer_cfg& c, const De
   P.sm_stages = static_cast<int>(o);
   o = align_up(o + static_cast<size_t>(P.max_stages) * sizeof(StageRec), 128);
   P.sm_route = static_cast<int>(o);
-  o = align_up(o + (9 * static_cast<size_t>(np) + 1) * 4, 128);
+  o = align_up(o + (9 * static_cast<size_t>(np) + 1 + (a.route ? c.E : 0)) * 4, 128);
   P.sm_zs = static_cast<int>(o);
   o = align_up(o + static_cast<size_t>(np + T) * P.rpc * 4, 128);  // z rows [np + T][rpc]
   P.sm_xq = static_cast<int>(o);

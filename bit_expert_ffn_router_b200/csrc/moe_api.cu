@@ -41,7 +41,6 @@ WsLayout ws_layout(const moe_layer_cfg& c, int T) {
   w.tile_offset = take((static_cast<size_t>(c.E) + 2) * 4);
   const bool decode = T <= MOE_DECODE_MAX_T;
   w.logits_rep = take(decode ? static_cast<size_t>(kRep) * Tz * c.E * 4 : 0);
-  w.slot_rep = take(decode ? static_cast<size_t>(kRep) * c.E * 4 : 0);
   // h: fp32 rows (kRep copies) on the decode path, fp16 rows (padded by one
   // tile) on the prefill path
   const size_t h32 = static_cast<size_t>(decode ? kRep : 1) * w.n_rows * c.f * 4;
@@ -204,7 +203,6 @@ static moe_status run_ffn(moe_ctx* ctx, const moe_layer_cfg* cfg, int bits, cons
     d.h = reinterpret_cast<float*>(a.h);
     d.y = y;
     d.logits_rep = reinterpret_cast<float*>(static_cast<char*>(ws) + w.logits_rep);
-    d.slot_rep = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + w.slot_rep);
     const cudaError_t e = launch_decode_layer(ctx->c, *cfg, d, s);
     if (e == cudaErrorNotSupported) return MOE_EUNSUPPORTED;
     return from_cuda(e);
@@ -447,7 +445,6 @@ moe_status moe_layer_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, const void*
     d.h = reinterpret_cast<float*>(b + w.h);
     d.y = y;
     d.logits_rep = reinterpret_cast<float*>(b + w.logits_rep);
-    d.slot_rep = reinterpret_cast<int32_t*>(b + w.slot_rep);
     const cudaError_t e = launch_decode_layer(ctx->c, *cfg, d, static_cast<cudaStream_t>(stream));
     if (e == cudaErrorNotSupported) return MOE_EUNSUPPORTED;
     return from_cuda(e);

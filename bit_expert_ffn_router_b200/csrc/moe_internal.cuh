@@ -55,7 +55,7 @@ struct WsLayout {
   size_t expert_count, expert_offset, pair_token, pair_j, pair_gate, pair_slot, pair_pos;
   size_t uniq_expert, uniq_slot, uniq_offset, n_uniq;
   size_t chunk_hist, tile_offset;
-  size_t logits_rep, slot_rep;  // decode path: kRep copies of [T, E] logits and [E] slots
+  size_t logits_rep;            // decode path: kRep copies of the [T, E] logits
   size_t h, z, x16;
   size_t tile_info;              // prefill: int4 per token tile
   size_t total;
@@ -163,7 +163,6 @@ struct DecodeArgs {
   moe_expert_layout lay;
   float* h;                 // fp32 [kRep][n_rows, f]
   float* logits_rep;        // route: [kRep][T, E]
-  int32_t* slot_rep;        // route: [kRep][E]
   void* y;
 };
 cudaError_t launch_decode_layer(const Ctx& ctx, const moe_layer_cfg& c, const DecodeArgs& a, cudaStream_t s);

@@ -38,7 +38,7 @@ def test_layer_prefill_tiny(bits, T):
 
 
 @pytest.mark.parametrize("bits", [2, 3])
-@pytest.mark.parametrize("count", [127, 128, 129, 257])
+@pytest.mark.parametrize("count", [127, 128, 129, 255, 256, 257])
 def test_prefill_tile_boundaries(bits, count):
     # every token picks experts {3, 5}: two experts with `count` pairs each,
     # the shared expert with `count` rows, all other experts empty
