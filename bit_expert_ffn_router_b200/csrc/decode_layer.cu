@@ -307,33 +307,67 @@ __device__ void quantise_x(const DLParams& P, int* xq, uint16_t* xs, int nct) {
   const int words = QV<BITS>::kWords * nb;
   const int jobs = P.T * nb;
   const int q = threadIdx.x & 3;
+  if constexpr (BITS == 2) {
+    // thread q of a block takes its 8 consecutive values in one 16-byte load
 #pragma unroll 1
-  for (int base0 = threadIdx.x & ~31; base0 < jobs * 4; base0 += kQD * nct) {
-    uint16_t bits[kQD][8];
+    for (int base0 = threadIdx.x & ~31; base0 < jobs * 4; base0 += kQD * nct) {
+      uint4 raw[kQD];
 #pragma unroll
-    for (int g = 0; g < kQD; ++g) {
-      if (base0 + g * nct >= jobs * 4) break;
-      const int job = min((base0 + g * nct + (threadIdx.x & 31)) >> 2, jobs - 1);
-      const size_t a = static_cast<size_t>(job / nb) * P.d + (job % nb) * kBlock + q;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) bits[g][k] = __ldcg(P.x + a + 4 * k);
-    }
-#pragma unroll
-    for (int g = 0; g < kQD; ++g) {
-      const int base = base0 + g * nct;  // warp-uniform
-      if (base >= jobs * 4) break;
-      const int job = (base + (threadIdx.x & 31)) >> 2;
-      const bool live = job < jobs;
-      const int t = live ? job / nb : 0, blk = live ? job % nb : 0;
-      const size_t at = static_cast<size_t>(t) * P.d + blk * kBlock + q;
-      float v[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        if (live) xs[at + 4 * k] = bits[g][k];
-        v[k] = live ? bf16_bits_to_float(bits[g][k]) : 0.f;
+      for (int g = 0; g < kQD; ++g) {
+        if (base0 + g * nct >= jobs * 4) break;
+        const int job = min((base0 + g * nct + (threadIdx.x & 31)) >> 2, jobs - 1);
+        const size_t a = static_cast<size_t>(job / nb) * P.d + (job % nb) * kBlock + 8 * q;
+        raw[g] = __ldcg(reinterpret_cast<const uint4*>(P.x + a));
       }
-      const int gl = blk / bpl, bb = blk % bpl;
-      quant_quad<BITS>(v, xq + t * words, nb, bb * P.gu_lpr + gl, q, live);
+#pragma unroll
+      for (int g = 0; g < kQD; ++g) {
+        const int base = base0 + g * nct;  // warp-uniform
+        if (base >= jobs * 4) break;
+        const int job = (base + (threadIdx.x & 31)) >> 2;
+        const bool live = job < jobs;
+        const int t = live ? job / nb : 0, blk = live ? job % nb : 0;
+        const size_t at = static_cast<size_t>(t) * P.d + blk * kBlock + 8 * q;
+        if (live) *reinterpret_cast<uint4*>(xs + at) = raw[g];
+        const uint32_t w[4] = {raw[g].x, raw[g].y, raw[g].z, raw[g].w};
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint16_t h = static_cast<uint16_t>(w[k >> 1] >> (16 * (k & 1)));
+          v[k] = live ? bf16_bits_to_float(h) : 0.f;
+        }
+        const int gl = blk / bpl, bb = blk % bpl;
+        quant_quad_c2(v, xq + t * words, nb, bb * P.gu_lpr + gl, q, live);
+      }
+    }
+  } else {
+#pragma unroll 1
+    for (int base0 = threadIdx.x & ~31; base0 < jobs * 4; base0 += kQD * nct) {
+      uint16_t bits[kQD][8];
+#pragma unroll
+      for (int g = 0; g < kQD; ++g) {
+        if (base0 + g * nct >= jobs * 4) break;
+        const int job = min((base0 + g * nct + (threadIdx.x & 31)) >> 2, jobs - 1);
+        const size_t a = static_cast<size_t>(job / nb) * P.d + (job % nb) * kBlock + q;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) bits[g][k] = __ldcg(P.x + a + 4 * k);
+      }
+#pragma unroll
+      for (int g = 0; g < kQD; ++g) {
+        const int base = base0 + g * nct;  // warp-uniform
+        if (base >= jobs * 4) break;
+        const int job = (base + (threadIdx.x & 31)) >> 2;
+        const bool live = job < jobs;
+        const int t = live ? job / nb : 0, blk = live ? job % nb : 0;
+        const size_t at = static_cast<size_t>(t) * P.d + blk * kBlock + q;
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (live) xs[at + 4 * k] = bits[g][k];
+          v[k] = live ? bf16_bits_to_float(bits[g][k]) : 0.f;
+        }
+        const int gl = blk / bpl, bb = blk % bpl;
+        quant_quad<BITS>(v, xq + t * words, nb, bb * P.gu_lpr + gl, q, live);
+      }
     }
   }
 }
@@ -346,30 +380,60 @@ __device__ void quantise_h(const DLParams& P, int lo, int hi, int* hq, int nct, 
   const int jobs = (hi - lo) * nb;
   const int q = threadIdx.x & 3;
   const float* hb = P.h + (blockIdx.x % kRep) * P.h_rep;
+  if constexpr (BITS == 2) {
+    // thread q of a block takes its 8 consecutive values in two 16-byte loads
 #pragma unroll 1
-  for (int base0 = threadIdx.x & ~31; base0 < jobs * 4; base0 += kQD * nct) {
-    float vals[kQD][8];
+    for (int base0 = threadIdx.x & ~31; base0 < jobs * 4; base0 += kQD * nct) {
+      float4 raw[kQD][2];
 #pragma unroll
-    for (int g = 0; g < kQD; ++g) {
-      if (base0 + g * nct >= jobs * 4) break;
-      const int job = min((base0 + g * nct + (threadIdx.x & 31)) >> 2, jobs - 1);
-      const float* src = hb + static_cast<size_t>(lo + job / nb) * P.f + (job % nb) * kBlock + q;
+      for (int g = 0; g < kQD; ++g) {
+        if (base0 + g * nct >= jobs * 4) break;
+        const int job = min((base0 + g * nct + (threadIdx.x & 31)) >> 2, jobs - 1);
+        const float4* src =
+            reinterpret_cast<const float4*>(hb + static_cast<size_t>(lo + job / nb) * P.f + (job % nb) * kBlock + 8 * q);
+        raw[g][0] = __ldcg(src);
+        raw[g][1] = __ldcg(src + 1);
+      }
 #pragma unroll
-      for (int k = 0; k < 8; ++k) vals[g][k] = __ldcg(src + 4 * k);
+      for (int g = 0; g < kQD; ++g) {
+        const int base = base0 + g * nct;  // warp-uniform
+        if (base >= jobs * 4) break;
+        const int job = (base + (threadIdx.x & 31)) >> 2;
+        const bool live = job < jobs;
+        const int r = live ? job / nb : 0, blk = live ? job % nb : 0;
+        const float v[8] = {raw[g][0].x, raw[g][0].y, raw[g][0].z, raw[g][0].w,
+                            raw[g][1].x, raw[g][1].y, raw[g][1].z, raw[g][1].w};
+        if (tr != nullptr && g == 0 && threadIdx.x == 0) tr[30] = global_timer_ns() + (__float_as_uint(v[0]) & 0u);
+        const int gl = blk / bpl, bb = blk % bpl;
+        quant_quad_c2(v, hq + r * words, nb, bb * P.dn_lpr + gl, q, live);
+      }
     }
+  } else {
+#pragma unroll 1
+    for (int base0 = threadIdx.x & ~31; base0 < jobs * 4; base0 += kQD * nct) {
+      float vals[kQD][8];
 #pragma unroll
-    for (int g = 0; g < kQD; ++g) {
-      const int base = base0 + g * nct;  // warp-uniform
-      if (base >= jobs * 4) break;
-      const int job = (base + (threadIdx.x & 31)) >> 2;
-      const bool live = job < jobs;
-      const int r = live ? job / nb : 0, blk = live ? job % nb : 0;
-      float v[8];
+      for (int g = 0; g < kQD; ++g) {
+        if (base0 + g * nct >= jobs * 4) break;
+        const int job = min((base0 + g * nct + (threadIdx.x & 31)) >> 2, jobs - 1);
+        const float* src = hb + static_cast<size_t>(lo + job / nb) * P.f + (job % nb) * kBlock + q;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) v[k] = live ? vals[g][k] : 0.f;
-      if (tr != nullptr && g == 0 && threadIdx.x == 0) tr[30] = global_timer_ns() + (__float_as_uint(v[0]) & 0u);
-      const int gl = blk / bpl, bb = blk % bpl;
-      quant_quad<BITS>(v, hq + r * words, nb, bb * P.dn_lpr + gl, q, live);
+        for (int k = 0; k < 8; ++k) vals[g][k] = __ldcg(src + 4 * k);
+      }
+#pragma unroll
+      for (int g = 0; g < kQD; ++g) {
+        const int base = base0 + g * nct;  // warp-uniform
+        if (base >= jobs * 4) break;
+        const int job = (base + (threadIdx.x & 31)) >> 2;
+        const bool live = job < jobs;
+        const int r = live ? job / nb : 0, blk = live ? job % nb : 0;
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = live ? vals[g][k] : 0.f;
+        if (tr != nullptr && g == 0 && threadIdx.x == 0) tr[30] = global_timer_ns() + (__float_as_uint(v[0]) & 0u);
+        const int gl = blk / bpl, bb = blk % bpl;
+        quant_quad<BITS>(v, hq + r * words, nb, bb * P.dn_lpr + gl, q, live);
+      }
     }
   }
 }

@@ -129,6 +129,37 @@ __device__ __forceinline__ void quant_quad(const float* v, int* vec, int nb, int
   }
 }
 
+// 2-bit layout only: the same block quantisation as quant_quad, for a thread
+// q of the block's four that holds the eight consecutive values 8q .. 8q+7
+// (two 16-byte loads instead of eight strided ones). Word 8(q/2) + 4(q%2) + i
+// of the block is the pair (8q + i, 8q + i + 4), exactly the words
+// quant_quad writes for those values.
+__device__ __forceinline__ void quant_quad_c2(const float* v, int* vec, int nb, int col, int q, bool store) {
+  float m = fmaxf(fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))),
+                  fmaxf(fmaxf(fabsf(v[4]), fabsf(v[5])), fmaxf(fabsf(v[6]), fabsf(v[7]))));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  const float inv = m > 0.f ? 32767.f / m : 0.f;
+  constexpr float kMagic = 12582912.f;  // 1.5 * 2^23
+  int r[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) r[k] = __float_as_int(fmaf(v[k], inv, kMagic));
+  unsigned us = (static_cast<unsigned>(r[0]) + static_cast<unsigned>(r[1])) +
+                (static_cast<unsigned>(r[2]) + static_cast<unsigned>(r[3])) +
+                ((static_cast<unsigned>(r[4]) + static_cast<unsigned>(r[5])) +
+                 (static_cast<unsigned>(r[6]) + static_cast<unsigned>(r[7])));
+  us += __shfl_xor_sync(0xffffffffu, us, 1);
+  us += __shfl_xor_sync(0xffffffffu, us, 2);
+  if (!store) return;
+  const int w0 = 8 * (q >> 1) + 4 * (q & 1);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) vec[(w0 + i) * nb + col] = static_cast<int>(__byte_perm(r[i], r[i + 4], 0x5410));
+  if (q == 0) {
+    vec[QV<2>::kSX * nb + col] = __float_as_int(m * (1.f / 32767.f));
+    vec[(QV<2>::kSX + 1) * nb + col] = static_cast<int>(us - 32u * 0x4B400000u);
+  }
+}
+
 // One block of a quantised vector, in registers.
 template <int BITS>
 struct XR {
