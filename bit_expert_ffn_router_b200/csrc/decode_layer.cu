@@ -469,7 +469,9 @@ __device__ __forceinline__ void process_gu(const StageRec& s, const uint8_t* rin
     v = group_sum2(v, lpr);
     if (tr != nullptr && lane == 0) tr[22] = clock64() + (__float_as_uint(v.y) & 0u);
     float hv = 0.f;
-    if (lane == 0) hv = v.x / (1.f + expf(-v.x)) * v.y;
+    // fast exponential and division: h is requantised to 16 bits for the
+    // down rows, far coarser than their few-ulp error
+    if (lane == 0) hv = __fdividef(v.x, 1.f + __expf(-v.x)) * v.y;
     hv = __shfl_sync(0xffffffffu, hv, 0);
     if (lane < kRep) P.h[lane * P.h_rep + static_cast<size_t>(p) * P.f + c] = hv;
     if (tr != nullptr && lane == 0) tr[23] = clock64();
