@@ -859,7 +859,7 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
         // Once the list is known, every earlier stage has normally been
         // consumed: free them, and if the rest of the list fits the ring
         // (and the stage mbarriers), lay it out by a prefix sum over the
-        // stage sizes and issue it at once, one stage per lane.
+        // stage sizes and issue it in order.
         planned = true;
         int okp = 1;
         if (lane == 0)
@@ -892,10 +892,26 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
             }
             __syncwarp();
             if (lane == 0 && i == n_sh) MOE_TRACE(16)
-            if (lane < cnt) stage_issue(S, st[i + lane], i + lane, ring, P, R);
+            // at most two stages in flight: stage j is issued once stage j-2
+            // has landed, so the copies arrive in the order they are consumed
+            int okq = 1;
+            if (lane == 0)
+              for (int j = 0; j < cnt; ++j) {
+                if (j >= 2 && !mbar_wait(&S->full[(i + j - 2) % kNB], ((i + j - 2) / kNB) & 1, deadline)) {
+                  okq = 0;
+                  rg.issued = i + j;
+                  break;
+                }
+                stage_issue(S, st[i + j], i + j, ring, P, R);
+              }
+            okq = __shfl_sync(0xffffffffu, okq, 0);
             __syncwarp();
             if (lane == 0 && i == n_sh) MOE_TRACE(17)
-
+            if (!okq) {
+              ok = false;
+              i = __shfl_sync(0xffffffffu, rg.issued, 0);
+              break;
+            }
             i = end;
             continue;
           }
@@ -975,7 +991,8 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
 #pragma unroll 1
   for (int i = 0;; ++i) {
     if (i == n_sh) {
-      cur_t = -1;  // the cached x row is not needed across the routing step (frees its registers)
+      // the cached x row (xr, cur_t) stays in registers across the routing
+      // step: the routed stages of a token reuse it
       if (tid == 0) MOE_TRACE(3)
       if (ROUTE) {
         if (tid == 0 && !aborted(S) && !gbar_wait(P.gbar, S->bar_target, deadline)) set_abort(S, P.status, 3);
