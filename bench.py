@@ -40,7 +40,7 @@ SEED = 0
 KERNELS_PER_LAYER_DECODE = 1  # one fused decode-layer kernel
 # dram__bytes_read.sum + dram__bytes_write.sum of one fused decode-layer launch
 # (T=1, 2-bit), from an ncu capture of that kernel
-DECODE_LAYER_DRAM_BYTES = 20540416
+DECODE_LAYER_DRAM_BYTES = 20537856
 
 
 def peaks():
