@@ -856,23 +856,13 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
         continue;
       }
       if (listed && !planned) {
-        // Once the list is known, every earlier stage has normally been
-        // consumed: free them, and if the rest of the list fits the ring
-        // (and the stage mbarriers), lay it out by a prefix sum over the
-        // stage sizes and issue it in order.
+        // Once the list is known, lay the rest of it out in the ring in one
+        // step (a prefix sum over the stage sizes) if it fits the ring and the
+        // stage mbarriers, and issue it in order. The stages before it (the
+        // shared expert's gate/up, consumed after the routing step) stay
+        // live: the layout goes after them, or, if it does not fit there,
+        // they are waited for and freed first.
         planned = true;
-        int okp = 1;
-        if (lane == 0)
-          while (rg.tail < rg.issued)
-            if (!ring_pop(S, st, rg, deadline)) {
-              okp = 0;
-              break;
-            }
-        okp = __shfl_sync(0xffffffffu, okp, 0);
-        if (!okp) {
-          ok = false;
-          break;
-        }
         const int cnt = end - i;
         if (cnt <= 32) {
           const int need =
@@ -884,11 +874,33 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
             if (lane >= o) incl += n;
           }
           const int tot = __shfl_sync(0xffffffffu, incl, 31);
-          if (tot <= P.ring_bytes) {
-            if (lane < cnt) st[i + lane].off = incl - need;
+          int base = -1, okp = 1;
+          if (lane == 0) {
+            // live stages stay if the layout fits after them and no stage of
+            // it shares an mbarrier with one of them
+            const bool live = rg.tail < rg.issued;
+            if (live && rg.head > st[rg.tail].off && rg.head + tot <= P.ring_bytes && end - rg.tail <= kNB) {
+              base = rg.head;
+            } else if (tot <= P.ring_bytes) {
+              while (rg.tail < rg.issued)
+                if (!ring_pop(S, st, rg, deadline)) {
+                  okp = 0;
+                  break;
+                }
+              base = 0;
+            }
+          }
+          okp = __shfl_sync(0xffffffffu, okp, 0);
+          base = __shfl_sync(0xffffffffu, base, 0);
+          if (!okp) {
+            ok = false;
+            break;
+          }
+          if (base >= 0) {
+            if (lane < cnt) st[i + lane].off = base + incl - need;
             if (lane == 0) {
-              rg.head = tot;
-              rg.issued = end;  // rg.tail == i: everything before was freed above
+              rg.head = base + tot;
+              rg.issued = end;
             }
             __syncwarp();
             if (lane == 0 && i == n_sh) MOE_TRACE(16)
@@ -982,15 +994,18 @@ __global__ void __launch_bounds__((consumer_warps(BITS) + 1) * 32, 1) decode_lay
     if (tid == 0 && !aborted(S)) S->bar_target = gbar_arrive(P.gbar, G);
   }
 
-  // gate/up stages: the shared expert's [0, n_sh) need no routing; routing is
-  // resolved when the loop reaches n_sh, then the routed stages follow
+  // gate/up stages: the shared expert's [0, n_sh) need no routing and are
+  // fetched from the start. With routing in the kernel it is resolved first
+  // (loop index 0): the shared stages then run while the routed stages'
+  // copies are on their way. Otherwise the list comes from the producer once
+  // the loop reaches n_sh. The routed stages follow.
   XR<BITS> xr[GBPL];
   int cur_t = -1;
   const int n_sh = S->n_sh;
   int n_gu = n_sh;
 #pragma unroll 1
   for (int i = 0;; ++i) {
-    if (i == n_sh) {
+    if (i == (ROUTE ? 0 : n_sh)) {
       // the cached x row (xr, cur_t) stays in registers across the routing
       // step: the routed stages of a token reuse it
       if (tid == 0) MOE_TRACE(3)
