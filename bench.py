@@ -39,8 +39,11 @@ HOT = 4500
 SEED = 0
 KERNELS_PER_LAYER_DECODE = 1  # one fused decode-layer kernel
 # dram__bytes_read.sum + dram__bytes_write.sum of one fused decode-layer launch
-# (T=1, 2-bit), from an ncu capture of that kernel
-DECODE_LAYER_DRAM_BYTES = 20537856
+# (T=1, 2-bit) from an ncu capture of the current kernel, or None when the
+# kernel has changed since the last capture (the last one, of the revision
+# before the routing step moved ahead of the shared expert's stages, read
+# 20,537,600 B and wrote 256 B per launch)
+DECODE_LAYER_DRAM_BYTES = None
 
 
 def peaks():
