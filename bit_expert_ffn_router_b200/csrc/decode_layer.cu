@@ -10,15 +10,17 @@
 //
 // One CTA per SM, 15 consumer warps + 1 producer warp:
 //   producer: cp.async.bulk copies of this CTA's weight rows into a
-//             shared-memory byte ring, one mbarrier per stage, issued as far
-//             ahead as the ring allows (the down-projection rows stream in
+//             shared-memory byte ring, one mbarrier per stage; once routing
+//             is known the rest of the stage list is laid out in one step and
+//             issued in consumption order (the down-projection rows stream in
 //             while gate/up is still computing);
 //   consumers: [router rows -> grid barrier -> top-k + grouping (every CTA
 //             computes it, CTA 0 publishes it)] -> gate/up + SwiGLU into h ->
 //             grid barrier -> down rows of this CTA's output slice for every
 //             (expert, token) -> combine in top-k order -> y.
-// The shared expert's gate/up rows are fetched before routing is known and
-// are computed while other CTAs finish their router rows.
+// The shared expert's gate/up rows are fetched before routing is known; with
+// routing in the kernel they are computed right after it, while the routed
+// experts' rows are on their way.
 //
 // Grid barriers and every mbarrier wait are bounded by a global-timer limit;
 // on expiry the kernel records MOE_ETIMEOUT in the context's status word,

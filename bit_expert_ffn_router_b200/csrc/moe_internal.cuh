@@ -18,9 +18,9 @@ constexpr int kMaxE = 1024;           // experts per layer
 constexpr int kMaxK = 32;             // experts per token
 constexpr int kGroupChunk = 512;      // pairs per chunk in the multi-CTA grouping
 constexpr int kTileN = 128;           // tokens per tile of the prefill grouped GEMM
-// Copies of the small arrays every CTA of the decode kernel reads (logits,
-// slots, h): CTA b reads copy b % kRep, so each cache line has ~148/kRep
-// readers instead of all of them.
+// Copies of the small arrays every CTA of the decode kernel reads after a
+// grid barrier (logits, h): CTA b reads copy b % kRep, so each cache line has
+// ~148/kRep readers instead of all of them.
 constexpr int kRep = 8;
 
 // Device status word codes (word 0 holds the first error seen).
