@@ -158,6 +158,18 @@ def test_layer_decode_full(bits, T):
     H.assert_close_rows(H.y_as_f64(y), ref["y"])
 
 
+@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("T", [1, 4])
+def test_layer_decode_256_experts(bits, T):
+    # the pages' pruned variant keeps 256 of each layer's 512 experts
+    # (news.blueqat.app/post/3262, section 量子化の種類とサイズ); top-10 of
+    # 256 + shared
+    L = H.Layer(M.FULL.replace(bits=bits, E=256), T, seed=60 + T, zipf=True)
+    y, _ = L.forward()
+    ref = L.oracle()
+    H.assert_close_rows(H.y_as_f64(y), ref["y"])
+
+
 def test_layer_decode_full_unbiased_router_T8():
     L = H.Layer(M.FULL, 8, seed=5)
     y, ws = L.forward()

@@ -68,6 +68,16 @@ def test_layer_prefill_full_zipf(bits):
     H.assert_close_rows(H.y_as_f64(y)[toks], ref["y"])
 
 
+def test_layer_prefill_256_experts():
+    # the pages' pruned variant: 256 experts per layer (news.blueqat.app/post/3262,
+    # section 量子化の種類とサイズ), top-10 + shared
+    L = H.Layer(M.FULL.replace(E=256), 300, seed=61, zipf=True)
+    y, _ = L.forward()
+    toks = list(range(3, 300, 13))
+    ref = L.oracle(tokens=toks)
+    H.assert_close_rows(H.y_as_f64(y)[toks], ref["y"])
+
+
 @pytest.mark.parametrize("bits", [2, 3])
 def test_layer_prefill_chunk_8192_sampled(bits):
     # the pages' prefill chunk: 8,192 tokens x top-10 of 512 + shared expert
