@@ -170,6 +170,36 @@ def test_layer_decode_256_experts(bits, T):
     H.assert_close_rows(H.y_as_f64(y), ref["y"])
 
 
+@pytest.mark.parametrize("bits", [2, 3])
+def test_decode_expert_ffn_on_given_grouping(bits):
+    """The unfused decode entry points: moe_group_tokens on the oracle's routing,
+    then moe_expert_ffn_q{bits} with no pair buffer (the fused down + combine
+    writes y), against the oracle's layer output."""
+    T, cfg = 3, M.FULL.replace(bits=bits)
+    L = H.Layer(cfg, T, seed=71, zipf=True)
+    dv = L.device()
+    ref = L.oracle()
+    ctx = H.ctx()
+    ws = M.workspace(cfg, T)
+    idx = torch.from_numpy(ref["idx"].astype(np.int32)).cuda()
+    gate = torch.from_numpy(ref["gate"].astype(np.float32)).cuda()
+    g = ctx.group_tokens(cfg, idx, gate, T, dv["slot_of"], L.n_slots, ws)
+    y = L.out_tensor()
+    ctx.expert_ffn(cfg, dv["x"], g, dv["pool"], dv["stride"], dv["shared"], ws, z_rows=None, y=y)
+    torch.cuda.synchronize()
+    assert ctx.check_device_status() == M.OK
+    H.assert_close_rows(H.y_as_f64(y), ref["y"])
+
+
+def test_layer_decode_more_than_512_experts():
+    # E > 512 routes with the separate router / top-k / grouping kernels and
+    # runs the decode expert kernel on the published grouping
+    cfg = M.LayerCfg(d=256, f=128, E=600, k=4)
+    L = H.Layer(cfg, 2, seed=72, zipf=True)
+    y, _ = L.forward()
+    H.assert_close_rows(H.y_as_f64(y), L.oracle()["y"])
+
+
 def test_layer_decode_full_unbiased_router_T8():
     L = H.Layer(M.FULL, 8, seed=5)
     y, ws = L.forward()
