@@ -210,6 +210,11 @@ class Context:
         _check(self.layer_forward_status(cfg, x, T, w_router, bias, slot_of, n_slots, pool, stride, shared, ws, y,
                                          stream), "moe_layer_forward")
 
+    def prepare_layer_forward(self, cfg, T, w_router, bias, slot_of, n_slots, pool, stride, shared, ws,
+                              stream=None) -> "PreparedLayer":
+        """moe_layer_forward with every argument but x and y marshalled once (for launch loops)."""
+        return PreparedLayer(self, cfg, T, w_router, bias, slot_of, n_slots, pool, stride, shared, ws, stream)
+
     def check_device_status(self, stream=None) -> int:
         return self.lib.moe_check_device_status(self.h, _stream(stream))
 
@@ -219,6 +224,29 @@ class Context:
         buf = np.zeros((n_ctas, 32), dtype=np.uint64)
         _check(self.lib.moe_trace_fetch(self.h, buf.ctypes.data, buf.size, _stream(stream)), "moe_trace_fetch")
         return buf
+
+
+class PreparedLayer:
+    """A moe_layer_forward call whose layer arguments (configuration, weights,
+    slot table, pool, workspace, stream) are converted to ctypes values once;
+    each call marshals only x and y. It passes exactly the arguments
+    Context.layer_forward_status would, and keeps the tensors it points into
+    alive."""
+
+    def __init__(self, ctx, cfg, T, w_router, bias, slot_of, n_slots, pool, stride, shared, ws, stream=None):
+        self._fn = ctx.lib.moe_layer_forward
+        self._cfg = cfg.c()
+        self._keep = (ctx, w_router, bias, slot_of, pool, shared, ws)
+        self._head = (ctx.h, ctypes.byref(self._cfg))
+        self._mid = (T, _ptr(w_router), _ptr(bias), _ptr(slot_of), n_slots, _ptr(pool), stride, _ptr(shared),
+                     _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size())
+        self._stream = _stream(stream)
+
+    def status(self, x, y) -> int:
+        return self._fn(*self._head, _ptr(x), *self._mid, _ptr(y), self._stream)
+
+    def __call__(self, x, y) -> None:
+        _check(self.status(x, y), "moe_layer_forward")
 
 
 # ------------------------------------------------------------------ buffers

@@ -72,3 +72,45 @@ def test_null_context_rejected_without_gpu():
     assert lib.moe_router_topk(None, ctypes.byref(cfg), None, None, None, 1, None, None, None, None) == M.EINVAL
     assert lib.moe_check_device_status(None, None) == M.EINVAL
     assert lib.moe_ctx_create(0, None) == M.EINVAL
+
+
+def test_prepared_layer_forward_passes_the_same_arguments():
+    """PreparedLayer marshals each argument once; its calls must hand the C entry
+    point exactly what Context.layer_forward_status hands it."""
+    import torch
+
+    calls = []
+
+    class FakeLib:
+        def moe_layer_forward(self, *args):
+            calls.append(args)
+            return 0
+
+    class FakeCtx:
+        lib = FakeLib()
+        h = ctypes.c_void_p(1234)
+
+    class FakeStream:
+        cuda_stream = 4321
+
+    def norm(a):
+        if isinstance(a, ctypes.c_void_p):
+            return ("p", a.value)
+        if type(a).__name__ == "CArgObject":  # ctypes.byref(struct)
+            return ("ref", bytes(a._obj))
+        return ("v", a)
+
+    cfg = M.FULL.replace(bits=3, out_fp32=0, residual=1)
+    t = lambda n: torch.zeros(n, dtype=torch.uint8)  # noqa: E731  (CPU tensors: only data_ptr is read)
+    w, bias, slots, pool, shared, ws = t(64), t(16), t(32), t(256), t(128), t(4096)
+    x, y = t(8), t(8)
+    args = (cfg, 3, w, bias, slots, 40, pool, 1536, shared, ws)
+    prep = M.PreparedLayer(FakeCtx(), *args, stream=FakeStream())
+    assert prep.status(x, y) == 0
+    M.Context.layer_forward_status(FakeCtx(), cfg, x, 3, w, bias, slots, 40, pool, 1536, shared, ws, y,
+                                   stream=FakeStream())
+    assert len(calls) == 2
+    a, b = [tuple(norm(v) for v in c) for c in calls]
+    assert a == b
+    # the pointers are the tensors' own addresses, the sizes the workspace's bytes
+    assert ("p", x.data_ptr()) in a and ("p", y.data_ptr()) in a and ("v", 4096) in a
