@@ -485,10 +485,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tB16, const __grid_const
 // position 2i+1 <- column i+8.
 __global__ void __launch_bounds__(256) gather_x_kernel(const uint16_t* __restrict__ x,
                                                        const int32_t* __restrict__ pair_token, int n_pairs,
-                                                       int n_rows, int d, __half* __restrict__ xg) {
+                                                       int n_rows, int T, int d, __half* __restrict__ xg) {
   const int r = blockIdx.x;
   if (r >= n_rows) return;
-  const int t = r < n_pairs ? __ldg(pair_token + r) : r - n_pairs;
+  // the token index is clamped into [0, T): a grouping that saw a bad expert
+  // index (reported as MOE_EDEVICE) must still not steer a read out of x
+  const int t = min(max(r < n_pairs ? __ldg(pair_token + r) : r - n_pairs, 0), T - 1);
   const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
   uint4* dst = reinterpret_cast<uint4*>(xg + static_cast<size_t>(r) * d);
   for (int gi = threadIdx.x; gi < d / 16; gi += blockDim.x) {
@@ -660,7 +662,7 @@ cudaError_t launch_ffn_prefill(const Ctx& ctx, const moe_layer_cfg& c, const Ffn
                                                            a.g->pair_slot, c.E, a.T, w.n_pairs, a.shared != nullptr,
                                                            info);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  gather_x_kernel<<<w.n_rows, 128, 0, s>>>(a.x, a.g->pair_token, w.n_pairs, w.n_rows, c.d, xg);
+  gather_x_kernel<<<w.n_rows, 128, 0, s>>>(a.x, a.g->pair_token, w.n_pairs, w.n_rows, a.T, c.d, xg);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return c.bits == 2 ? run_ffn<2>(ctx, c, a, info, xg, h16, z_rows, w.n_pairs, w.n_rows, s)
                      : run_ffn<3>(ctx, c, a, info, xg, h16, z_rows, w.n_pairs, w.n_rows, s);

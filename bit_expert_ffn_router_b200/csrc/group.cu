@@ -99,12 +99,15 @@ __device__ int finish_counts(int e, int count, int E, int T, int n_pairs, int n_
   return off;
 }
 
+// The one mapping of an expert index every grouping pass applies: an index
+// outside [0, E) is filed under expert 0 (and reported once, by the counting
+// pass), so the counting and scatter passes agree on every pair's expert and
+// the sorted positions stay a permutation of [0, T*k).
+__device__ __forceinline__ int mapped_expert(int e, int E) { return (e < 0 || e >= E) ? 0 : e; }
+
 __device__ __forceinline__ int checked_expert(int e, int E, int p, int* status) {
-  if (e < 0 || e >= E) {
-    report(status, kDevBadExpert, p);
-    return 0;
-  }
-  return e;
+  if (e < 0 || e >= E) report(status, kDevBadExpert, p);
+  return mapped_expert(e, E);
 }
 
 // ---------------------------------------------------------------- one CTA (small T*k)
@@ -159,7 +162,7 @@ group_chunk_kernel(const int32_t* __restrict__ idx, const float* __restrict__ ga
     const int p = pb + lane;
     const bool valid = p < p1;
     int e = -1;
-    if (valid) e = kScatter ? min(max(idx[p], 0), E - 1) : checked_expert(idx[p], E, p, status);
+    if (valid) e = kScatter ? mapped_expert(idx[p], E) : checked_expert(idx[p], E, p, status);
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(peers & ((1u << lane) - 1u));
     const int before = valid ? cnt[e] : 0;

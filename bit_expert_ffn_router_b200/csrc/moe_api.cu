@@ -23,7 +23,11 @@ WsLayout ws_layout(const moe_layer_cfg& c, int T) {
     o = align_up(o + bytes, 256);
     return at;
   };
-  w.logits = take(Tz * c.E * 4);
+  const bool decode = T <= MOE_DECODE_MAX_T;
+  // logits [T, E]; on the decode path kRep copies of them, the first being
+  // the logits array itself
+  w.logits = take((decode ? kRep : 1) * Tz * c.E * 4);
+  w.logits_rep = w.logits;
   w.idx = take(Tz * c.k * 4);
   w.gate = take(Tz * c.k * 4);
   w.expert_count = take(static_cast<size_t>(c.E) * 4);
@@ -39,8 +43,6 @@ WsLayout ws_layout(const moe_layer_cfg& c, int T) {
   w.n_uniq = take(16);
   w.chunk_hist = take(static_cast<size_t>(w.n_chunks) * c.E * 4);
   w.tile_offset = take((static_cast<size_t>(c.E) + 2) * 4);
-  const bool decode = T <= MOE_DECODE_MAX_T;
-  w.logits_rep = take(decode ? static_cast<size_t>(kRep) * Tz * c.E * 4 : 0);
   // h: fp32 rows (kRep copies) on the decode path, fp16 rows (padded by one
   // tile) on the prefill path
   const size_t h32 = static_cast<size_t>(decode ? kRep : 1) * w.n_rows * c.f * 4;
@@ -93,20 +95,28 @@ static bool aligned(const void* p, size_t a) {
 
 static thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
+void record_cuda_error(cudaError_t e) {
+  if (e != cudaSuccess) g_last_cuda_error = e;
+}
+
 static moe_status from_cuda(cudaError_t e) {
   if (e == cudaSuccess) return MOE_OK;
   g_last_cuda_error = e;
   return MOE_ECUDA;
 }
 
-// Makes the context's device current for this host thread (kernels launch on
-// the runtime's current device).
-static bool use_device(const moe_ctx* ctx) {
-  int cur = -1;
-  cudaError_t e = cudaGetDevice(&cur);
-  if (e == cudaSuccess && cur != ctx->c.device) e = cudaSetDevice(ctx->c.device);
-  if (e != cudaSuccess) g_last_cuda_error = e;
-  return e == cudaSuccess;
+DeviceGuard::DeviceGuard(int device) {
+  cudaError_t e = cudaGetDevice(&prev);
+  if (e == cudaSuccess && prev != device) {
+    e = cudaSetDevice(device);
+    switched = e == cudaSuccess;
+  }
+  ok = e == cudaSuccess;
+  record_cuda_error(e);
+}
+
+DeviceGuard::~DeviceGuard() {
+  if (switched) cudaSetDevice(prev);
 }
 
 static moe_expert_layout layout_of(const moe_layer_cfg& c) {
@@ -163,7 +173,8 @@ static moe_status run_ffn(moe_ctx* ctx, const moe_layer_cfg* cfg, int bits, cons
                           const uint8_t* shared, void* ws, size_t ws_bytes, float* z_rows,
                           void* y, moe_stream stream) {
   if (ctx == nullptr || grp == nullptr) return MOE_EINVAL;
-  if (!use_device(ctx)) return MOE_ECUDA;
+  DeviceGuard dg(ctx->c.device);
+  if (!dg.ok) return MOE_ECUDA;
   moe_status st = check_cfg(cfg);
   if (st != MOE_OK) return st;
   if (cfg->bits != bits) return MOE_EINVAL;
@@ -225,7 +236,8 @@ moe_status moe_ctx_create(int device, moe_ctx** out) {
   moe_ctx* ctx = new (std::nothrow) moe_ctx;
   if (ctx == nullptr) return MOE_EINVAL;
   ctx->c.device = device;
-  if (cudaSetDevice(device) != cudaSuccess ||
+  DeviceGuard dg(device);
+  if (!dg.ok ||
       cudaDeviceGetAttribute(&ctx->c.num_sms, cudaDevAttrMultiProcessorCount, ctx->c.device) !=
           cudaSuccess ||
       cudaMalloc(&ctx->c.d_status, 64) != cudaSuccess) {
@@ -258,7 +270,7 @@ moe_status moe_ctx_create(int device, moe_ctx** out) {
 
 void moe_ctx_destroy(moe_ctx* ctx) {
   if (ctx == nullptr) return;
-  use_device(ctx);
+  DeviceGuard dg(ctx->c.device);
   if (ctx->c.d_trace != nullptr) cudaFree(ctx->c.d_trace);
   cudaFree(ctx->c.d_status);
   delete ctx;
@@ -281,7 +293,8 @@ const char* moe_status_string(moe_status s) {
 
 moe_status moe_check_device_status(moe_ctx* ctx, moe_stream stream) {
   if (ctx == nullptr) return MOE_EINVAL;
-  if (!use_device(ctx)) return MOE_ECUDA;
+  DeviceGuard dg(ctx->c.device);
+  if (!dg.ok) return MOE_ECUDA;
   int h[4] = {0, 0, 0, 0};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemcpyAsync(h, ctx->c.d_status, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
@@ -298,7 +311,8 @@ moe_status moe_check_device_status(moe_ctx* ctx, moe_stream stream) {
 moe_status moe_trace_fetch(moe_ctx* ctx, unsigned long long* host, int n, moe_stream stream) {
   if (ctx == nullptr || host == nullptr || n < 0) return MOE_EINVAL;
   if (ctx->c.d_trace == nullptr) return MOE_EINVAL;
-  if (!use_device(ctx)) return MOE_ECUDA;
+  DeviceGuard dg(ctx->c.device);
+  if (!dg.ok) return MOE_ECUDA;
   const int cap = kTraceCtas * kTraceSlots;
   const size_t bytes = static_cast<size_t>(n < cap ? n : cap) * sizeof(unsigned long long);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -307,6 +321,23 @@ moe_status moe_trace_fetch(moe_ctx* ctx, unsigned long long* host, int n, moe_st
       cudaStreamSynchronize(s) != cudaSuccess)
     return from_cuda(cudaGetLastError());
   return MOE_OK;
+}
+
+moe_status moe_layer_routing(const moe_layer_cfg* cfg, int T, void* ws, size_t ws_bytes, moe_routing* out) {
+  if (out == nullptr) return MOE_EINVAL;
+  const moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0 || ws == nullptr || !aligned(ws, 256)) return MOE_EINVAL;
+  const WsLayout w = ws_layout(*cfg, T);
+  if (ws_bytes < w.total) return MOE_ENOSPACE;
+  char* b = static_cast<char*>(ws);
+  out->T = T;
+  out->k = cfg->k;
+  out->E = cfg->E;
+  out->logits = reinterpret_cast<float*>(b + w.logits);
+  out->idx = reinterpret_cast<int32_t*>(b + w.idx);
+  out->gate = reinterpret_cast<float*>(b + w.gate);
+  return fill_grouping(*cfg, T, ws, &out->grouping);
 }
 
 moe_status moe_expert_layout_get(const moe_layer_cfg* cfg, moe_expert_layout* out) {
@@ -326,7 +357,8 @@ moe_status moe_router_topk(moe_ctx* ctx, const moe_layer_cfg* cfg, const void* x
                            const float* w_router, const float* logit_bias, int T, float* logits,
                            int32_t* idx, float* gate, moe_stream stream) {
   if (ctx == nullptr) return MOE_EINVAL;
-  if (!use_device(ctx)) return MOE_ECUDA;
+  DeviceGuard dg(ctx->c.device);
+  if (!dg.ok) return MOE_ECUDA;
   moe_status st = check_cfg(cfg);
   if (st != MOE_OK) return st;
   if (T < 0) return MOE_EINVAL;
@@ -344,7 +376,8 @@ moe_status moe_router_topk(moe_ctx* ctx, const moe_layer_cfg* cfg, const void* x
 moe_status moe_topk(moe_ctx* ctx, const moe_layer_cfg* cfg, const float* logits, int T,
                     int32_t* idx, float* gate, moe_stream stream) {
   if (ctx == nullptr) return MOE_EINVAL;
-  if (!use_device(ctx)) return MOE_ECUDA;
+  DeviceGuard dg(ctx->c.device);
+  if (!dg.ok) return MOE_ECUDA;
   moe_status st = check_cfg(cfg);
   if (st != MOE_OK) return st;
   if (T < 0) return MOE_EINVAL;
@@ -357,7 +390,8 @@ moe_status moe_group_tokens(moe_ctx* ctx, const moe_layer_cfg* cfg, const int32_
                             const float* gate, int T, const int32_t* slot_of, int n_slots,
                             void* ws, size_t ws_bytes, moe_grouping* out, moe_stream stream) {
   if (ctx == nullptr || out == nullptr) return MOE_EINVAL;
-  if (!use_device(ctx)) return MOE_ECUDA;
+  DeviceGuard dg(ctx->c.device);
+  if (!dg.ok) return MOE_ECUDA;
   moe_status st = check_cfg(cfg);
   if (st != MOE_OK) return st;
   if (T < 0 || n_slots <= 0) return MOE_EINVAL;
@@ -390,7 +424,8 @@ moe_status moe_expert_ffn_q3(moe_ctx* ctx, const moe_layer_cfg* cfg, const void*
 moe_status moe_combine(moe_ctx* ctx, const moe_layer_cfg* cfg, const moe_grouping* grouping,
                        const float* z_rows, const void* x, int T, void* y, moe_stream stream) {
   if (ctx == nullptr || grouping == nullptr) return MOE_EINVAL;
-  if (!use_device(ctx)) return MOE_ECUDA;
+  DeviceGuard dg(ctx->c.device);
+  if (!dg.ok) return MOE_ECUDA;
   moe_status st = check_cfg(cfg);
   if (st != MOE_OK) return st;
   if (T < 0 || grouping->T != T || grouping->k != cfg->k) return MOE_EINVAL;
@@ -408,7 +443,8 @@ moe_status moe_layer_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, const void*
                              size_t slot_stride, const uint8_t* shared_expert, void* ws,
                              size_t ws_bytes, void* y, moe_stream stream) {
   if (ctx == nullptr) return MOE_EINVAL;
-  if (!use_device(ctx)) return MOE_ECUDA;
+  DeviceGuard dg(ctx->c.device);
+  if (!dg.ok) return MOE_ECUDA;
   moe_status st = check_cfg(cfg);
   if (st != MOE_OK) return st;
   if (T < 0 || n_slots <= 0) return MOE_EINVAL;

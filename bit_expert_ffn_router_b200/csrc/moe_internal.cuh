@@ -35,6 +35,7 @@ struct Ctx {
   unsigned long long* d_gbar = nullptr;  // grid-barrier arrival counter of the decode kernel
   unsigned long long timeout_ns = 200ull * 1000 * 1000;  // limit of every device-side wait
   unsigned long long* d_trace = nullptr;  // phase timestamps (MOE_TRACE), kTraceSlots per CTA
+  void* static_scratch = nullptr;  // device address of the static scratch (first static call)
 };
 constexpr int kTraceSlots = 32;
 constexpr int kTraceCtas = 1024;
@@ -63,6 +64,23 @@ struct WsLayout {
 };
 
 WsLayout ws_layout(const moe_layer_cfg& c, int T);
+
+// Makes `device` current for the lifetime of the guard and then restores the
+// caller's current device, so that no entry point leaves the host thread on
+// another device than it found.
+struct DeviceGuard {
+  explicit DeviceGuard(int device);
+  ~DeviceGuard();
+  DeviceGuard(const DeviceGuard&) = delete;
+  DeviceGuard& operator=(const DeviceGuard&) = delete;
+  bool ok = false;
+  bool switched = false;
+  int prev = 0;
+};
+
+// Records a failed CUDA call as the host thread's last error (read by
+// moe_last_cuda_error).
+void record_cuda_error(cudaError_t e);
 
 // ---------------------------------------------------------------- device helpers
 

@@ -9,8 +9,6 @@
 // The array is part of the library's device image: the driver reserves it on
 // each device when the module loads there, so no call allocates. The step
 // itself is the unchanged moe_layer_forward, given the array as workspace.
-#include <mutex>
-
 #include "moe_internal.cuh"
 
 namespace {
@@ -25,21 +23,18 @@ static_assert(kStaticScratchBytes % 256 == 0, "scratch size");
 // earlier in the same call.
 static __device__ __align__(256) unsigned char g_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_scratch on `device`, looked up once per device with the
-// device current (the caller has made it current).
-cudaError_t scratch_on(int device, void** out) {
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_ptr[device] == nullptr) {
+// Device address of g_scratch on the context's device, looked up on the
+// context's first call with that device current and kept in the context. A
+// context lives on one device and does not outlive a reset of it, so the
+// address it holds stays valid for as long as the context does.
+cudaError_t scratch_of(moe::Ctx& c, void** out) {
+  if (c.static_scratch == nullptr) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_ptr[device] = p;
+    c.static_scratch = p;
   }
-  *out = g_scratch_ptr[device];
+  *out = c.static_scratch;
   return cudaSuccess;
 }
 
@@ -52,15 +47,17 @@ moe_status moe_layer_forward_static(moe_ctx* ctx, const moe_layer_cfg* cfg, cons
                                     int n_slots, const uint8_t* slot_pool, size_t slot_stride,
                                     const uint8_t* shared_expert, void* y, moe_stream stream) {
   if (ctx == nullptr || cfg == nullptr || T < 0) return MOE_EINVAL;
-  if (ctx->c.device < 0 || ctx->c.device >= kMaxDevices) return MOE_EUNSUPPORTED;
   const size_t need = moe_workspace_bytes(cfg, T);
   if (need == 0) return MOE_EINVAL;  // invalid configuration
   if (need > kStaticScratchBytes) return MOE_ENOSPACE;
-  int cur = -1;
-  if (cudaGetDevice(&cur) != cudaSuccess) return MOE_ECUDA;
-  if (cur != ctx->c.device && cudaSetDevice(ctx->c.device) != cudaSuccess) return MOE_ECUDA;
+  moe::DeviceGuard dg(ctx->c.device);
+  if (!dg.ok) return MOE_ECUDA;
   void* scratch = nullptr;
-  if (scratch_on(ctx->c.device, &scratch) != cudaSuccess) return MOE_ECUDA;
+  const cudaError_t e = scratch_of(ctx->c, &scratch);
+  if (e != cudaSuccess) {
+    moe::record_cuda_error(e);
+    return MOE_ECUDA;
+  }
   return moe_layer_forward(ctx, cfg, x, T, w_router, logit_bias, slot_of, n_slots, slot_pool, slot_stride,
                            shared_expert, scratch, kStaticScratchBytes, y, stream);
 }

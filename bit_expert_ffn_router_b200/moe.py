@@ -44,6 +44,12 @@ class Grouping(ctypes.Structure):
          "uniq_expert", "uniq_slot", "uniq_offset", "n_uniq", "internal")]
 
 
+class Routing(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int), ("k", ctypes.c_int), ("E", ctypes.c_int),
+                ("logits", ctypes.c_void_p), ("idx", ctypes.c_void_p), ("gate", ctypes.c_void_p),
+                ("grouping", Grouping)]
+
+
 @dataclasses.dataclass(frozen=True)
 class LayerCfg:
     d: int
@@ -89,6 +95,7 @@ _SIGS = {
     "moe_combine": (_I, [_P, ctypes.POINTER(_Cfg), ctypes.POINTER(Grouping), _P, _P, _I, _P, _S]),
     "moe_layer_forward": (_I, [_P, ctypes.POINTER(_Cfg), _P, _I, _P, _P, _P, _I, _P, _Z, _P, _P, _Z, _P,
                                _S]),
+    "moe_layer_routing": (_I, [ctypes.POINTER(_Cfg), _I, _P, _Z, ctypes.POINTER(Routing)]),
     "moe_layer_forward_static": (_I, [_P, ctypes.POINTER(_Cfg), _P, _I, _P, _P, _P, _I, _P, _Z, _P, _P, _S]),
 }
 
@@ -214,6 +221,41 @@ class Context:
                               stream=None) -> "PreparedLayer":
         """moe_layer_forward with every argument but x and y marshalled once (for launch loops)."""
         return PreparedLayer(self, cfg, T, w_router, bias, slot_of, n_slots, pool, stride, shared, ws, stream)
+
+    def layer_routing(self, cfg, T, ws) -> dict:
+        """The routing a whole-step call with workspace `ws` computed (moe_layer_routing), as torch views
+        into ws: logits [T,E], idx [T,k], gate [T,k] and the grouping arrays. Read them after the call
+        has completed on its stream."""
+        import torch
+        r = Routing()
+        nbytes = ws.numel() * ws.element_size()
+        _check(self.lib.moe_layer_routing(ctypes.byref(cfg.c()), T, _ptr(ws), nbytes, ctypes.byref(r)),
+               "moe_layer_routing")
+        raw = ws.view(torch.uint8).view(-1)
+        base = ws.data_ptr()
+
+        def view(ptr, n, dtype):
+            off = ptr - base
+            return raw[off:off + 4 * n].view(dtype)
+
+        g = r.grouping
+        n_pairs, nu_max = T * cfg.k, min(T * cfg.k, cfg.E)
+        return {
+            "logits": view(r.logits, T * cfg.E, torch.float32).view(T, cfg.E),
+            "idx": view(r.idx, T * cfg.k, torch.int32).view(T, cfg.k),
+            "gate": view(r.gate, T * cfg.k, torch.float32).view(T, cfg.k),
+            "expert_count": view(g.expert_count, cfg.E, torch.int32),
+            "expert_offset": view(g.expert_offset, cfg.E + 1, torch.int32),
+            "pair_token": view(g.pair_token, n_pairs, torch.int32),
+            "pair_j": view(g.pair_j, n_pairs, torch.int32),
+            "pair_gate": view(g.pair_gate, n_pairs, torch.float32),
+            "pair_slot": view(g.pair_slot, n_pairs, torch.int32),
+            "pair_pos": view(g.pair_pos, n_pairs, torch.int32),
+            "uniq_expert": view(g.uniq_expert, nu_max, torch.int32),
+            "uniq_slot": view(g.uniq_slot, nu_max, torch.int32),
+            "uniq_offset": view(g.uniq_offset, nu_max + 1, torch.int32),
+            "n_uniq": view(g.n_uniq, 1, torch.int32),
+        }
 
     def check_device_status(self, stream=None) -> int:
         return self.lib.moe_check_device_status(self.h, _stream(stream))

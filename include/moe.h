@@ -219,6 +219,26 @@ MOE_API moe_status moe_layer_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, con
                              size_t slot_stride, const uint8_t* shared_expert, void* ws,
                              size_t ws_bytes, void* y, moe_stream stream);
 
+/* The routing a whole-step call computed, as views into its workspace.
+ * After moe_layer_forward(cfg, T, ws) has completed on its stream, the
+ * workspace holds that step's router logits, top-k and grouping; this fills
+ * *out with device pointers to them (no device work, no synchronisation):
+ *   logits [T, E] fp32 (router output plus bias), idx [T, k] int32 and
+ *   gate [T, k] fp32 (as moe_router_topk), grouping (as moe_group_tokens).
+ * The same views serve moe_router_topk / moe_group_tokens callers that pass
+ * this workspace. A later call with the same workspace overwrites them.
+ * This is the per-token expert choice the pages' engine logs and tallies to
+ * pick its hot experts (vramglass.com, section その1). */
+typedef struct {
+  int T, k, E;
+  float* logits;
+  int32_t* idx;
+  float* gate;
+  moe_grouping grouping;
+} moe_routing;
+MOE_API moe_status moe_layer_routing(const moe_layer_cfg* cfg, int T, void* ws, size_t ws_bytes,
+                                     moe_routing* out);
+
 /* moe_layer_forward without a workspace argument: the step's scratch is a
  * static device array of MOE_STATIC_SCRATCH_BYTES inside the library image,
  * reserved on each device when the library's module loads there, so the call

@@ -11,6 +11,8 @@ Tolerances:
 """
 from __future__ import annotations
 
+import copy
+
 import numpy as np
 import torch
 
@@ -79,6 +81,22 @@ class Layer:
                 "pool": pool, "stride": stride, "shared": shared,
             }
         return self._dev
+
+    def with_inputs(self, x, bias, wr=None):
+        """The same experts, pool and slot table with other tokens (x [T,d] bf16 bits, bias [T,E] or
+        None) and optionally another router matrix; the device pool is shared, not rebuilt."""
+        L = copy.copy(self)
+        L.T = x.shape[0]
+        L.x = x
+        L.bias = None if bias is None else np.asarray(bias, dtype=np.float32)
+        if wr is not None:
+            L.wr = np.asarray(wr, dtype=np.float32)
+        dv = dict(self.device())
+        dv["x"] = torch.from_numpy(np.ascontiguousarray(L.x).view(np.int16)).cuda()
+        dv["bias"] = None if L.bias is None else torch.from_numpy(L.bias).cuda()
+        dv["wr"] = torch.from_numpy(L.wr).cuda()
+        L._dev = dv
+        return L
 
     def out_tensor(self):
         dt = torch.float32 if self.cfg.out_fp32 else torch.bfloat16

@@ -137,6 +137,38 @@ def test_grouping_reports_bad_indices():
     assert H.ctx().check_device_status() == M.EDEVICE
 
 
+def test_multi_cta_grouping_reports_bad_index_and_keeps_a_permutation():
+    """T*k > 512 takes the multi-CTA grouping; an expert index = E is reported
+    as MOE_EDEVICE, filed under expert 0 by both of its passes, and the sorted
+    positions still form a permutation of [0, T*k)."""
+    cfg = M.FULL
+    T = 60
+    g = np.random.default_rng(17)
+    idx = np.stack([g.choice(cfg.E, size=cfg.k, replace=False) for _ in range(T)]).astype(np.int32)
+    idx[7, 3] = cfg.E
+    idx[40, 0] = -1
+    gate = g.random((T, cfg.k)).astype(np.float32)
+    ws = M.workspace(cfg, T)
+    ws.fill_(0xAB)  # stale contents must not survive anywhere in the result
+    grp = H.ctx().group_tokens(cfg, torch.from_numpy(idx).cuda(), torch.from_numpy(gate).cuda(), T,
+                               torch.arange(cfg.E, dtype=torch.int32, device="cuda"), cfg.E, ws)
+    assert H.ctx().check_device_status() == M.EDEVICE
+    n = T * cfg.k
+    raw = ws.view(torch.uint8)
+
+    def dev(ptr, count):
+        return raw[ptr - ws.data_ptr():][: count * 4].view(torch.int32).cpu().numpy()
+
+    pos = dev(grp.pair_pos, n)
+    assert np.array_equal(np.sort(pos), np.arange(n))
+    mapped = np.where((idx < 0) | (idx >= cfg.E), 0, idx)
+    ref = O.group(mapped, gate, cfg.E)
+    assert np.array_equal(pos, ref["pair_pos"].reshape(-1))
+    assert np.array_equal(dev(grp.pair_token, n), ref["pair_token"])
+    assert np.array_equal(dev(grp.expert_count, cfg.E), ref["expert_count"])
+    assert H.ctx().check_device_status() == M.OK
+
+
 # ------------------------------------------------------------------ whole layer, decode path
 
 @pytest.mark.parametrize("bits", [2, 3])
