@@ -16,7 +16,7 @@ OBJDIR = os.path.join(HERE, "_build")
 LIB = os.path.join(LIBDIR, "libmoe.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
-SOURCES = ["moe_api.cu", "router.cu", "router_tc.cu", "group.cu", "decode_layer.cu", "ffn_prefill.cu",
+SOURCES = ["moe_api.cu", "router.cu", "router_tc.cu", "group.cu", "decode_stack.cu", "ffn_prefill.cu",
            "combine.cu", "noalloc.cu"]
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = [

@@ -23,11 +23,8 @@ WsLayout ws_layout(const moe_layer_cfg& c, int T) {
     o = align_up(o + bytes, 256);
     return at;
   };
-  const bool decode = T <= MOE_DECODE_MAX_T;
-  // logits [T, E]; on the decode path kRep copies of them, the first being
-  // the logits array itself
-  w.logits = take((decode ? kRep : 1) * Tz * c.E * 4);
-  w.logits_rep = w.logits;
+  // routing record
+  w.logits = take(Tz * c.E * 4);
   w.idx = take(Tz * c.k * 4);
   w.gate = take(Tz * c.k * 4);
   w.expert_count = take(static_cast<size_t>(c.E) * 4);
@@ -41,17 +38,20 @@ WsLayout ws_layout(const moe_layer_cfg& c, int T) {
   w.uniq_slot = take(static_cast<size_t>(w.n_uniq_max) * 4);
   w.uniq_offset = take((static_cast<size_t>(w.n_uniq_max) + 1) * 4);
   w.n_uniq = take(16);
+  w.rec_bytes = o;
+  // grouping kernels' scratch
   w.chunk_hist = take(static_cast<size_t>(w.n_chunks) * c.E * 4);
   w.tile_offset = take((static_cast<size_t>(c.E) + 2) * 4);
-  // h: fp32 rows (kRep copies) on the decode path, fp16 rows (padded by one
-  // tile) on the prefill path
-  const size_t h32 = static_cast<size_t>(decode ? kRep : 1) * w.n_rows * c.f * 4;
-  const size_t h16 = (static_cast<size_t>(w.n_rows) + kTileN) * c.f * 2;
-  w.h = take(h32 > h16 ? h32 : h16);
-  w.z = take(T > MOE_DECODE_MAX_T ? static_cast<size_t>(w.n_rows) * c.d * 4 : 0);
-  // x gathered into pair order as fp16 (prefill grouped GEMM operand)
-  w.x16 = take(static_cast<size_t>(w.n_rows) * c.d * 2);
-  w.tile_info = take((static_cast<size_t>(w.n_rows) / kTileN + c.E + 2) * 16);
+  if (T <= MOE_DECODE_MAX_T) {
+    w.exchange = take(decode_exchange_bytes(c, T));
+  } else {
+    // h: fp16 rows padded by one tile; z: the fp32 pair buffer; x gathered
+    // into pair order as fp16 (the grouped GEMM's operand)
+    w.h = take((static_cast<size_t>(w.n_rows) + kTileN) * c.f * 2);
+    w.z = take(static_cast<size_t>(w.n_rows) * c.d * 4);
+    w.x16 = take(static_cast<size_t>(w.n_rows) * c.d * 2);
+    w.tile_info = take((static_cast<size_t>(w.n_rows) / kTileN + c.E + 2) * 16);
+  }
   w.total = o;
   return w;
 }
@@ -201,20 +201,20 @@ static moe_status run_ffn(moe_ctx* ctx, const moe_layer_cfg* cfg, int bits, cons
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (z_rows == nullptr) {
     if (T > MOE_DECODE_MAX_T || y == nullptr || !aligned(y, 16)) return MOE_EINVAL;
-    DecodeArgs d{};
+    StackArgs d{};
     d.route = false;
     d.x = a.x;
     d.T = T;
+    d.L = 1;
     d.n_slots = 0x7fffffff;
     d.g = &g;
     d.pool = pool;
     d.stride = stride;
     d.shared = a.shared;
     d.lay = a.lay;
-    d.h = reinterpret_cast<float*>(a.h);
     d.y = y;
-    d.logits_rep = reinterpret_cast<float*>(static_cast<char*>(ws) + w.logits_rep);
-    const cudaError_t e = launch_decode_layer(ctx->c, *cfg, d, s);
+    d.exchange = static_cast<char*>(ws) + w.exchange;
+    const cudaError_t e = launch_decode_stack(ctx->c, *cfg, d, s);
     if (e == cudaErrorNotSupported) return MOE_EUNSUPPORTED;
     return from_cuda(e);
   }
@@ -222,6 +222,53 @@ static moe_status run_ffn(moe_ctx* ctx, const moe_layer_cfg* cfg, int bits, cons
   const cudaError_t e = launch_ffn_prefill(ctx->c, *cfg, a, ws, z_rows, s);
   if (e == cudaErrorNotSupported) return MOE_EUNSUPPORTED;
   return from_cuda(e);
+}
+
+// The fused decode kernel over L chained layers (L = 1: moe_layer_forward).
+// Arguments are checked by the caller; ws holds L routing records followed
+// by the rest of a one-layer workspace.
+static moe_status run_stack(moe_ctx* ctx, const moe_layer_cfg& c, int L, const void* x, int T,
+                            const float* w_router, const float* logit_bias, const int32_t* slot_of,
+                            int n_slots, const uint8_t* pool, size_t stride, const uint8_t* shared, void* ws,
+                            void* y, moe_stream stream) {
+  const WsLayout w = ws_layout(c, T);
+  char* b = static_cast<char*>(ws);
+  StackArgs d{};
+  d.route = true;
+  d.x = static_cast<const uint16_t*>(x);
+  d.T = T;
+  d.L = L;
+  d.wr = w_router;
+  d.bias = logit_bias;
+  d.slot_of = slot_of;
+  d.n_slots = n_slots;
+  d.pool = pool;
+  d.stride = stride;
+  d.shared = c.n_shared ? shared : nullptr;
+  d.lay = layout_of(c);
+  d.y = y;
+  d.rec = b;
+  d.rec_bytes = w.rec_bytes;
+  const size_t offs[14] = {w.logits, w.idx, w.gate, w.expert_count, w.expert_offset, w.pair_token, w.pair_j,
+                           w.pair_gate, w.pair_slot, w.pair_pos, w.uniq_expert, w.uniq_slot, w.uniq_offset,
+                           w.n_uniq};
+  for (int i = 0; i < 14; ++i) d.ro[i] = static_cast<int>(offs[i]);
+  d.exchange = b + static_cast<size_t>(L - 1) * w.rec_bytes + w.exchange;
+  const cudaError_t e = launch_decode_stack(ctx->c, c, d, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return MOE_EUNSUPPORTED;
+  return from_cuda(e);
+}
+
+static moe_status fill_routing(const moe_layer_cfg& c, int T, void* rec, moe_routing* out) {
+  const WsLayout w = ws_layout(c, T);
+  char* b = static_cast<char*>(rec);
+  out->T = T;
+  out->k = c.k;
+  out->E = c.E;
+  out->logits = reinterpret_cast<float*>(b + w.logits);
+  out->idx = reinterpret_cast<int32_t*>(b + w.idx);
+  out->gate = reinterpret_cast<float*>(b + w.gate);
+  return fill_grouping(c, T, rec, &out->grouping);
 }
 
 }  // namespace moe
@@ -244,7 +291,6 @@ moe_status moe_ctx_create(int device, moe_ctx** out) {
     delete ctx;
     return MOE_ECUDA;
   }
-  ctx->c.d_gbar = reinterpret_cast<unsigned long long*>(ctx->c.d_status + 8);
   // limit of every device-side wait (default 200 ms): MOE_TIMEOUT_US overrides it
   if (const char* t = getenv("MOE_TIMEOUT_US")) {
     const long long us = atoll(t);
@@ -301,9 +347,10 @@ moe_status moe_check_device_status(moe_ctx* ctx, moe_stream stream) {
       cudaStreamSynchronize(s) != cudaSuccess)
     return MOE_ECUDA;
   if (h[0] == 0) return MOE_OK;
-  // clear the status word and the decode kernel's grid-barrier words (an
-  // interrupted barrier leaves them mid-episode)
-  if (cudaMemsetAsync(ctx->c.d_status, 0, 64, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+  // clear the status word, and move the decode kernel's tag counter past any
+  // tag an interrupted launch may have written
+  if (cudaMemsetAsync(ctx->c.d_status, 0, 64, s) != cudaSuccess || decode_skip_tags(s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
     return MOE_ECUDA;
   return h[0] == kDevTimeout ? MOE_ETIMEOUT : MOE_EDEVICE;
 }
@@ -328,16 +375,48 @@ moe_status moe_layer_routing(const moe_layer_cfg* cfg, int T, void* ws, size_t w
   const moe_status st = check_cfg(cfg);
   if (st != MOE_OK) return st;
   if (T < 0 || ws == nullptr || !aligned(ws, 256)) return MOE_EINVAL;
+  if (ws_bytes < ws_layout(*cfg, T).rec_bytes) return MOE_ENOSPACE;
+  return fill_routing(*cfg, T, ws, out);
+}
+
+size_t moe_stack_workspace_bytes(const moe_layer_cfg* cfg, int L, int T) {
+  if (check_cfg(cfg) != MOE_OK || L < 1 || T < 0 || T > MOE_DECODE_MAX_T) return 0;
   const WsLayout w = ws_layout(*cfg, T);
-  if (ws_bytes < w.total) return MOE_ENOSPACE;
-  char* b = static_cast<char*>(ws);
-  out->T = T;
-  out->k = cfg->k;
-  out->E = cfg->E;
-  out->logits = reinterpret_cast<float*>(b + w.logits);
-  out->idx = reinterpret_cast<int32_t*>(b + w.idx);
-  out->gate = reinterpret_cast<float*>(b + w.gate);
-  return fill_grouping(*cfg, T, ws, &out->grouping);
+  return static_cast<size_t>(L - 1) * w.rec_bytes + w.total;
+}
+
+moe_status moe_stack_routing(const moe_layer_cfg* cfg, int L, int T, void* ws, size_t ws_bytes, int layer,
+                             moe_routing* out) {
+  if (out == nullptr) return MOE_EINVAL;
+  const moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (L < 1 || layer < 0 || layer >= L || T < 0 || T > MOE_DECODE_MAX_T) return MOE_EINVAL;
+  if (ws == nullptr || !aligned(ws, 256)) return MOE_EINVAL;
+  if (ws_bytes < moe_stack_workspace_bytes(cfg, L, T)) return MOE_ENOSPACE;
+  const WsLayout w = ws_layout(*cfg, T);
+  return fill_routing(*cfg, T, static_cast<char*>(ws) + static_cast<size_t>(layer) * w.rec_bytes, out);
+}
+
+moe_status moe_stack_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, int L, const void* x, int T,
+                             const float* w_router, const float* logit_bias, const int32_t* slot_of, int n_slots,
+                             const uint8_t* slot_pool, size_t slot_stride, const uint8_t* shared_experts,
+                             void* ws, size_t ws_bytes, void* y, moe_stream stream) {
+  if (ctx == nullptr) return MOE_EINVAL;
+  DeviceGuard dg(ctx->c.device);
+  if (!dg.ok) return MOE_ECUDA;
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (L < 1 || T < 0 || T > MOE_DECODE_MAX_T || n_slots <= 0) return MOE_EINVAL;
+  if (cfg->E > 512) return MOE_EUNSUPPORTED;
+  if (L > 1 && cfg->out_fp32) return MOE_EINVAL;  // layer l + 1 reads layer l's bf16 output
+  if (T == 0) return MOE_OK;
+  if (x == nullptr || w_router == nullptr || slot_of == nullptr || y == nullptr) return MOE_EINVAL;
+  if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(y, 16)) return MOE_EINVAL;
+  if (ws == nullptr || !aligned(ws, 256)) return MOE_EINVAL;
+  if (ws_bytes < moe_stack_workspace_bytes(cfg, L, T)) return MOE_ENOSPACE;
+  if ((st = check_pool(*cfg, slot_pool, slot_stride, shared_experts)) != MOE_OK) return st;
+  return run_stack(ctx, *cfg, L, x, T, w_router, logit_bias, slot_of, n_slots, slot_pool, slot_stride,
+                   shared_experts, ws, y, stream);
 }
 
 moe_status moe_expert_layout_get(const moe_layer_cfg* cfg, moe_expert_layout* out) {
@@ -459,32 +538,9 @@ moe_status moe_layer_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, const void*
   float* logits = reinterpret_cast<float*>(b + w.logits);
   int32_t* idx = reinterpret_cast<int32_t*>(b + w.idx);
   float* gate = reinterpret_cast<float*>(b + w.gate);
-  if (T <= MOE_DECODE_MAX_T && cfg->E <= 512) {
-    // one fused kernel: router, top-k, grouping, experts and combine
-    const GroupPtrs g = group_ptrs(*cfg, T, ws);
-    DecodeArgs d{};
-    d.route = true;
-    d.x = static_cast<const uint16_t*>(x);
-    d.T = T;
-    d.wr = w_router;
-    d.bias = logit_bias;
-    d.logits = logits;
-    d.idx = idx;
-    d.gate = gate;
-    d.slot_of = slot_of;
-    d.n_slots = n_slots;
-    d.g = &g;
-    d.pool = slot_pool;
-    d.stride = slot_stride;
-    d.shared = cfg->n_shared ? shared_expert : nullptr;
-    d.lay = layout_of(*cfg);
-    d.h = reinterpret_cast<float*>(b + w.h);
-    d.y = y;
-    d.logits_rep = reinterpret_cast<float*>(b + w.logits_rep);
-    const cudaError_t e = launch_decode_layer(ctx->c, *cfg, d, static_cast<cudaStream_t>(stream));
-    if (e == cudaErrorNotSupported) return MOE_EUNSUPPORTED;
-    return from_cuda(e);
-  }
+  if (T <= MOE_DECODE_MAX_T && cfg->E <= 512)  // one fused kernel: router, top-k, grouping, experts, combine
+    return run_stack(ctx, *cfg, 1, x, T, w_router, logit_bias, slot_of, n_slots, slot_pool, slot_stride,
+                     shared_expert, ws, y, stream);
   if ((st = moe_router_topk(ctx, cfg, x, w_router, logit_bias, T, logits, idx, gate, stream)) != MOE_OK)
     return st;
   moe_grouping g;

@@ -18,10 +18,6 @@ constexpr int kMaxE = 1024;           // experts per layer
 constexpr int kMaxK = 32;             // experts per token
 constexpr int kGroupChunk = 512;      // pairs per chunk in the multi-CTA grouping
 constexpr int kTileN = 128;           // tokens per tile of the prefill grouped GEMM
-// Copies of the small arrays every CTA of the decode kernel reads after a
-// grid barrier (logits, h): CTA b reads copy b % kRep, so each cache line has
-// ~148/kRep readers instead of all of them.
-constexpr int kRep = 8;
 
 // Device status word codes (word 0 holds the first error seen).
 constexpr int kDevBadExpert = 1;
@@ -32,10 +28,10 @@ struct Ctx {
   int device = 0;
   int num_sms = 0;
   int* d_status = nullptr;     // [4] ints: code, detail, spare, spare
-  unsigned long long* d_gbar = nullptr;  // grid-barrier arrival counter of the decode kernel
   unsigned long long timeout_ns = 200ull * 1000 * 1000;  // limit of every device-side wait
   unsigned long long* d_trace = nullptr;  // phase timestamps (MOE_TRACE), kTraceSlots per CTA
   void* static_scratch = nullptr;  // device address of the static scratch (first static call)
+  bool coop_pdl = false;           // a cooperative launch also takes programmatic serialization
 };
 constexpr int kTraceSlots = 32;
 constexpr int kTraceCtas = 1024;
@@ -51,13 +47,16 @@ namespace moe {
 
 // ---------------------------------------------------------------- workspace
 
+// Workspace of one call: the routing record (what moe_layer_routing views)
+// first, then the scratch of the path the call takes.
 struct WsLayout {
   size_t logits, idx, gate;
   size_t expert_count, expert_offset, pair_token, pair_j, pair_gate, pair_slot, pair_pos;
   size_t uniq_expert, uniq_slot, uniq_offset, n_uniq;
+  size_t rec_bytes;              // end of the routing record
   size_t chunk_hist, tile_offset;
-  size_t logits_rep;            // decode path: kRep copies of the [T, E] logits
-  size_t h, z, x16;
+  size_t exchange;               // decode path: the tagged-word exchange area
+  size_t h, z, x16;              // prefill path
   size_t tile_info;              // prefill: int4 per token tile
   size_t total;
   int n_pairs, n_rows, n_chunks, n_uniq_max;
@@ -162,28 +161,32 @@ cudaError_t launch_group(const Ctx& ctx, const moe_layer_cfg& c, const int32_t* 
                          const float* gate, int T, const int32_t* slot_of, int n_slots,
                          const GroupPtrs& g, cudaStream_t s);
 
-// decode_layer.cu
-struct DecodeArgs {
+// decode_stack.cu
+struct StackArgs {
   bool route;               // true: router + top-k + grouping run inside the kernel
-  const uint16_t* x;        // [T, d] bf16
-  int T;
-  const float* wr;          // route: [E, d]
-  const float* bias;        // route: [T, E] or null
-  float* logits;            // route: [T, E] (workspace)
-  int32_t* idx;             // route: [T, k]
-  float* gate;              // route: [T, k]
-  const int32_t* slot_of;   // route: [E]
+  const uint16_t* x;        // [T, d] bf16: layer 0's input
+  int T, L;                 // tokens, layers (L > 1 only with route)
+  const float* wr;          // route: [L, E, d]
+  const float* bias;        // route: [L, T, E] or null
+  const int32_t* slot_of;   // route: [L, E]
   int n_slots;
-  const GroupPtrs* g;       // grouping (written when route, read otherwise)
   const uint8_t* pool;
   size_t stride;
-  const uint8_t* shared;    // record or null
+  const uint8_t* shared;    // layer l's shared record at shared + l * stride, or null
   moe_expert_layout lay;
-  float* h;                 // fp32 [kRep][n_rows, f]
-  float* logits_rep;        // route: [kRep][T, E]
-  void* y;
+  void* y;                  // [L, T, d]
+  char* rec;                // route: layer l's routing record at rec + l * rec_bytes
+  size_t rec_bytes;
+  int ro[14];               // offsets in a record: logits, idx, gate, expert_count, expert_offset,
+                            // pair_token, pair_j, pair_gate, pair_slot, pair_pos, uniq_expert,
+                            // uniq_slot, uniq_offset, n_uniq
+  const GroupPtrs* g;       // not route: the given grouping
+  char* exchange;           // decode_exchange_bytes(cfg, T) bytes, 256-byte aligned
 };
-cudaError_t launch_decode_layer(const Ctx& ctx, const moe_layer_cfg& c, const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const StackArgs& a, cudaStream_t s);
+size_t decode_exchange_bytes(const moe_layer_cfg& c, int T);
+// Moves the decode kernel's tag counter past an interrupted launch's tags.
+cudaError_t decode_skip_tags(cudaStream_t s);
 bool decode_geometry_ok(int d, int f);
 
 // FFN arguments of the prefill path
@@ -212,7 +215,7 @@ cudaError_t launch_combine(const Ctx& ctx, const moe_layer_cfg& c, const int32_t
                            cudaStream_t s);
 
 // kernel attribute set-up, once per context
-cudaError_t decode_init(const Ctx& ctx);
+cudaError_t decode_init(Ctx& ctx);
 cudaError_t router_init(const Ctx& ctx);
 
 // router_tc.cu: prefill router logits on the tensor cores

@@ -96,6 +96,9 @@ _SIGS = {
     "moe_layer_forward": (_I, [_P, ctypes.POINTER(_Cfg), _P, _I, _P, _P, _P, _I, _P, _Z, _P, _P, _Z, _P,
                                _S]),
     "moe_layer_routing": (_I, [ctypes.POINTER(_Cfg), _I, _P, _Z, ctypes.POINTER(Routing)]),
+    "moe_stack_workspace_bytes": (_Z, [ctypes.POINTER(_Cfg), _I, _I]),
+    "moe_stack_forward": (_I, [_P, ctypes.POINTER(_Cfg), _I, _P, _I, _P, _P, _P, _I, _P, _Z, _P, _P, _Z, _P, _S]),
+    "moe_stack_routing": (_I, [ctypes.POINTER(_Cfg), _I, _I, _P, _Z, _I, ctypes.POINTER(Routing)]),
     "moe_layer_forward_static": (_I, [_P, ctypes.POINTER(_Cfg), _P, _I, _P, _P, _P, _I, _P, _Z, _P, _P, _S]),
 }
 
@@ -180,6 +183,19 @@ class Context:
                                           0 if ws is None else ws.numel() * ws.element_size(), _ptr(y),
                                           _stream(stream))
 
+    def stack_forward_status(self, cfg, L, x, T, w_router, bias, slot_of, n_slots, pool, stride, shared, ws, y,
+                             stream=None):
+        return self.lib.moe_stack_forward(self.h, ctypes.byref(cfg.c()), L, _ptr(x), T, _ptr(w_router), _ptr(bias),
+                                          _ptr(slot_of), n_slots, _ptr(pool), stride, _ptr(shared), _ptr(ws),
+                                          0 if ws is None else ws.numel() * ws.element_size(), _ptr(y),
+                                          _stream(stream))
+
+    def stack_forward(self, cfg, L, x, T, w_router, bias, slot_of, n_slots, pool, stride, shared, ws, y,
+                      stream=None):
+        """moe_stack_forward: L chained decode layers in one launch (layer l + 1 reads y[l])."""
+        _check(self.stack_forward_status(cfg, L, x, T, w_router, bias, slot_of, n_slots, pool, stride, shared, ws,
+                                         y, stream), "moe_stack_forward")
+
     def layer_forward_static_status(self, cfg, x, T, w_router, bias, slot_of, n_slots, pool, stride, shared, y,
                                     stream=None):
         """moe_layer_forward with the library's static scratch (no workspace argument)."""
@@ -222,15 +238,20 @@ class Context:
         """moe_layer_forward with every argument but x and y marshalled once (for launch loops)."""
         return PreparedLayer(self, cfg, T, w_router, bias, slot_of, n_slots, pool, stride, shared, ws, stream)
 
-    def layer_routing(self, cfg, T, ws) -> dict:
-        """The routing a whole-step call with workspace `ws` computed (moe_layer_routing), as torch views
-        into ws: logits [T,E], idx [T,k], gate [T,k] and the grouping arrays. Read them after the call
-        has completed on its stream."""
+    def layer_routing(self, cfg, T, ws, stack_layers=None, layer=0) -> dict:
+        """The routing a whole-step call with workspace `ws` computed (moe_layer_routing; with
+        stack_layers=L, layer `layer` of a moe_stack_forward workspace), as torch views into ws:
+        logits [T,E], idx [T,k], gate [T,k] and the grouping arrays. Read them after the call has
+        completed on its stream."""
         import torch
         r = Routing()
         nbytes = ws.numel() * ws.element_size()
-        _check(self.lib.moe_layer_routing(ctypes.byref(cfg.c()), T, _ptr(ws), nbytes, ctypes.byref(r)),
-               "moe_layer_routing")
+        if stack_layers is None:
+            _check(self.lib.moe_layer_routing(ctypes.byref(cfg.c()), T, _ptr(ws), nbytes, ctypes.byref(r)),
+                   "moe_layer_routing")
+        else:
+            _check(self.lib.moe_stack_routing(ctypes.byref(cfg.c()), stack_layers, T, _ptr(ws), nbytes, layer,
+                                              ctypes.byref(r)), "moe_stack_routing")
         raw = ws.view(torch.uint8).view(-1)
         base = ws.data_ptr()
 
@@ -298,6 +319,14 @@ def workspace(cfg: LayerCfg, T: int, device="cuda"):
     n = workspace_bytes(cfg, T)
     if n == 0:
         raise MoeError(EINVAL, "moe_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def stack_workspace(cfg: LayerCfg, L: int, T: int, device="cuda"):
+    import torch
+    n = int(load_library().moe_stack_workspace_bytes(ctypes.byref(cfg.c()), L, T))
+    if n == 0:
+        raise MoeError(EINVAL, "moe_stack_workspace_bytes")
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 

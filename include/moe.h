@@ -32,8 +32,13 @@
  *     errors detected by a kernel are recorded in the context's device status
  *     word and returned by moe_check_device_status().
  *   - No exception or abort crosses the ABI. A context may be used by one host
- *     thread at a time; it belongs to the device named at its creation, and
- *     every call made with it launches there.
+ *     thread and one stream at a time; it belongs to the device named at its
+ *     creation, and every call made with it launches there (the caller's
+ *     current device is restored before the call returns).
+ *   - The decode path (T <= MOE_DECODE_MAX_T) is one cooperative launch of a
+ *     CTA per SM: it starts once every SM is free, and decode calls on one
+ *     device must not overlap in time (one stream, or calls ordered with
+ *     events), since they share a per-device tag counter.
  *
  * Expert record (one routed or shared expert, `moe_expert_layout`):
  *   gu_codes  [2f rows, d cols] packed codes; row 2c is gate channel c,
@@ -238,6 +243,41 @@ typedef struct {
 } moe_routing;
 MOE_API moe_status moe_layer_routing(const moe_layer_cfg* cfg, int T, void* ws, size_t ws_bytes,
                                      moe_routing* out);
+
+/* ---- the decode stack ----------------------------------------------------- */
+
+/* L consecutive layers of the decode path in one launch: layer 0 reads x,
+ * layer l + 1 reads layer l's output y[l] (a model's MoE layers in a row, with
+ * the per-layer join of the pages' engine between them: vramglass.com,
+ * section その2). Per layer the same step as moe_layer_forward (router,
+ * top-k, grouping, experts, combine; with cfg->residual, y[l] = x_l + moe(x_l)).
+ * While layer l runs, layer l + 1's router rows and shared expert, which do
+ * not depend on x, are already being fetched.
+ *   - T: 1..MOE_DECODE_MAX_T tokens; cfg->E <= 512; L >= 1.
+ *   - w_router: [L, E, d] fp32; logit_bias: NULL or [L, T, E] fp32;
+ *     slot_of: [L, E] int32 (the stack's slot table, one row per layer);
+ *     slot_pool / slot_stride: the pool as for moe_layer_forward;
+ *     shared_experts: layer l's shared expert record at
+ *     shared_experts + l * slot_stride (NULL when cfg->n_shared == 0).
+ *   - y: [L, T, d]; bf16 (cfg->out_fp32 must be 0 when L > 1, since the
+ *     next layer reads it as its bf16 input).
+ *   - ws: moe_stack_workspace_bytes(cfg, L, T) bytes, 256-byte aligned.
+ *     After the call has completed, layer l's routing is readable through
+ *     moe_stack_routing. Nothing in it needs to start at zero.
+ * The kernel is a cooperative launch of one CTA per SM whose CTAs exchange
+ * data while they run: the launch waits until every SM is free, and calls on
+ * one device must not overlap in time (issue them on one stream, or order
+ * them with events). Same status and error conventions as every call. */
+MOE_API size_t moe_stack_workspace_bytes(const moe_layer_cfg* cfg, int L, int T);
+MOE_API moe_status moe_stack_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, int L, const void* x, int T,
+                                     const float* w_router, const float* logit_bias, const int32_t* slot_of,
+                                     int n_slots, const uint8_t* slot_pool, size_t slot_stride,
+                                     const uint8_t* shared_experts, void* ws, size_t ws_bytes, void* y,
+                                     moe_stream stream);
+/* Views of layer `layer`'s routing inside a stack workspace (as
+ * moe_layer_routing). */
+MOE_API moe_status moe_stack_routing(const moe_layer_cfg* cfg, int L, int T, void* ws, size_t ws_bytes,
+                                     int layer, moe_routing* out);
 
 /* moe_layer_forward without a workspace argument: the step's scratch is a
  * static device array of MOE_STATIC_SCRATCH_BYTES inside the library image,
