@@ -2,16 +2,24 @@
 
 Default workload (decode): the full-size layer (d=2048, f=768, 512 routed
 experts, top-10 plus 1 shared, 2-bit block-32 fp16-scale weights, Zipf(1.1)
-routing) at T=1, run for 48 layers in a row, every layer with its own seeded
-input tokens, router, shared expert and 512 experts in a 24,576-slot pool
-(36.2 GB) behind a slot table whose 4,500 most popular experts sit in slots
-0..4,499. (Chaining x_{l+1} = x_l + y_l through random-weight layers with no
-normalisation diverges within three layers, after which the router no longer
-follows the seeded routing; each layer therefore reads its own seeded x_l.)
-One step = one pass of all 48 layers; the 48 layers' weights (~1 GB touched
-per step) do not fit in the 126 MB L2, so every layer reads its weights from
-HBM.
+routing) at T=1, run for 48 layers in a row by moe_stack_forward (one launch
+per step): layer l + 1 reads layer l's output (a residual stream
+y_l = x_l + moe(x_l)), every layer has its own router, shared expert, Zipf
+popularity and 512 experts in a 24,576-slot pool (36.2 GB) behind a slot
+table whose 4,500 most popular experts sit in slots 0..4,499. The seeded
+bias (+20 on each token's Zipf-drawn experts, against router logits of
+about +-2) keeps the routing on the seeded draw along the chain. One step =
+one pass of all 48 layers; the 48 layers' weights (~1 GB touched per step)
+do not fit in the 126 MB L2, so every layer reads its weights from HBM.
 
+The default line also carries, under config.extras, the other
+configurations: the same layers as 48 single-layer launches, the 48-layer
+stack at the verify width T=4 over 256 consecutive steps with 70 % of each
+token position's experts kept from the step before, the 3-bit stack at
+T = 1..4 (64 correlated steps each) and the T=8192 prefill chunk (2- and
+3-bit).
+
+--workload stack: that T=4 (--tokens 4) correlated stack as the headline.
 --workload prefill: one full-size layer at T=8192 (81,920 token-expert pairs,
 Zipf-skewed over 512 experts), the prefill chunk of the pages.
 
@@ -37,13 +45,11 @@ METRIC = "MoE decode tok/s & expert-weight GB/s vs HBM peak (2-bit, top-10 of 51
 LAYERS = 48
 HOT = 4500
 SEED = 0
-KERNELS_PER_LAYER_DECODE = 1  # one fused decode-layer kernel
-# dram__bytes_read.sum + dram__bytes_write.sum of one fused decode-layer launch
-# (T=1, 2-bit) from an ncu capture of the current kernel, or None when the
-# kernel has changed since the last capture (the last one, of the revision
-# before the routing step moved ahead of the shared expert's stages, read
-# 20,537,600 B and wrote 256 B per launch)
-DECODE_LAYER_DRAM_BYTES = None
+# dram__bytes_read.sum + dram__bytes_write.sum of one decode stack launch from
+# an ncu capture of the current kernel, keyed by (T, bits, layers, correlated
+# workload), scaled to the stack's layers when the capture ran fewer; absent
+# until a capture of the current kernel exists
+DECODE_STACK_DRAM_BYTES = {}
 
 
 def peaks():
@@ -144,122 +150,121 @@ def allreduce_max(v: float, world: int) -> float:
 
 # ------------------------------------------------------------------ workload
 
-class DecodeStack:
-    """48 layers of the full-size decode layer, T tokens, pools on the device."""
+def cpu_info():
+    """Host cores and CPU model (the oracle baseline runs there)."""
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "model": model}
 
-    def __init__(self, T=1, bits=2, layers=LAYERS, seed=SEED):
+
+def make_pool(bits, layers=LAYERS, seed=SEED):
+    """The stack's device tensors: a layers*512-slot pool of full-size records
+    (uniform random codes, fp16 U(0.005, 0.02) scales), one shared expert per
+    layer, the routers W_r [L, 512, 2048] ~ N(0, 0.02^2) and the hot-slot table
+    (the 4,500 most popular experts of the 48 layers in slots 0..4,499)."""
+    import torch
+    from bit_expert_ffn_router_b200 import moe as M
+    from bit_expert_ffn_router_b200 import synth
+    cfg = M.FULL.replace(bits=bits, out_fp32=0, residual=1)
+    lay = M.expert_layout(cfg)
+    stride = lay["bytes"]
+    n_slots = layers * cfg.E
+    dev = "cuda"
+    pool = torch.empty(n_slots, stride, dtype=torch.uint8, device=dev)
+    synth.fill_random_bytes_(pool, seed + 11)
+    shared = torch.empty(layers, stride, dtype=torch.uint8, device=dev)
+    synth.fill_random_bytes_(shared, seed + 12)
+    for name, seedoff in (("gu_scales", 13), ("dn_scales", 14)):
+        lo = lay[name]
+        n = (2 * cfg.f * (cfg.d // 32) if name == "gu_scales" else cfg.d * (cfg.f // 32)) * 2
+        for s0 in range(0, n_slots, 2048):
+            s1 = min(s0 + 2048, n_slots)
+            synth.fill_scales_(pool[s0:s1, lo:lo + n], seed + seedoff * 100003 + s0)
+        synth.fill_scales_(shared[:, lo:lo + n], seed + seedoff)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed + 15)
+    wr = torch.randn(layers, cfg.E, cfg.d, generator=g, device=dev) * 0.02
+    hot = HOT * layers // LAYERS  # the hot share of the pool stays 4,500 / 24,576
+    slot_of = torch.from_numpy(synth.hot_slot_table(layers, cfg.E, hot, seed)).to(dev)
+    return {"cfg": cfg, "bits": bits, "layers": layers, "lay": lay, "stride": stride, "n_slots": n_slots,
+            "pool": pool, "shared": shared, "wr": wr, "slot_of": slot_of, "hot": hot}
+
+
+class DecodeStack:
+    """L chained full-size decode layers run by moe_stack_forward (one launch
+    per step; layer l + 1 reads layer l's output, a residual stream y_l =
+    x_l + moe(x_l)). Routing per layer follows a Zipf(1.1) popularity: one
+    fixed draw (steps=1), or `steps` consecutive decode steps in which every
+    token position keeps `keep` of its previous step's experts."""
+
+    def __init__(self, pool, T=1, steps=1, keep=None, seed=SEED):
         import torch
         from bit_expert_ffn_router_b200 import moe as M
         from bit_expert_ffn_router_b200 import synth
-        self.M, self.torch = M, torch
-        self.T, self.L = T, layers
-        self.cfg = M.FULL.replace(bits=bits, out_fp32=0)
-        cfg = self.cfg
-        self.lay = M.expert_layout(cfg)
-        self.stride = self.lay["bytes"]
-        self.n_slots = layers * cfg.E
-        dev = "cuda"
-        # pool: uniform random code bytes, then fp16 U(0.005, 0.02) scales in the scale sections
-        self.pool = torch.empty(self.n_slots, self.stride, dtype=torch.uint8, device=dev)
-        synth.fill_random_bytes_(self.pool, seed + 11)
-        self.shared = torch.empty(layers, self.stride, dtype=torch.uint8, device=dev)
-        synth.fill_random_bytes_(self.shared, seed + 12)
-        for name, seedoff in (("gu_scales", 13), ("dn_scales", 14)):
-            lo = self.lay[name]
-            n = (2 * cfg.f * (cfg.d // 32) if name == "gu_scales" else cfg.d * (cfg.f // 32)) * 2
-            for s0 in range(0, self.n_slots, 2048):
-                s1 = min(s0 + 2048, self.n_slots)
-                synth.fill_scales_(self.pool[s0:s1, lo:lo + n], seed + seedoff * 100003 + s0)
-            synth.fill_scales_(self.shared[:, lo:lo + n], seed + seedoff)
-        g = torch.Generator(device=dev)
-        g.manual_seed(seed + 15)
-        self.wr = torch.randn(layers, cfg.E, cfg.d, generator=g, device=dev) * 0.02
-        hot = HOT * layers // LAYERS  # the hot share of the pool stays 4,500 / 24,576
-        self.slot_of = torch.from_numpy(synth.hot_slot_table(layers, cfg.E, hot, seed)).to(dev)
-        bias = np.stack([synth.bias_from_sets(synth.zipf_sets(T, cfg.E, cfg.k, seed + 1000 * l), cfg.E)
-                         for l in range(layers)])
-        self.bias = torch.from_numpy(bias).to(dev)
-        self.x_host = np.stack([synth.activations(T, cfg.d, seed + 1000 * l + 16) for l in range(layers)])
-        self.x_in = torch.from_numpy(self.x_host.view(np.int16)).to(dev).view(torch.bfloat16)  # [L, T, d]
-        self.y_out = torch.empty(layers, T, cfg.d, dtype=torch.bfloat16, device=dev)
-        self.ws = M.workspace(cfg, T)
+        self.M, self.torch, self.p = M, torch, pool
+        self.cfg = cfg = pool["cfg"]
+        self.T, self.L = T, pool["layers"]
+        L, E, k = self.L, cfg.E, cfg.k
+        if keep is None:
+            sets = np.stack([synth.zipf_sets(T, E, k, seed + 1000 * l) for l in range(L)])[None]  # [1, L, T, k]
+        else:
+            sets = np.stack([synth.correlated_sets(steps, T, E, k, keep, seed + 1000 * l) for l in range(L)],
+                            axis=1)  # [S, L, T, k]
+        self.sets = sets
+        self.S = sets.shape[0]
+        bias = np.zeros((self.S, L, T, E), dtype=np.float32)
+        np.put_along_axis(bias, sets.astype(np.int64), np.float32(synth.BIAS), axis=3)
+        self.bias = torch.from_numpy(bias).to("cuda")
+        self.uniq = np.array([[len(np.unique(sets[s, l])) for l in range(L)] for s in range(self.S)])
+        self.x_host = synth.activations(T, cfg.d, seed + 16)
+        self.x0 = torch.from_numpy(self.x_host.view(np.int16)).to("cuda").view(torch.bfloat16)
+        self.y = torch.empty(L, T, cfg.d, dtype=torch.bfloat16, device="cuda")
+        self.ws = M.stack_workspace(cfg, L, T)
         self.ctx = M.Context(torch.cuda.current_device())
-        self.graph = None
-        # unique experts per layer (for the byte count)
-        idx = [np.argsort(-bias[l], axis=1)[:, :cfg.k] for l in range(layers)]
-        self.uniq = [len(np.unique(i)) for i in idx]
-        self.expert_bytes_step = sum((u + cfg.n_shared) * self.stride for u in self.uniq)
-        self.router_bytes_step = layers * cfg.E * cfg.d * 4
+        self.call = self.ctx.prepare_stack_forward(cfg, L, T, pool["wr"], pool["slot_of"], pool["n_slots"],
+                                                   pool["pool"], pool["stride"], pool["shared"], self.ws)
 
-    def layer(self, l, x, y):
+    def step(self, s=0):
+        self.call(self.x0, self.bias[s % self.S], self.y)
+        return self.y
+
+    def expert_bytes(self, s):
+        return int((self.uniq[s % self.S] + self.cfg.n_shared).sum()) * self.p["stride"]
+
+    def step_bytes(self, s):
+        """Algorithmic bytes of one step: the records of the selected and
+        shared experts, the routers and every layer's x and y."""
         cfg = self.cfg
-        self.ctx.layer_forward(cfg, x, self.T, self.wr[l], self.bias[l], self.slot_of[l * cfg.E:(l + 1) * cfg.E],
-                               self.n_slots, self.pool, self.stride, self.shared[l], self.ws, y)
+        return self.expert_bytes(s) + self.L * cfg.E * cfg.d * 4 + self.L * 2 * self.T * cfg.d * 2
 
-    def step_eager(self):
-        for l in range(self.L):
-            self.layer(l, self.x_in[l], self.y_out[l])
-        return self.y_out
 
-    def prepare(self):
-        """One prepared moe_layer_forward per layer (arguments marshalled once), as
-        a host program driving the C ABI would hold them."""
-        cfg = self.cfg
-        self.prepared = [
-            (self.ctx.prepare_layer_forward(cfg, self.T, self.wr[l], self.bias[l],
-                                            self.slot_of[l * cfg.E:(l + 1) * cfg.E], self.n_slots, self.pool,
-                                            self.stride, self.shared[l], self.ws),
-             self.x_in[l], self.y_out[l])
-            for l in range(self.L)]
-
-    def step_prepared(self):
-        for call, x, y in self.prepared:
-            call(x, y)
-        return self.y_out
-
-    def capture(self):
-        torch = self.torch
-        s = torch.cuda.Stream()
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
-            self.step_eager()  # warm (attributes, lazy init) outside capture
-        torch.cuda.current_stream().wait_stream(s)
+def time_steps(st, steps, warmup, world, local, first=0):
+    """Device time (ms, max over ranks) of `steps` consecutive stack steps after
+    `warmup` untimed ones, with the clocks sampled during the timed region."""
+    import torch
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        st.step(first + i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(steps):
+            st.step(first + warmup + i)
+        e1.record(stream)
         torch.cuda.synchronize()
-        self.graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.graph):
-            self.out = self.step_eager()
-        torch.cuda.synchronize()
-
-    def time_expert_ffn(self, reps=3):
-        """CUDA-event time of the decode expert kernels (gate/up + down/combine) per layer."""
-        torch, M, cfg = self.torch, self.M, self.cfg
-        st = torch.cuda.current_stream()
-        logits = torch.empty(self.T, cfg.E, device="cuda")
-        idx = torch.empty(self.T, cfg.k, dtype=torch.int32, device="cuda")
-        gate = torch.empty(self.T, cfg.k, device="cuda")
-        groups = []
-        wss = []
-        for l in range(self.L):
-            ws = M.workspace(cfg, self.T)
-            self.ctx.router_topk(cfg, self.x_in[l], self.wr[l], self.bias[l], self.T, logits, idx, gate)
-            groups.append(self.ctx.group_tokens(cfg, idx, gate, self.T, self.slot_of[l * cfg.E:(l + 1) * cfg.E],
-                                                self.n_slots, ws))
-            wss.append(ws)
-        y = torch.empty(self.T, cfg.d, dtype=torch.bfloat16, device="cuda")
-        evs = []
-        for r in range(reps + 1):
-            for l in range(self.L):
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(st)
-                self.ctx.expert_ffn(cfg, self.x_in[l], groups[l], self.pool, self.stride, self.shared[l], wss[l], None,
-                                    y)
-                b.record(st)
-                if r > 0:
-                    evs.append((a, b, l))
-        torch.cuda.synchronize()
-        ms = [a.elapsed_time(b) for a, b, _ in evs]
-        bytes_ = [(self.uniq[l] + cfg.n_shared) * self.stride for _, _, l in evs]
-        return float(np.mean(ms)), float(np.mean(bytes_))
+    barrier(world)
+    st.ctx.check_device_status() == 0 or sys.exit("device error in the timed steps")
+    return allreduce_max(e0.elapsed_time(e1), world), clk.summary()
 
 
 KERNELS_PER_LAYER_PREFILL = 9  # router GEMM, top-k, 3 grouping, x gather, 2 grouped GEMMs, combine
@@ -438,118 +443,152 @@ def run_prefill(args):
         dist.destroy_process_group()
 
 
+def workload_name(T, bits, layers=LAYERS, correlated=False):
+    what = (f"48-layer stack at the verify width T={T}, 256 consecutive decode steps with routing temporally "
+            f"correlated (each token position keeps 7 of its 10 experts from the step before)"
+            if correlated else f"decode layer, T={T}")
+    return (f"{what}: d=2048 f=768 E=512 top-10 + 1 shared, {bits}-bit block-32 fp16-scale, Zipf(1.1) routing, "
+            f"{layers} chained layers per step (layer l+1 reads layer l's output), {layers * 512}-slot pool with "
+            f"{HOT * layers // LAYERS} hot slots")
+
+
+def stack_record(st, ms_total, steps, first, hbm, world):
+    """Compact numbers of a timed run of stack steps [first, first + steps)."""
+    idx = [(first + i) % st.S for i in range(steps)]
+    ms_step = ms_total / steps
+    ebytes = float(np.mean([st.expert_bytes(s) for s in idx]))
+    sbytes = float(np.mean([st.step_bytes(s) for s in idx]))
+    u = st.uniq[idx]
+    return {
+        "tok_s": round(st.T * steps * world / (ms_total / 1e3), 1),
+        "ms_per_step": round(ms_step, 4), "layer_us": round(ms_step * 1e3 / st.L, 3),
+        "uniq_experts_per_layer": {"mean": round(float(u.mean()), 2), "min": int(u.min()), "max": int(u.max())},
+        "expert_gbs": round(ebytes / (ms_step / 1e3) / 1e9, 1),
+        "expert_frac_of_hbm": round(ebytes / (ms_step / 1e3) / 1e9 / hbm, 4),
+        "step_gbs": round(sbytes / (ms_step / 1e3) / 1e9, 1),
+        "step_frac_of_hbm": round(sbytes / (ms_step / 1e3) / 1e9 / hbm, 4),
+    }
+
+
+def layer_call_record(st, steps, world):
+    """The same stack as L separate moe_layer_forward launches (one CUDA graph
+    per step): the single-layer entry point's speed."""
+    import torch
+    M, cfg, p = st.M, st.cfg, st.p
+    ws = M.workspace(cfg, st.T)
+    bias = st.bias[0]
+    calls = [st.ctx.prepare_layer_forward(cfg, st.T, p["wr"][l], bias[l], p["slot_of"][l * cfg.E:(l + 1) * cfg.E],
+                                          p["n_slots"], p["pool"], p["stride"], p["shared"][l], ws)
+             for l in range(st.L)]
+
+    def run():
+        x = st.x0
+        for l, c in enumerate(calls):
+            c(x, st.y[l])
+            x = st.y[l]
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        run()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = allreduce_max(e0.elapsed_time(e1), world) / steps
+    return {"tok_s": round(st.T * world / (ms / 1e3), 1), "layer_us": round(ms * 1e3 / st.L, 3),
+            "how": f"{st.L} moe_layer_forward launches per step in one CUDA graph"}
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_setup()
     hbm, tf, tf_s, peak_kind = peaks()
-    st = DecodeStack(T=args.tokens, bits=args.bits, layers=args.layers)
-    st.capture()
-    stream = torch.cuda.current_stream()
-    for _ in range(args.warmup):
-        st.graph.replay()
-    torch.cuda.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            st.graph.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    ms = e0.elapsed_time(e1)
-    ms_max = allreduce_max(ms, world)
-    ms_step = ms_max / args.steps
-    tokens = st.T * args.steps * world
-    value = tokens / (ms_max / 1e3 * LAYERS / st.L)  # per 48-layer stack (st.L < 48 only when profiling)
+    T = args.tokens
+    stack_wl = args.workload == "stack"
+    pool = make_pool(args.bits, layers=args.layers)
+    if stack_wl:  # 256 consecutive decode steps, 7 of each position's 10 experts kept from the step before
+        st = DecodeStack(pool, T=T, steps=256, keep=7)
+    else:
+        st = DecodeStack(pool, T=T)
+    steps = args.steps
+    ms_max, clocks = time_steps(st, steps, args.warmup, world, local)
+    ms_step = ms_max / steps
+    scale = LAYERS / st.L  # per 48-layer stack (st.L < 48 only when profiling)
+    value = st.T * steps * world / (ms_max / 1e3 * scale)
+    rec = stack_record(st, ms_max, steps, args.warmup, hbm, world)
+    # roofline of the one kernel of the step: the stack launch's algorithmic
+    # bytes over its average duration (CUDA events on its stream)
+    idx = [(args.warmup + i) % st.S for i in range(steps)]
+    launch_bytes = float(np.mean([st.step_bytes(s) for s in idx]))
+    achieved = launch_bytes / (ms_step / 1e3) / 1e9
 
-    # The dominant (and only) kernel of the timed step is the fused decode-layer
-    # kernel, one launch per layer: its average launch time over the timed
-    # region and its algorithmic bytes per launch (the selected experts'
-    # records, the router matrix, x and y).
-    layer_launch_s = ms_step / 1e3 / st.L
-    layer_bytes = (st.expert_bytes_step + st.router_bytes_step) / st.L + 2 * st.T * st.cfg.d * 2
-    achieved = layer_bytes / layer_launch_s / 1e9
-    # side measurement: the expert FFN alone (grouping given), cold weights
-    ffn_ms, ffn_bytes = st.time_expert_ffn()
-
-    # end to end through the public API: pinned host x in, 48 eager layer calls
-    # (each layer's arguments marshalled once, before the timed region), host y out
+    # end to end through the public API: pinned host x -> moe_stack_forward ->
+    # pinned host y of the last layer, every step inside the timed region
     xh = torch.from_numpy(st.x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
-    yh = torch.empty_like(xh).pin_memory()
-    how = "48 eager moe_layer_forward calls (arguments marshalled once per layer)"
-    try:
-        st.prepare()
-        step = st.step_prepared
-        st.x_in.copy_(xh, non_blocking=True)
-        step()
-        torch.cuda.synchronize()
-    except st.M.MoeError:
-        raise
-    except Exception as exc:  # the binding's prepared form failed: time the plain calls instead
-        print(f"prepared calls unavailable ({exc!r}); timing the plain binding calls", file=sys.stderr)
-        step, how = st.step_eager, "48 eager moe_layer_forward calls"
-    for _ in range(2):
-        st.x_in.copy_(xh, non_blocking=True)
-        out = step()
-        yh.copy_(out, non_blocking=True)
+    yh = torch.empty(st.T, st.cfg.d, dtype=torch.bfloat16).pin_memory()
+    stream = torch.cuda.current_stream()
+    for i in range(3):
+        st.x0.copy_(xh, non_blocking=True)
+        yh.copy_(st.step(i)[st.L - 1], non_blocking=True)
     torch.cuda.synchronize()
     barrier(world)
+    n_e2e = max(3, steps // 2)
     e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2.record(stream)
-    n_e2e = max(3, args.steps // 4)
-    for _ in range(n_e2e):
-        st.x_in.copy_(xh, non_blocking=True)
-        out = step()
-        yh.copy_(out, non_blocking=True)
+    for i in range(n_e2e):
+        st.x0.copy_(xh, non_blocking=True)
+        yh.copy_(st.step(i)[st.L - 1], non_blocking=True)
     e3.record(stream)
     torch.cuda.synchronize()
     e2e_ms = allreduce_max(e2.elapsed_time(e3), world)
-    e2e_value = st.T * n_e2e * world / (e2e_ms / 1e3 * LAYERS / st.L)
+    e2e_value = st.T * n_e2e * world / (e2e_ms / 1e3 * scale)
 
-    layer_us = ms_step * 1e3 / st.L
-    expert_gbs_layer = st.expert_bytes_step / (ms_step / 1e3) / 1e9
     res = {
         "metric": METRIC,
         "value": round(value, 2),
         "unit": "tokens/s (48-layer MoE stack)",
         "n_gpus": world,
-        "steps": args.steps,
+        "steps": steps,
         "warmup": args.warmup,
         "ms_per_step": round(ms_step, 5),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "u2 codes x bf16 act, f32 accumulate",
+        "dtype": f"u{args.bits} codes x int16 block-requantised activations (dp2a), f32 block sums",
         "data": "synthetic (seeded; random-init weights of the stated shapes)",
         "config": {
-            "workload": f"decode layer d=2048 f=768 E=512 top-10 + 1 shared, T={st.T}, "
-                        f"{args.bits}-bit block-32 fp16-scale, Zipf(1.1) routing; {st.L} distinct layers per step",
+            "workload": workload_name(st.T, args.bits, st.L, stack_wl),
             "global_batch": st.T * world, "seq_len": 1, "parallelism": f"replicas x{world}",
-            "l2": "inputs larger than L2 (48 layers, ~1 GB touched per step)",
-            "layer_us": round(layer_us, 3),
-            "layer_tok_s": round(1e6 / layer_us * st.T, 1),
-            "expert_gbs_in_stack": round(expert_gbs_layer, 1),
-            "expert_bytes_per_step": st.expert_bytes_step,
-            "router_bytes_per_step": st.router_bytes_step,
-            "uniq_experts_per_layer": round(float(np.mean(st.uniq)), 2),
+            "l2": f"inputs larger than L2 ({st.L} layers, ~{launch_bytes / 1e9:.2f} GB touched per step)",
+            **rec,
         },
         "roofline": {
-            "kernel": "fused decode layer kernel (router, top-k, grouping, experts, combine), one launch per layer",
+            "kernel": "decode stack kernel (router, top-k, grouping, experts, combine of all layers), "
+                      "one launch per step",
             "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
             "frac": round(achieved / hbm, 4), "peak_source": f"{peak_kind} copy bandwidth",
-            "traffic": DECODE_LAYER_DRAM_BYTES if st.T == 1 and args.bits == 2 else None,
-            "avg_launch_us": round(layer_launch_s * 1e6, 3), "bytes_per_launch": round(layer_bytes),
-            "expert_ffn_only": {"avg_launch_us": round(ffn_ms * 1e3, 3), "expert_bytes": ffn_bytes,
-                                "gbs": round(ffn_bytes / (ffn_ms / 1e3) / 1e9, 1)},
+            "traffic": DECODE_STACK_DRAM_BYTES.get((st.T, args.bits, st.L, stack_wl)),
+            "avg_launch_us": round(ms_step * 1e3, 3), "bytes_per_launch": round(launch_bytes),
         },
         "e2e": {"value": round(e2e_value, 2), "unit": "tokens/s (48-layer MoE stack)",
-                "h2d_bytes_per_step": st.L * st.T * st.cfg.d * 2, "d2h_bytes_per_step": st.L * st.T * st.cfg.d * 2,
-                "how": f"pinned host x (48 layers' tokens) -> {how} -> pinned host y, CUDA events"},
-        "gpu_launches": KERNELS_PER_LAYER_DECODE * st.L * args.steps,
-        "clocks": clk.summary(),
+                "h2d_bytes_per_step": st.T * st.cfg.d * 2, "d2h_bytes_per_step": st.T * st.cfg.d * 2,
+                "how": "pinned host x -> moe_stack_forward (C ABI) -> pinned host y of the last layer, CUDA events"},
+        "gpu_launches": steps,
+        "clocks": clocks,
     }
+    if not args.no_extras and not stack_wl and st.L == LAYERS:
+        res["config"]["extras"] = run_extras(args, pool, st, world, local, hbm, tf)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(st, min(args.cpu_layers, st.L))
     if rank == 0:
@@ -559,40 +598,107 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_extras(args, pool2, st1, world, local, hbm, tf):
+    """The other configurations, as compact sub-records of the headline line:
+    the same layers as 48 single-layer launches; the 48-layer stack at T=4
+    over 256 correlated steps; the 3-bit stack at T = 1..4; the T=8192 prefill
+    chunk (2- and 3-bit)."""
+    import torch
+    out = {}
+    out["layer_calls_t1"] = layer_call_record(st1, 20, world)
+    st4 = DecodeStack(pool2, T=4, steps=256, keep=7)
+    ms, clk = time_steps(st4, 256, 3, world, local)
+    out["stack_t4_correlated_q2"] = {**stack_record(st4, ms, 256, 3, hbm, world), "steps": 256, "clocks": clk}
+    del st4, st1
+    torch.cuda.empty_cache()
+    for k in ("pool", "shared", "wr"):
+        pool2[k] = None
+    torch.cuda.empty_cache()
+    pool3 = make_pool(3)
+    q3 = {}
+    for T in (1, 2, 3, 4):
+        st3 = DecodeStack(pool3, T=T, steps=64, keep=7)
+        ms, _ = time_steps(st3, 64, 3, world, local)
+        q3[f"T{T}"] = stack_record(st3, ms, 64, 3, hbm, world)
+        del st3
+    out["stack_q3_correlated"] = q3
+    del pool3
+    torch.cuda.empty_cache()
+    for bits in (2, 3):
+        pl = PrefillLayer(T=8192, bits=bits)
+        pl.capture()
+        for _ in range(3):
+            pl.graph.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(10):
+            pl.graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = allreduce_max(e0.elapsed_time(e1), world) / 10
+        parts = pl.time_parts(reps=3)
+        ffn = parts["expert_ffn"]
+        ach = pl.flops / (ffn / 1e3) / 1e12
+        out[f"prefill_t8192_q{bits}"] = {
+            "tok_s_per_layer": round(pl.T * world / (ms / 1e3), 1), "ms_per_layer": round(ms, 4),
+            "parts_ms": {k: round(v, 4) for k, v in parts.items()},
+            "expert_ffn_tflops": round(ach, 1), "expert_ffn_frac_of_bf16_peak": round(ach / tf, 4),
+            "useful_gflop": round(pl.flops / 1e9, 1)}
+        del pl
+        torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------------ CPU oracle baseline
 
-def oracle_layer_inputs(st, l):
-    """Host copies of layer l's inputs (router, bias, the records it selects)."""
-    from oracle import moe_oracle as O
-    cfg = st.cfg
-    wr = st.wr[l].cpu().numpy()
-    bias = st.bias[l].cpu().numpy()
-    sel = np.unique(np.argsort(-bias, axis=1)[:, :cfg.k])
-    slot_of = st.slot_of[l * cfg.E:(l + 1) * cfg.E].cpu().numpy()
-    recs = {int(e): st.pool[int(slot_of[e])].cpu().numpy() for e in sel}
-    shared = st.shared[l].cpu().numpy()
-    return wr, bias, recs, shared
+def oracle_stack_inputs(st, n_layers):
+    """Host copies of the first n_layers layers' inputs (router, bias, the records they select)."""
+    cfg, p = st.cfg, st.p
+    out = []
+    for l in range(n_layers):
+        wr = p["wr"][l].cpu().numpy()
+        bias = st.bias[0, l].cpu().numpy()
+        slot_of = p["slot_of"][l * cfg.E:(l + 1) * cfg.E].cpu().numpy()
+        sel = np.unique(st.sets[0, l])
+        recs = {int(e): p["pool"][int(slot_of[e])].cpu().numpy() for e in sel}
+        out.append((wr, bias, recs, p["shared"][l].cpu().numpy()))
+    return out
 
 
 def cpu_baseline(st, n_layers):
-    """The fp64 oracle, as it stands, on a sample of the stack's layers (T tokens each)."""
+    """The fp64 oracle, as it stands, on the first n_layers of the chained
+    stack (layer l + 1 reads the oracle's bf16-rounded output of layer l)."""
     from oracle import moe_oracle as O
-    import threadpoolctl
     cfg = st.cfg
-    inputs = [oracle_layer_inputs(st, l) for l in range(n_layers)]
+    inputs = oracle_stack_inputs(st, n_layers)
+    x = st.x_host
     t0 = time.perf_counter()
-    for l, (wr, bias, recs, shared) in enumerate(inputs):
+    for wr, bias, recs, shared in inputs:
         cache = O.ExpertCache(lambda e, r=recs: O.sections_from_record(r[e], cfg.d, cfg.f, cfg.bits),
                               cfg.d, cfg.f, cfg.bits)
         sh = O.expert_weights(O.sections_from_record(shared, cfg.d, cfg.f, cfg.bits), cfg.d, cfg.f, cfg.bits)
-        O.layer_forward(st.x_host[l], wr, cfg.k, cache, sh, bias=bias)
+        y = O.layer_forward(x, wr, cfg.k, cache, sh, bias=bias, residual=True)["y"]
+        x = _bf16_bits(y)
     dt = time.perf_counter() - t0
     per_layer = dt / n_layers
-    info = threadpoolctl.threadpool_info()
-    cores = max([i.get("num_threads", 1) for i in info] + [1])
+    cores = _oracle_threads()
     return {"value": round(st.T / (per_layer * LAYERS), 4), "unit": "tokens/s (48-layer MoE stack)",
-            "cores": cores, "kind": "oracle",
-            "sample": f"{n_layers} of 48 layers at T={st.T} (fp64 numpy oracle, {dt:.1f} s), scaled to 48 layers"}
+            "cores": cores, "kind": "oracle", "host": cpu_info(),
+            "sample": f"first {n_layers} of 48 chained layers at T={st.T} (fp64 numpy oracle, {dt:.1f} s), "
+                      f"scaled to 48 layers"}
+
+
+def _bf16_bits(y):
+    """fp64 -> bf16 bits, round to nearest even (the next layer's input)."""
+    f = np.asarray(y, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = ((f + 0x7FFF + ((f >> 16) & 1)) >> 16).astype(np.uint16)
+    return r
+
+
+def _oracle_threads():
+    import threadpoolctl
+    return max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
 
 
 def prefill_oracle_inputs(pl, tokens):
@@ -617,7 +723,7 @@ def cpu_baseline_prefill(pl, n_tokens):
     dt = time.perf_counter() - t0
     cores = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
     return {"value": round(n_tokens / dt, 3), "unit": f"tokens/s (one MoE layer, prefill chunk T={pl.T})",
-            "cores": cores, "kind": "oracle",
+            "cores": cores, "kind": "oracle", "host": cpu_info(),
             "sample": f"first {n_tokens} of {pl.T} tokens of the chunk (fp64 numpy oracle, {dt:.1f} s)"}
 
 
@@ -631,10 +737,9 @@ def run_reference(args):
         return run_reference_prefill(args, world)
     from oracle import moe_oracle as O
     from bit_expert_ffn_router_b200 import synth
-    import threadpoolctl
     cfg_d, cfg_f, E, k, bits = 2048, 768, 512, 10, args.bits
     T = args.tokens
-    layers_per_step = 2
+    layers_per_step = 2  # the first two layers of the chain per step
     layers = []
     for l in range(layers_per_step):
         wr = synth.router_weights(E, cfg_d, SEED + 1000 * l + 1)
@@ -642,32 +747,32 @@ def run_reference(args):
         sel = np.unique(np.argsort(-bias, axis=1)[:, :k])
         secs = {int(e): synth.expert_sections(cfg_d, cfg_f, bits, SEED + 100 + 1000 * l + int(e)) for e in sel}
         shared = synth.expert_sections(cfg_d, cfg_f, bits, SEED + 99 + 1000 * l)
-        x = synth.activations(T, cfg_d, SEED + 1000 * l + 16)
-        layers.append((x, wr, bias, secs, shared))
+        layers.append((wr, bias, secs, shared))
+    x0 = synth.activations(T, cfg_d, SEED + 16)
     times = []
     for step in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        for x, wr, bias, secs, shared in layers:
+        x = x0
+        for wr, bias, secs, shared in layers:
             cache = O.ExpertCache(lambda e, s=secs: s[e], cfg_d, cfg_f, bits)
             sh = O.expert_weights(shared, cfg_d, cfg_f, bits)
-            O.layer_forward(x, wr, k, cache, sh, bias=bias)
+            x = _bf16_bits(O.layer_forward(x, wr, k, cache, sh, bias=bias, residual=True)["y"])
         dt = time.perf_counter() - t0
         if step >= args.warmup:
             times.append(dt / layers_per_step)
     per_layer = float(np.mean(times))
     value = T / (per_layer * LAYERS)
-    cores = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
-    sample = f"{layers_per_step} of 48 layers per step at T={T}, scaled to 48 layers"
+    sample = (f"the first {layers_per_step} of 48 chained layers per step at T={T} "
+              f"({per_layer * layers_per_step * 1e3:.0f} ms of oracle work per step), scaled to 48 layers")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s (48-layer MoE stack)",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(per_layer * LAYERS * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": round(per_layer * layers_per_step * 1e3, 2), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"decode layer d=2048 f=768 E=512 top-10 + 1 shared, T={T}, {bits}-bit; "
-                               f"48 distinct layers per step (oracle sample)", "global_batch": T, "seq_len": 1,
-                   "parallelism": "cpu"},
-        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s (48-layer MoE stack)", "cores": cores,
-                         "kind": "oracle", "sample": sample},
+        "config": {"workload": workload_name(T, bits, correlated=args.workload == "stack"), "global_batch": T,
+                   "seq_len": 1, "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s (48-layer MoE stack)",
+                         "cores": _oracle_threads(), "kind": "oracle", "sample": sample, "host": cpu_info()},
         "e2e": {"value": round(value, 4), "unit": "tokens/s (48-layer MoE stack)", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }), flush=True)
@@ -695,7 +800,7 @@ def run_reference_prefill(args, world):
         if step >= args.warmup:
             times.append(time.perf_counter() - t0)
     value = n / float(np.mean(times))
-    cores = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
+    cores = _oracle_threads()
     unit = f"tokens/s (one MoE layer, prefill chunk T={T})"
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world,
@@ -705,7 +810,7 @@ def run_reference_prefill(args, world):
                                f"(oracle on {n} tokens per step)", "global_batch": n, "seq_len": T,
                    "parallelism": "cpu"},
         "cpu_baseline": {"value": round(value, 3), "unit": unit, "cores": cores, "kind": "oracle",
-                         "sample": f"{n} of {T} tokens per step"},
+                         "sample": f"{n} of {T} tokens per step", "host": cpu_info()},
         "e2e": {"value": round(value, 3), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
@@ -720,13 +825,24 @@ def main():
     ap.add_argument("--bits", type=int, default=2)
     ap.add_argument("--cpu-layers", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"])
+    ap.add_argument("--no-extras", action="store_true", help="decode: only the headline configuration")
+    ap.add_argument("--workload", default="decode", choices=["decode", "stack", "prefill"],
+                    help="decode: T tokens, one routing draw; stack: the 48-layer stack over 256 correlated "
+                         "decode steps (use --tokens 4 for the verify width); prefill: one layer, T=8192")
     ap.add_argument("--layers", type=int, default=LAYERS,
                     help="decode: layers in the stack (fewer only to profile a small case)")
     ap.add_argument("--cpu-tokens", type=int, default=32, help="prefill: oracle sample size")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: relaunch under torch.distributed.run
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+               "--master-addr=127.0.0.1", "--master-port=29531", os.path.abspath(__file__)] + sys.argv[1:]
+        sys.exit(subprocess.call(cmd))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.gpus != world:
+        sys.exit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     if args.impl == "reference":
         run_reference(args)
     elif args.workload == "prefill":

@@ -31,6 +31,8 @@
 // Every wait is bounded by a global-timer deadline; on expiry the kernel
 // records MOE_ETIMEOUT in the context's status word, stops working and
 // returns. A kernel that finds the status word already set does nothing.
+#include <cstdio>
+#include <cstdlib>
 #include <random>
 
 #include "moe_internal.cuh"
@@ -39,12 +41,13 @@
 namespace moe {
 
 __host__ __device__ constexpr int ds_consumer_warps(int bits) { return bits == 2 ? 15 : 11; }
-constexpr int kDsNGU = 8;       // gate/up ring slots (at most)
-constexpr int kDsNDN = 16;      // down ring slots (at most)
+constexpr int kDsNS = 12;       // weight ring slots (at most)
 constexpr int kDsNHS = 4;       // h staging slots of the gate/up epilogue
 constexpr int kDsCps = 16;      // gate/up channels per ring stage
 constexpr int kQW = 18;         // words per quantised 32-value block: 16 int16 pairs, scale, sum
 constexpr int kDsMaxCtas = 256;  // grid size limit (done words per layer parity)
+constexpr int kDsLogitCopies = 4;  // copies of the logit words: CTA b reads copy b % 4
+constexpr int kDsPollNs = 64;      // back-off between polls of words that were not there yet
 
 // Tag source: every launch reads it and the last CTA to exit advances it by
 // the number of layers; tags of a launch are base + 1 .. base + L.
@@ -73,7 +76,7 @@ struct DSParams {
   size_t rec_bytes;
   RecOff ro;
   GroupPtrs g;                  // not route: the given grouping
-  unsigned long long* logits_ll;  // [T, E]
+  unsigned long long* logits_ll;  // [kDsLogitCopies, T, E]
   unsigned long long* h_ll;       // [n_rows, f/32, kQW]
   unsigned long long* y_ll;       // [2, T, d/2]
   unsigned long long* done_ll;    // [2, kDsMaxCtas]
@@ -84,14 +87,15 @@ struct DSParams {
   int gu_lpr, dn_lpr, gran, n_units;
   int gu_row, gu_sc, dn_row, dn_sc;  // bytes per row: codes, scales
   int rpc;                      // output rows per CTA (at most)
-  int n_gu, n_dn, gu_slot, dn_slot;
+  int n_ring, slot_bytes;       // weight ring: slots and bytes per slot
+  int dn_stride, gpd;           // bytes per down stage, down stages per ring slot
   int hq_rows;
-  int sm_wr, sm_x, sm_xq, sm_hs, sm_zs, sm_route, sm_xres, sm_gu, sm_dn;
+  int sm_wr, sm_x, sm_xq, sm_hs, sm_zs, sm_route, sm_xres, sm_ring, sm_shdn;
 };
 
 struct DSShared {
-  uint64_t gu_full[kDsNGU], gu_empty[kDsNGU];
-  uint64_t dn_full[kDsNDN], dn_empty[kDsNDN];
+  uint64_t full[kDsNS], empty[kDsNS];   // weight ring
+  uint64_t shdn_full[2], shdn_empty[2];  // the shared expert's down rows, by layer parity
   uint64_t wr_full, wr_empty, route_bar;
   int abort_flag;
   unsigned base_tag;
@@ -177,17 +181,6 @@ __device__ __forceinline__ bool ds_aborted(const DSShared* S) {
   return *reinterpret_cast<const volatile int*>(&S->abort_flag) != 0;
 }
 
-// Polls a tagged word until its tag matches (false on timeout or abort).
-__device__ __forceinline__ bool poll_ll(const unsigned long long* p, uint32_t tag, unsigned long long& w,
-                                        const DSShared* S, uint64_t deadline) {
-  while (!tag_ok(w, tag)) {
-    if (ds_aborted(S) || global_timer_ns() > deadline) return false;
-    __nanosleep(20);
-    w = ld_ll(p);
-  }
-  return true;
-}
-
 // Warp-wide bounded mbarrier wait by lane 0 (false on timeout or abort).
 __device__ __forceinline__ bool ds_wait_warp(uint64_t* b, uint32_t parity, const DSShared* S, uint64_t deadline) {
   int ok = 1;
@@ -248,9 +241,14 @@ __device__ __forceinline__ uint32_t quant_block_warp(float v, int lane) {
 
 // ------------------------------------------------------------------ x of a layer
 // Every consumer thread takes part. Layer 0 (or the given-grouping mode)
-// reads the bf16 input; layer l > 0 polls the previous layer's output words
-// and every CTA's done word. Writes the raw bf16 rows (xs, for the router),
-// the quantised gate/up operand (xq) and this CTA's residual rows (xres).
+// reads the bf16 input; layer l > 0 reads the previous layer's output words
+// and every CTA's done word. A thread issues the loads of up to kXB jobs
+// (four words each) at once and re-polls, all together, only the words whose
+// tag was not there yet, so a batch costs about one L2 round trip. Writes the
+// raw bf16 rows (xs, for the router), the quantised gate/up operand (xq) and
+// this CTA's residual rows (xres).
+constexpr int kXB = 4;
+
 template <int BITS>
 __device__ void ds_read_x(const DSParams& P, int l, uint32_t tag, uint16_t* xs, int* xq, float* xres, int r0,
                           int r1, DSShared* S, uint64_t deadline, int CT) {
@@ -260,56 +258,88 @@ __device__ void ds_read_x(const DSParams& P, int l, uint32_t tag, uint16_t* xs, 
   const int tid = threadIdx.x;
   const bool chained = l > 0;
   const unsigned long long* yl = P.y_ll + static_cast<size_t>((l - 1) & 1) * P.T * (P.d / 2);
-  if (chained && tid < gridDim.x) {  // every CTA has finished the previous layer
-    const unsigned long long* dp = P.done_ll + static_cast<size_t>((l - 1) & 1) * kDsMaxCtas + tid;
-    unsigned long long w = ld_ll(dp);
-    if (!poll_ll(dp, tag - 1, w, S, deadline) && !ds_aborted(S)) ds_abort(S, P.status, 20);
-  }
+  const int per_thread = (jobs + CT - 1) / CT;
 #pragma unroll 1
-  for (int j = tid; j < ((jobs + CT - 1) / CT) * CT; j += CT) {
-    const bool live = j < jobs;
-    const int blk_all = live ? j >> 2 : 0;
-    const int q = j & 3;
-    const int t = blk_all / nb, blk = blk_all % nb;
-    uint32_t w4[4];
+  for (int k0 = 0; k0 < per_thread; k0 += kXB) {
+    uint32_t w4[kXB][4];
     if (!chained) {
-      const uint4 raw = __ldcg(reinterpret_cast<const uint4*>(P.x + static_cast<size_t>(t) * P.d + blk * kBlock + 8 * q));
-      w4[0] = raw.x;
-      w4[1] = raw.y;
-      w4[2] = raw.z;
-      w4[3] = raw.w;
-    } else {
-      const unsigned long long* p = yl + static_cast<size_t>(t) * (P.d / 2) + blk * 16 + 4 * q;
-      unsigned long long a, b, c, d;
-      ld_ll2(p, a, b);
-      ld_ll2(p + 2, c, d);
-      if (!ds_aborted(S)) {
-        bool ok = poll_ll(p, tag - 1, a, S, deadline) && poll_ll(p + 1, tag - 1, b, S, deadline) &&
-                  poll_ll(p + 2, tag - 1, c, S, deadline) && poll_ll(p + 3, tag - 1, d, S, deadline);
-        if (!ok && !ds_aborted(S)) ds_abort(S, P.status, 21);
+#pragma unroll
+      for (int i = 0; i < kXB; ++i) {
+        const int j = tid + (k0 + i) * CT;
+        const int job = j < jobs ? j >> 2 : 0, q = j & 3;
+        const int t = job / nb, blk = job % nb;
+        const uint4 raw =
+            __ldcg(reinterpret_cast<const uint4*>(P.x + static_cast<size_t>(t) * P.d + blk * kBlock + 8 * q));
+        w4[i][0] = raw.x;
+        w4[i][1] = raw.y;
+        w4[i][2] = raw.z;
+        w4[i][3] = raw.w;
       }
-      w4[0] = static_cast<uint32_t>(a);
-      w4[1] = static_cast<uint32_t>(b);
-      w4[2] = static_cast<uint32_t>(c);
-      w4[3] = static_cast<uint32_t>(d);
-    }
-    float v[8];
+    } else {
+      unsigned long long v[kXB][4];
+      const unsigned long long* src[kXB];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint16_t h = static_cast<uint16_t>(w4[i >> 1] >> (16 * (i & 1)));
-      v[i] = live ? bf16_bits_to_float(h) : 0.f;
-    }
-    if (live) {
-      if (xs != nullptr)
-        *reinterpret_cast<uint4*>(xs + static_cast<size_t>(t) * P.d + blk * kBlock + 8 * q) =
-            make_uint4(w4[0], w4[1], w4[2], w4[3]);
-      const int c0 = blk * kBlock + 8 * q;
+      for (int i = 0; i < kXB; ++i) {
+        const int j = tid + (k0 + i) * CT;
+        const int job = j < jobs ? j >> 2 : 0, q = j & 3;
+        const int t = job / nb, blk = job % nb;
+        src[i] = yl + static_cast<size_t>(t) * (P.d / 2) + blk * 16 + 4 * q;
+        ld_ll2(src[i], v[i][0], v[i][1]);
+        ld_ll2(src[i] + 2, v[i][2], v[i][3]);
+      }
+      // every CTA's done word rides along in the first batch
+      const unsigned long long* dp = P.done_ll + static_cast<size_t>((l - 1) & 1) * kDsMaxCtas + tid;
+      const bool has_done = k0 == 0 && tid < static_cast<int>(gridDim.x);
+      unsigned long long dw = has_done ? ld_ll(dp) : ll_word(0u, tag - 1);
+      while (true) {
+        bool all = tag_ok(dw, tag - 1);
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (c0 + i >= r0 && c0 + i < r1) xres[t * P.rpc + (c0 + i - r0)] = v[i];
+        for (int i = 0; i < kXB; ++i)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) all = all && tag_ok(v[i][c], tag - 1);
+        if (all) break;
+        if (ds_aborted(S) || global_timer_ns() > deadline) {
+          if (!ds_aborted(S)) ds_abort(S, P.status, 21);
+          break;
+        }
+        __nanosleep(kDsPollNs);
+        if (!tag_ok(dw, tag - 1)) dw = ld_ll(dp);
+#pragma unroll
+        for (int i = 0; i < kXB; ++i)
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            if (!tag_ok(v[i][c], tag - 1)) v[i][c] = ld_ll(src[i] + c);
+      }
+#pragma unroll
+      for (int i = 0; i < kXB; ++i)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) w4[i][c] = static_cast<uint32_t>(v[i][c]);
     }
-    const int gl = blk / bpl, bb = blk % bpl;
-    quant_quad_c2(v, xq + t * words, nb, bb * P.gu_lpr + gl, q, live);
+#pragma unroll
+    for (int i = 0; i < kXB; ++i) {
+      if (k0 + i >= per_thread) break;  // uniform across the warp
+      const int j = tid + (k0 + i) * CT;
+      const bool live = j < jobs;
+      const int job = live ? j >> 2 : 0, q = j & 3;
+      const int t = job / nb, blk = job % nb;
+      float v8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint16_t h = static_cast<uint16_t>(w4[i][e >> 1] >> (16 * (e & 1)));
+        v8[e] = live ? bf16_bits_to_float(h) : 0.f;
+      }
+      if (live) {
+        if (xs != nullptr)
+          *reinterpret_cast<uint4*>(xs + static_cast<size_t>(t) * P.d + blk * kBlock + 8 * q) =
+              make_uint4(w4[i][0], w4[i][1], w4[i][2], w4[i][3]);
+        const int c0 = blk * kBlock + 8 * q;
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (c0 + e >= r0 && c0 + e < r1) xres[t * P.rpc + (c0 + e - r0)] = v8[e];
+      }
+      const int gl = blk / bpl, bb = blk % bpl;
+      quant_quad_c2(v8, xq + t * words, nb, bb * P.gu_lpr + gl, q, live);
+    }
   }
 }
 
@@ -339,13 +369,26 @@ __device__ void ds_topk(const DSParams& P, const DSRoute& R, int t, uint32_t tag
                         unsigned long long* scratch, DSShared* S, uint64_t deadline) {
   constexpr int VPL = 16;
   const int lane = threadIdx.x & 31;
-  const unsigned long long* row = P.logits_ll + static_cast<size_t>(t) * P.E;
+  const unsigned long long* row =
+      P.logits_ll + (static_cast<size_t>(blockIdx.x % kDsLogitCopies) * P.T + t) * P.E;
   unsigned long long w[VPL];
 #pragma unroll
   for (int v = 0; v < VPL; ++v) w[v] = ld_ll(row + min(v * 32 + lane, P.E - 1));
   bool ok = true;
+  while (true) {  // re-poll only the words not there yet, all at once
+    bool all = true;
 #pragma unroll
-  for (int v = 0; v < VPL; ++v) ok = ok && poll_ll(row + min(v * 32 + lane, P.E - 1), tag, w[v], S, deadline);
+    for (int v = 0; v < VPL; ++v) all = all && tag_ok(w[v], tag);
+    if (all) break;
+    if (ds_aborted(S) || global_timer_ns() > deadline) {
+      ok = false;
+      break;
+    }
+    __nanosleep(kDsPollNs);
+#pragma unroll
+    for (int v = 0; v < VPL; ++v)
+      if (!tag_ok(w[v], tag)) w[v] = ld_ll(row + min(v * 32 + lane, P.E - 1));
+  }
   if (!__all_sync(0xffffffffu, ok)) {
     if (lane == 0 && !ds_aborted(S)) ds_abort(S, P.status, 22);
     return;
@@ -575,7 +618,8 @@ __device__ void ds_router(const DSParams& P, int l, uint32_t tag, const float* w
       acc = fmaf(w.w, __uint_as_float(xb.y & 0xffff0000u), acc);
     }
     acc = warp_sum(acc);
-    if (lane == 0) st_ll(P.logits_ll + o, ll_word(__float_as_uint(acc + bv), tag));
+    if (lane < kDsLogitCopies)
+      st_ll(P.logits_ll + static_cast<size_t>(lane) * P.T * P.E + o, ll_word(__float_as_uint(acc + bv), tag));
   }
 }
 
@@ -644,37 +688,76 @@ __device__ __forceinline__ void gu_task(const DSParams& P, const DSRoute& R, con
 }
 
 // ------------------------------------------------------------------ down
-// Stages the quantised h rows [rows of DN stages i0..i1) into hq by polling
-// their tagged words (every consumer thread takes part), in stage order.
+// Stages the quantised h rows of DN stages [i0, i1) into hq (every consumer
+// thread takes part), in stage order. A thread loads up to kHB 16-byte units
+// at once and re-polls, together, only the words not there yet.
+constexpr int kHB = 8;
+
 __device__ void ds_stage_h(const DSParams& P, const DSRoute& R, int np, int i0, int i1, bool sh_first, uint32_t tag,
                            int* hq, DSShared* S, uint64_t deadline, int CT) {
   const int nbf = P.f / kBlock, bpl = nbf / P.dn_lpr;
   const int units_per_row = nbf * (kQW / 2);  // 16-byte units
-  int row_base = 0;
-#pragma unroll 1
+  // rows of the round: stage order, each stage's rows contiguous in h
+  int n_rows = 0;
   for (int i = i0; i < i1; ++i) {
     const int u = (sh_first && i == 0) ? -1 : i - (sh_first ? 1 : 0);
     int first, n;
     expert_h_rows(R, u, np, P.T, first, n);
-    const int units = n * units_per_row;
+    n_rows += n;
+  }
+  const int units = n_rows * units_per_row;
 #pragma unroll 1
-    for (int j = threadIdx.x; j < units; j += CT) {
+  for (int j0 = threadIdx.x; j0 < units; j0 += kHB * CT) {
+    unsigned long long v[kHB][2];
+    const unsigned long long* src[kHB];
+    int dst_row[kHB], dst_col[kHB], dst_w[kHB];
+#pragma unroll
+    for (int k = 0; k < kHB; ++k) {
+      const int j = min(j0 + k * CT, units - 1);
       const int r = j / units_per_row, rem = j % units_per_row;
-      const int blk = rem / (kQW / 2), w2 = rem % (kQW / 2);
-      const unsigned long long* src =
-          P.h_ll + (static_cast<size_t>(first + r) * nbf + blk) * kQW + 2 * w2;
-      unsigned long long a, b;
-      ld_ll2(src, a, b);
-      if (!ds_aborted(S)) {
-        const bool ok = poll_ll(src, tag, a, S, deadline) && poll_ll(src + 1, tag, b, S, deadline);
-        if (!ok && !ds_aborted(S)) ds_abort(S, P.status, 23);
+      // row r of the round -> its h row (walk the stages)
+      int base = 0, hrow = 0;
+      for (int i = i0; i < i1; ++i) {
+        const int u = (sh_first && i == 0) ? -1 : i - (sh_first ? 1 : 0);
+        int first, n;
+        expert_h_rows(R, u, np, P.T, first, n);
+        if (r < base + n) {
+          hrow = first + (r - base);
+          break;
+        }
+        base += n;
       }
-      const int col = (blk % bpl) * P.dn_lpr + blk / bpl;
-      int* dst = hq + (row_base + r) * kQW * nbf;
-      dst[(2 * w2) * nbf + col] = static_cast<int>(static_cast<uint32_t>(a));
-      dst[(2 * w2 + 1) * nbf + col] = static_cast<int>(static_cast<uint32_t>(b));
+      const int blk = rem / (kQW / 2), w2 = rem % (kQW / 2);
+      src[k] = P.h_ll + (static_cast<size_t>(hrow) * nbf + blk) * kQW + 2 * w2;
+      dst_row[k] = r;
+      dst_col[k] = (blk % bpl) * P.dn_lpr + blk / bpl;
+      dst_w[k] = 2 * w2;
+      ld_ll2(src[k], v[k][0], v[k][1]);
     }
-    row_base += n;
+    while (true) {
+      bool all = true;
+#pragma unroll
+      for (int k = 0; k < kHB; ++k) all = all && tag_ok(v[k][0], tag) && tag_ok(v[k][1], tag);
+      if (all) break;
+      if (ds_aborted(S) || global_timer_ns() > deadline) {
+        if (!ds_aborted(S)) ds_abort(S, P.status, 23);
+        break;
+      }
+      __nanosleep(kDsPollNs);
+#pragma unroll
+      for (int k = 0; k < kHB; ++k) {
+        if (!tag_ok(v[k][0], tag)) v[k][0] = ld_ll(src[k]);
+        if (!tag_ok(v[k][1], tag)) v[k][1] = ld_ll(src[k] + 1);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kHB; ++k) {
+      if (j0 + k * CT < units) {
+        int* dst = hq + dst_row[k] * kQW * nbf;
+        dst[dst_w[k] * nbf + dst_col[k]] = static_cast<int>(static_cast<uint32_t>(v[k][0]));
+        dst[(dst_w[k] + 1) * nbf + dst_col[k]] = static_cast<int>(static_cast<uint32_t>(v[k][1]));
+      }
+    }
   }
 }
 
@@ -707,32 +790,34 @@ __device__ __forceinline__ void dn_task(const DSParams& P, const DSRoute& R, con
 }
 
 // ------------------------------------------------------------------ producer
-struct DSProducer {
-  uint32_t gu_seq = 0, dn_seq = 0;
-};
-
+// One ring of fixed-size slots carries, in order, every gate/up stage (16
+// channels) and down group (the down rows of up to `gpd` routed experts) of
+// a layer; consumers free a slot with 16 arrivals. Down groups follow the
+// gate/up stages, so they stream in while gate/up is still computing.
 __device__ __forceinline__ bool ring_slot_free(uint64_t* empty, uint32_t seq, int n) {
   return seq < static_cast<uint32_t>(n) || mbar_test(&empty[seq % n], ((seq / n) - 1) & 1);
 }
 
-__device__ __forceinline__ void issue_gu(const DSParams& P, DSShared* S, uint8_t* ring, uint32_t seq,
-                                         const uint8_t* rec, int ch0) {
-  const int slot = seq % P.n_gu;
-  uint8_t* dst = ring + static_cast<size_t>(slot) * P.gu_slot;
-  const uint32_t cb = 2 * kDsCps * P.gu_row, sb = 2 * kDsCps * P.gu_sc;
-  mbar_arrive_expect_tx(&S->gu_full[slot], cb + sb);
-  bulk_g2s(dst, rec + P.lay.gu_codes + static_cast<size_t>(2 * ch0) * P.gu_row, cb, &S->gu_full[slot]);
-  bulk_g2s(dst + cb, rec + P.lay.gu_scales + static_cast<size_t>(2 * ch0) * P.gu_sc, sb, &S->gu_full[slot]);
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
 }
 
-__device__ __forceinline__ void issue_dn(const DSParams& P, DSShared* S, uint8_t* ring, uint32_t seq,
-                                         const uint8_t* rec, int r0, int r1) {
-  const int slot = seq % P.n_dn;
-  uint8_t* dst = ring + static_cast<size_t>(slot) * P.dn_slot;
+__device__ __forceinline__ void issue_gu(const DSParams& P, DSShared* S, uint8_t* ring, uint32_t seq,
+                                         const uint8_t* rec, int ch0) {
+  const int slot = seq % P.n_ring;
+  uint8_t* dst = ring + static_cast<size_t>(slot) * P.slot_bytes;
+  const uint32_t cb = 2 * kDsCps * P.gu_row, sb = 2 * kDsCps * P.gu_sc;
+  mbar_arrive_expect_tx(&S->full[slot], cb + sb);
+  bulk_g2s(dst, rec + P.lay.gu_codes + static_cast<size_t>(2 * ch0) * P.gu_row, cb, &S->full[slot]);
+  bulk_g2s(dst + cb, rec + P.lay.gu_scales + static_cast<size_t>(2 * ch0) * P.gu_sc, sb, &S->full[slot]);
+}
+
+// Down rows [r0, r1) of one record into dst (codes, then scales).
+__device__ __forceinline__ void copy_dn(const DSParams& P, uint8_t* dst, const uint8_t* rec, int r0, int r1,
+                                        uint64_t* bar) {
   const uint32_t cb = (r1 - r0) * P.dn_row, sb = (r1 - r0) * P.dn_sc;
-  mbar_arrive_expect_tx(&S->dn_full[slot], cb + sb);
-  bulk_g2s(dst, rec + P.lay.dn_codes + static_cast<size_t>(r0) * P.dn_row, cb, &S->dn_full[slot]);
-  bulk_g2s(dst + cb, rec + P.lay.dn_scales + static_cast<size_t>(r0) * P.dn_sc, sb, &S->dn_full[slot]);
+  bulk_g2s(dst, rec + P.lay.dn_codes + static_cast<size_t>(r0) * P.dn_row, cb, bar);
+  bulk_g2s(dst + cb, rec + P.lay.dn_scales + static_cast<size_t>(r0) * P.dn_sc, sb, bar);
 }
 
 // Waits (bounded) until ring slot `seq` may be reused.
@@ -760,8 +845,8 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
   float* hs = reinterpret_cast<float*>(smem + P.sm_hs);
   float* zs = reinterpret_cast<float*>(smem + P.sm_zs);
   float* xres = reinterpret_cast<float*>(smem + P.sm_xres);
-  uint8_t* gu_ring = reinterpret_cast<uint8_t*>(smem + P.sm_gu);
-  uint8_t* dn_ring = reinterpret_cast<uint8_t*>(smem + P.sm_dn);
+  uint8_t* ring = reinterpret_cast<uint8_t*>(smem + P.sm_ring);
+  uint8_t* shdn = reinterpret_cast<uint8_t*>(smem + P.sm_shdn);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, b = blockIdx.x;
@@ -780,13 +865,13 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
   const bool wr_rows = ROUTE && e1 > e0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kDsNGU; ++i) {
-      mbar_init(&S->gu_full[i], 1);
-      mbar_init(&S->gu_empty[i], kDsCps);
+    for (int i = 0; i < kDsNS; ++i) {
+      mbar_init(&S->full[i], 1);
+      mbar_init(&S->empty[i], kDsCps);
     }
-    for (int i = 0; i < kDsNDN; ++i) {
-      mbar_init(&S->dn_full[i], 1);
-      mbar_init(&S->dn_empty[i], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S->shdn_full[i], 1);
+      mbar_init(&S->shdn_empty[i], 1);
     }
     mbar_init(&S->wr_full, 1);
     mbar_init(&S->wr_empty, CW);
@@ -809,32 +894,47 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
   const uint64_t t_start = global_timer_ns();
   const uint64_t deadline = t_start + P.timeout_ns;
   unsigned long long* trace = P.trace != nullptr && b < kTraceCtas ? P.trace + b * kTraceSlots : nullptr;
+  const int dl = P.L > 1 ? 1 : 0;
 
   if (warp == CW) {
     // ============================================================ producer
     if (lane == 0) {
-      uint32_t gu_seq = 0, dn_seq = 0, wr_count = 0;
+      uint32_t seq = 0, wr_count = 0, shdn_count = 0;
       bool ok = true;
-      auto issue_shared = [&](int l) {
-        const uint8_t* rec = P.shared + static_cast<size_t>(l) * P.stride;
-        for (int blk = sb0; blk < sb1 && ok; ++blk)
-          for (int s = 0; s < 32 / kDsCps && ok; ++s) {
-            if (!(ok = wait_slot(S, S->gu_empty, gu_seq, P.n_gu, deadline))) break;
-            issue_gu(P, S, gu_ring, gu_seq++, rec, blk * 32 + s * kDsCps);
-          }
-        if (ok && has_rows) {
-          if ((ok = wait_slot(S, S->dn_empty, dn_seq, P.n_dn, deadline))) issue_dn(P, S, dn_ring, dn_seq++, rec, r0, r1);
-        }
-      };
       auto issue_wr = [&](int l) {
         const uint32_t bytes = static_cast<uint32_t>((e1 - e0) * P.d * 4);
         mbar_arrive_expect_tx(&S->wr_full, bytes);
         bulk_g2s(wrs, P.wr + (static_cast<size_t>(l) * P.E + e0) * P.d, bytes, &S->wr_full);
         ++wr_count;
       };
+      // layer l's shared-expert down rows: buffer l & 1, its (l >> 1)-th use
+      auto issue_shdn = [&](int l) {
+        const int j = l & 1;
+        if (l >= 2) {
+          while (!mbar_try_wait(&S->shdn_empty[j], ((l >> 1) - 1) & 1, 20000u)) {
+            if (ds_aborted(S) || global_timer_ns() > deadline) {
+              ok = false;
+              return;
+            }
+          }
+        }
+        const uint8_t* rec = P.shared + static_cast<size_t>(l) * P.stride;
+        mbar_arrive_expect_tx(&S->shdn_full[j], (r1 - r0) * (P.dn_row + P.dn_sc));
+        copy_dn(P, shdn + j * P.dn_stride, rec, r0, r1, &S->shdn_full[j]);
+        ++shdn_count;
+      };
+      auto issue_shgu = [&](int l) {
+        const uint8_t* rec = P.shared + static_cast<size_t>(l) * P.stride;
+        for (int blk = sb0; blk < sb1 && ok; ++blk)
+          for (int q = 0; q < 32 / kDsCps && ok; ++q) {
+            if (!(ok = wait_slot(S, S->empty, seq, P.n_ring, deadline))) break;
+            issue_gu(P, S, ring, seq++, rec, blk * 32 + q * kDsCps);
+          }
+      };
       if (!ds_aborted(S)) {
         if (wr_rows) issue_wr(0);
-        if (P.has_shared) issue_shared(0);
+        if (P.has_shared && has_rows) issue_shdn(0);
+        if (P.has_shared) issue_shgu(0);
       }
       for (int l = 0; l < P.L && ok && !ds_aborted(S); ++l) {
         // routing of layer l is in shared memory once route_bar completes
@@ -845,30 +945,34 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
           }
         }
         if (!ok) break;
+        unsigned long long* td = (trace != nullptr && l == dl) ? trace : nullptr;
+        if (td) td[16] = global_timer_ns();
         const int nu = S->n_uniq;
         const int tot = nu * nbf;
         const int rb0 = static_cast<int>((static_cast<long long>(tot) * b) / G);
         const int rb1 = static_cast<int>((static_cast<long long>(tot) * (b + 1)) / G);
-        const int n_gu = (rb1 - rb0) * (32 / kDsCps);
-        const int n_dn = has_rows ? nu : 0;
-        int ig = 0, id = 0;
-        // gate/up stages first; a down stage whenever the gate/up ring is full
-        while ((ig < n_gu || id < n_dn) && ok) {
-          if (ig < n_gu && ring_slot_free(S->gu_empty, gu_seq, P.n_gu)) {
-            const int blk = rb0 + ig / (32 / kDsCps);
-            const int u = blk / nbf, cb = blk % nbf;
-            const uint8_t* rec = P.pool + static_cast<size_t>(R.uniq_slot[u]) * P.stride;
-            issue_gu(P, S, gu_ring, gu_seq++, rec, cb * 32 + (ig % (32 / kDsCps)) * kDsCps);
-            ++ig;
-          } else if (id < n_dn && ring_slot_free(S->dn_empty, dn_seq, P.n_dn)) {
-            const uint8_t* rec = P.pool + static_cast<size_t>(R.uniq_slot[id]) * P.stride;
-            issue_dn(P, S, dn_ring, dn_seq++, rec, r0, r1);
-            ++id;
-          } else {
-            if (ds_aborted(S) || global_timer_ns() > deadline) ok = false;
-            __nanosleep(32);
-          }
+        for (int ig = 0; ig < (rb1 - rb0) * (32 / kDsCps) && ok; ++ig) {
+          const int blk = rb0 + ig / (32 / kDsCps);
+          const int u = blk / nbf, cb = blk % nbf;
+          if (!(ok = wait_slot(S, S->empty, seq, P.n_ring, deadline))) break;
+          issue_gu(P, S, ring, seq++, P.pool + static_cast<size_t>(R.uniq_slot[u]) * P.stride,
+                   cb * 32 + (ig % (32 / kDsCps)) * kDsCps);
+          if (td && ig == 0) td[17] = global_timer_ns();
         }
+        if (td) td[18] = global_timer_ns();
+        const int n_grp = has_rows ? (nu + P.gpd - 1) / P.gpd : 0;
+        for (int g = 0; g < n_grp && ok; ++g) {
+          if (!(ok = wait_slot(S, S->empty, seq, P.n_ring, deadline))) break;
+          const int u0 = g * P.gpd, u1 = min(nu, u0 + P.gpd);
+          const int slot = seq % P.n_ring;
+          uint8_t* dst = ring + static_cast<size_t>(slot) * P.slot_bytes;
+          mbar_arrive_expect_tx(&S->full[slot], (u1 - u0) * (r1 - r0) * (P.dn_row + P.dn_sc));
+          for (int u = u0; u < u1; ++u)
+            copy_dn(P, dst + (u - u0) * P.dn_stride, P.pool + static_cast<size_t>(R.uniq_slot[u]) * P.stride, r0, r1,
+                    &S->full[slot]);
+          ++seq;
+        }
+        if (td) td[19] = global_timer_ns();
         if (!ok) break;
         if (l + 1 < P.L) {
           // the next layer's inputs that do not depend on x
@@ -882,18 +986,19 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
             if (!ok) break;
             issue_wr(l + 1);
           }
-          if (P.has_shared) issue_shared(l + 1);
+          if (P.has_shared && has_rows) issue_shdn(l + 1);
+          if (P.has_shared && ok) issue_shgu(l + 1);
         }
       }
       if (!ok && !ds_aborted(S)) ds_abort(S, P.status, 10);
       // every issued copy lands before the CTA may exit (they take
       // microseconds; the 100 ms bound only guards against the impossible)
       const uint64_t d2 = global_timer_ns() + 100000000ull;
-      for (uint32_t s = gu_seq > static_cast<uint32_t>(P.n_gu) ? gu_seq - P.n_gu : 0; s < gu_seq; ++s)
-        while (!mbar_try_wait(&S->gu_full[s % P.n_gu], (s / P.n_gu) & 1, 20000u) && global_timer_ns() < d2) {
+      for (uint32_t q = seq > static_cast<uint32_t>(P.n_ring) ? seq - P.n_ring : 0; q < seq; ++q)
+        while (!mbar_try_wait(&S->full[q % P.n_ring], (q / P.n_ring) & 1, 20000u) && global_timer_ns() < d2) {
         }
-      for (uint32_t s = dn_seq > static_cast<uint32_t>(P.n_dn) ? dn_seq - P.n_dn : 0; s < dn_seq; ++s)
-        while (!mbar_try_wait(&S->dn_full[s % P.n_dn], (s / P.n_dn) & 1, 20000u) && global_timer_ns() < d2) {
+      for (uint32_t q = shdn_count > 2u ? shdn_count - 2u : 0u; q < shdn_count; ++q)
+        while (!mbar_try_wait(&S->shdn_full[q & 1], (q >> 1) & 1, 20000u) && global_timer_ns() < d2) {
         }
       if (wr_count > 0)
         while (!mbar_try_wait(&S->wr_full, (wr_count - 1) & 1, 20000u) && global_timer_ns() < d2) {
@@ -903,12 +1008,15 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
   } else {
     // ============================================================ consumers
     const int tid = threadIdx.x;
-    uint32_t gu_seq = 0, dn_seq = 0, blk_seq = 0;
+    uint32_t seq = 0, blk_seq = 0;
     XR<BITS> xr[GBPL];
 #pragma unroll 1
     for (int l = 0; l < P.L; ++l) {
       const uint32_t tag = base + 1 + static_cast<uint32_t>(l);
-      const bool traced = trace != nullptr && l < 4 && tid == 0;
+      // trace slots: 8 phase stamps for layers 0 and 1, then details of
+      // layer dl (the second one when there is one)
+      const bool traced = trace != nullptr && l < 2 && tid == 0;
+      unsigned long long* tdet = (trace != nullptr && l == dl) ? trace : nullptr;
       if (traced) trace[8 * l] = global_timer_ns();
       // ---- x of this layer
       if (!ds_aborted(S))
@@ -937,10 +1045,12 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
                                : nullptr;
         if (warp < P.T && !ds_aborted(S))
           ds_topk(P, R, warp, tag, pub, reinterpret_cast<unsigned long long*>(hs) + warp * 32, S, deadline);
+        if (tdet && tid == 0) tdet[20] = global_timer_ns();
         named_sync(1, CT);
         if (!ds_aborted(S)) ds_group(P, R, S, np, CT);
         else named_sync(1, CT), named_sync(1, CT);
         nu = S->n_uniq;
+        if (tdet && tid == 0) tdet[21] = global_timer_ns();
         if (tid == 0) mbar_arrive(&S->route_bar);
         if (publisher && !ds_aborted(S)) ds_publish(P, R, l, np, nu, CT);
       } else {
@@ -979,8 +1089,8 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
         const int beta = task >> 5, c = task & 31;
         GUBlock gb;
         gu_block_of(beta, nsh, sb0, rb0, nbf, gb);
-        const uint32_t seq = gu_seq + beta * (32 / kDsCps) + c / kDsCps;
-        const int slot = seq % P.n_gu;
+        const uint32_t sq = seq + beta * (32 / kDsCps) + c / kDsCps;
+        const int slot = sq % P.n_ring;
         const uint32_t bid = blk_seq + beta;
         const int hslot = bid % kDsNHS;
         const int gen = bid / kDsNHS;
@@ -996,17 +1106,22 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok || !ds_wait_warp(&S->gu_full[slot], (seq / P.n_gu) & 1, S, deadline)) {
+        if (!ok || !ds_wait_warp(&S->full[slot], (sq / P.n_ring) & 1, S, deadline)) {
           if (lane == 0 && !ds_aborted(S)) ds_abort(S, P.status, 2);
           break;
         }
+        if (tdet && tid == 0) {
+          const int it = task / CW;
+          if (it == 0) tdet[22] = global_timer_ns();
+          if (it < 8) tdet[24 + it] = global_timer_ns();
+        }
         float* hsl = hs + hslot * P.T * 32;
-        gu_task<BITS, GBPL>(P, R, gu_ring + static_cast<size_t>(slot) * P.gu_slot, c % kDsCps, xq, gb.u, np, hsl,
+        gu_task<BITS, GBPL>(P, R, ring + static_cast<size_t>(slot) * P.slot_bytes, c % kDsCps, xq, gb.u, np, hsl,
                             c, cur_t, xr);
         __syncwarp();
         int last = 0;
         if (lane == 0) {
-          mbar_arrive(&S->gu_empty[slot]);
+          mbar_arrive(&S->empty[slot]);
           __threadfence_block();
           last = atomicAdd(&S->hs_done[hslot], 1) == 31;
         }
@@ -1030,57 +1145,87 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
           }
         }
       }
-      gu_seq += n_blk * (32 / kDsCps);
+      if (tdet && tid == 0) tdet[23] = global_timer_ns();
+      seq += n_blk * (32 / kDsCps);
       blk_seq += n_blk;
       named_sync(1, CT);
       if (traced) trace[8 * l + 4] = global_timer_ns();
 
-      // ---- down rows of this CTA for every expert (shared first)
-      const int n_dn = has_rows ? nu + (P.has_shared ? 1 : 0) : 0;
-      const bool sh_first = P.has_shared != 0;
+      // ---- down rows of this CTA for every expert (shared first). Stage i:
+      // the shared expert (i = 0, its own buffer) or routed expert u, whose
+      // rows sit in ring group u / gpd. A round of stages never spans more
+      // groups than the ring has slots, so no warp waits on a slot whose
+      // previous use in this layer is still pending.
+      const int sh = (P.has_shared && has_rows) ? 1 : 0;
+      const int n_dn = has_rows ? nu + sh : 0;
       const int nr_out = r1 - r0;
+      const uint32_t grp0 = seq;  // sequence number of this layer's first down group
 #pragma unroll 1
       for (int i0 = 0; i0 < n_dn;) {
-        // the stages whose h rows fit the staging area
         int i1 = i0, rows = 0;
         while (i1 < n_dn) {
-          const int u = (sh_first && i1 == 0) ? -1 : i1 - (sh_first ? 1 : 0);
+          const int u = i1 - sh;
+          if (u >= 0 && i1 > i0) {
+            const int ua = max(i0 - sh, 0);
+            if (u / P.gpd - ua / P.gpd >= P.n_ring) break;
+          }
           int first, n;
           expert_h_rows(R, u, np, P.T, first, n);
           if (rows + n > P.hq_rows) break;
           rows += n;
           ++i1;
         }
-        if (!ds_aborted(S)) ds_stage_h(P, R, np, i0, i1, sh_first, tag, hq, S, deadline, CT);
+        if (!ds_aborted(S)) ds_stage_h(P, R, np, i0, i1, sh != 0, tag, hq, S, deadline, CT);
         named_sync(1, CT);
         if (traced && i0 == 0) trace[8 * l + 5] = global_timer_ns();
-        // each warp takes whole stages; the hq row of stage i is the rows
-        // of the stages before it in this chunk
+        // each warp takes whole stages; the hq row of stage i is the rows of
+        // the stages before it in this round
 #pragma unroll 1
         for (int i = i0 + warp; i < i1; i += CW) {
           if (ds_aborted(S)) break;
           int row0 = 0;
           for (int j = i0; j < i; ++j) {
-            const int uj = (sh_first && j == 0) ? -1 : j - (sh_first ? 1 : 0);
             int fj, nj;
-            expert_h_rows(R, uj, np, P.T, fj, nj);
+            expert_h_rows(R, j - sh, np, P.T, fj, nj);
             row0 += nj;
           }
-          const int u = (sh_first && i == 0) ? -1 : i - (sh_first ? 1 : 0);
-          const uint32_t seq = dn_seq + i;
-          const int slot = seq % P.n_dn;
-          if (!ds_wait_warp(&S->dn_full[slot], (seq / P.n_dn) & 1, S, deadline)) {
+          const int u = i - sh;
+          const uint8_t* st;
+          uint64_t* full;
+          uint32_t parity;
+          int slot = 0;
+          if (u < 0) {
+            st = shdn + (l & 1) * P.dn_stride;
+            full = &S->shdn_full[l & 1];
+            parity = (l >> 1) & 1;
+          } else {
+            const uint32_t sq = grp0 + u / P.gpd;
+            slot = sq % P.n_ring;
+            st = ring + static_cast<size_t>(slot) * P.slot_bytes + (u % P.gpd) * P.dn_stride;
+            full = &S->full[slot];
+            parity = (sq / P.n_ring) & 1;
+          }
+          if (!ds_wait_warp(full, parity, S, deadline)) {
             if (lane == 0 && !ds_aborted(S)) ds_abort(S, P.status, 3);
             break;
           }
-          dn_task<BITS, DBPL>(P, R, dn_ring + static_cast<size_t>(slot) * P.dn_slot, u, np, hq, row0, nr_out, zs);
+          dn_task<BITS, DBPL>(P, R, st, u, np, hq, row0, nr_out, zs);
           __syncwarp();
-          if (lane == 0) mbar_arrive(&S->dn_empty[slot]);
+          if (lane == 0) {
+            if (u < 0) {
+              mbar_arrive(&S->shdn_empty[l & 1]);
+            } else {
+              // the group's 16 arrivals: its first expert brings the ones the
+              // group has no expert for
+              const int m = min(nu - (u / P.gpd) * P.gpd, P.gpd);
+              mbar_arrive_cnt(&S->empty[slot], (u % P.gpd) == 0 ? kDsCps - (m - 1) : 1);
+            }
+          }
         }
         named_sync(1, CT);
         i0 = i1;
       }
-      dn_seq += n_dn;
+      seq += has_rows ? (nu + P.gpd - 1) / P.gpd : 0;
       // this CTA has read everything of layer l that other CTAs wrote
       if (tid == 0 && ROUTE && l + 1 < P.L)
         st_ll(P.done_ll + static_cast<size_t>(l & 1) * kDsMaxCtas + b, ll_word(0u, tag));
@@ -1188,7 +1333,7 @@ bool decode_geometry_ok(int d, int f) {
 
 size_t decode_exchange_bytes(const moe_layer_cfg& c, int T) {
   const size_t n_rows = static_cast<size_t>(T) * c.k + (c.n_shared ? T : 0);
-  const size_t lg = ds_align(static_cast<size_t>(T) * c.E * 8, 256);
+  const size_t lg = ds_align(static_cast<size_t>(kDsLogitCopies) * T * c.E * 8, 256);
   const size_t h = ds_align(n_rows * (c.f / kBlock) * kQW * 8, 256);
   const size_t y = ds_align(2 * static_cast<size_t>(T) * (c.d / 2) * 8, 256);
   const size_t dn = 2 * kDsMaxCtas * 8;
@@ -1290,7 +1435,7 @@ cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const St
   if (a.g != nullptr) P.g = *a.g;
   {
     char* ex = a.exchange;
-    const size_t lg = ds_align(static_cast<size_t>(T) * c.E * 8, 256);
+    const size_t lg = ds_align(static_cast<size_t>(kDsLogitCopies) * T * c.E * 8, 256);
     const size_t h = ds_align(static_cast<size_t>(n_rows) * nbf * kQW * 8, 256);
     const size_t y = ds_align(2 * static_cast<size_t>(T) * (c.d / 2) * 8, 256);
     P.logits_ll = reinterpret_cast<unsigned long long*>(ex);
@@ -1316,8 +1461,12 @@ cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const St
   P.n_units = c.d / gran;
   P.rpc = gran * ((P.n_units + G - 1) / G);
   const int wr_rows = a.route ? (c.E + G - 1) / G : 0;
-  P.gu_slot = static_cast<int>(ds_align(static_cast<size_t>(2 * kDsCps) * (P.gu_row + P.gu_sc), 128));
-  P.dn_slot = static_cast<int>(ds_align(static_cast<size_t>(P.rpc) * (P.dn_row + P.dn_sc), 128));
+  // ring slots hold one gate/up stage (16 channels) or a group of down
+  // stages (this CTA's output rows of up to gpd experts)
+  const size_t gu_stage = static_cast<size_t>(2 * kDsCps) * (P.gu_row + P.gu_sc);
+  P.dn_stride = static_cast<int>(ds_align(static_cast<size_t>(P.rpc) * (P.dn_row + P.dn_sc), 16));
+  P.slot_bytes = static_cast<int>(ds_align(gu_stage > static_cast<size_t>(P.dn_stride) ? gu_stage : P.dn_stride, 128));
+  P.gpd = P.slot_bytes / P.dn_stride;
   // shared-memory map
   size_t o = ds_align(sizeof(DSShared), 128);
   P.sm_route = static_cast<int>(o);
@@ -1334,43 +1483,37 @@ cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const St
   o = ds_align(o + static_cast<size_t>(T) * kQW * nbd * 4, 128);
   P.sm_wr = static_cast<int>(o);
   o = ds_align(o + static_cast<size_t>(wr_rows) * c.d * 4, 128);
+  P.sm_shdn = static_cast<int>(o);
+  o = ds_align(o + 2 * static_cast<size_t>(P.dn_stride), 128);
   P.sm_x = static_cast<int>(o);
   const size_t fixed = o;
+  // the staging area: raw x for the router, then the quantised h rows of a
+  // round of down stages (all rows if they fit in 48 KB, else 48 KB worth,
+  // at least T rows); at least three ring slots
   const size_t xs_bytes = a.route ? static_cast<size_t>(T) * c.d * 2 : 0;
   const size_t hq_row = static_cast<size_t>(kQW) * nbf * 4;
-  // rings: at least two gate/up and two down slots; the staging area takes
-  // all h rows if that leaves room, else as many as fit (at least T)
-  const long long min_rings = 2LL * P.gu_slot + 2LL * P.dn_slot;
-  long long avail_x = static_cast<long long>(kDsSmemMax) - static_cast<long long>(fixed) - min_rings;
-  if (avail_x < static_cast<long long>(xs_bytes) || avail_x < static_cast<long long>(T * hq_row))
-    return cudaErrorNotSupported;
-  const size_t want_x = (xs_bytes > n_rows * hq_row) ? xs_bytes : n_rows * hq_row;
-  const size_t x_bytes = ds_align(want_x < static_cast<size_t>(avail_x) ? want_x : static_cast<size_t>(avail_x), 128);
+  size_t hq_bytes = static_cast<size_t>(n_rows) * hq_row;
+  const size_t hq_cap = 48 * 1024 > T * hq_row ? 48 * 1024 : T * hq_row;
+  if (hq_bytes > hq_cap) hq_bytes = hq_cap;
+  const size_t x_bytes = ds_align(xs_bytes > hq_bytes ? xs_bytes : hq_bytes, 128);
   P.hq_rows = static_cast<int>(x_bytes / hq_row);
   if (P.hq_rows > n_rows) P.hq_rows = n_rows;
   o = ds_align(fixed + x_bytes, 128);
-  // ring slots: all of a layer's gate/up stages if they fit, then down
   const long long rem = static_cast<long long>(kDsSmemMax) - static_cast<long long>(o);
-  const int nu_max = np < c.E ? np : c.E;
-  const int want_gu = 2 * ((nu_max * nbf + G - 1) / G + (nbf + G - 1) / G);
-  const int want_dn = nu_max + 1;
-  int n_dn = 2;
-  int n_gu = static_cast<int>((rem - static_cast<long long>(n_dn) * P.dn_slot) / P.gu_slot);
-  if (n_gu > kDsNGU) n_gu = kDsNGU;
-  if (n_gu > want_gu && want_gu >= 2) n_gu = want_gu;
-  if (n_gu < 2) return cudaErrorNotSupported;
-  n_dn = static_cast<int>((rem - static_cast<long long>(n_gu) * P.gu_slot) / P.dn_slot);
-  if (n_dn > kDsNDN) n_dn = kDsNDN;
-  if (n_dn > want_dn) n_dn = want_dn;
-  if (n_dn < 2) n_dn = 2;
-  P.n_gu = n_gu;
-  P.n_dn = n_dn;
-  P.sm_gu = static_cast<int>(o);
-  o += static_cast<size_t>(n_gu) * P.gu_slot;
-  P.sm_dn = static_cast<int>(o);
-  o += static_cast<size_t>(n_dn) * P.dn_slot;
+  int n_ring = static_cast<int>(rem / P.slot_bytes);
+  if (n_ring > kDsNS) n_ring = kDsNS;
+  if (n_ring < 3) return cudaErrorNotSupported;
+  P.n_ring = n_ring;
+  P.sm_ring = static_cast<int>(o);
+  o += static_cast<size_t>(n_ring) * P.slot_bytes;
   if (o > static_cast<size_t>(kDsSmemMax)) return cudaErrorNotSupported;
 
+  if (getenv("MOE_DEBUG") != nullptr)
+    fprintf(stderr,
+            "decode_stack: bits=%d T=%d L=%d route=%d G=%d smem=%zu n_ring=%d slot=%d gpd=%d dn_stride=%d "
+            "hq_rows=%d rpc=%d gran=%d coop_pdl=%d\n",
+            c.bits, T, a.L, a.route ? 1 : 0, G, o, P.n_ring, P.slot_bytes, P.gpd, P.dn_stride, P.hq_rows, P.rpc,
+            P.gran, ctx.coop_pdl ? 1 : 0);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G);
   cfg.blockDim = dim3((CW + 1) * 32);

@@ -347,6 +347,7 @@ moe_status moe_check_device_status(moe_ctx* ctx, moe_stream stream) {
       cudaStreamSynchronize(s) != cudaSuccess)
     return MOE_ECUDA;
   if (h[0] == 0) return MOE_OK;
+  ctx->c.last_detail = h[1];
   // clear the status word, and move the decode kernel's tag counter past any
   // tag an interrupted launch may have written
   if (cudaMemsetAsync(ctx->c.d_status, 0, 64, s) != cudaSuccess || decode_skip_tags(s) != cudaSuccess ||
@@ -354,6 +355,8 @@ moe_status moe_check_device_status(moe_ctx* ctx, moe_stream stream) {
     return MOE_ECUDA;
   return h[0] == kDevTimeout ? MOE_ETIMEOUT : MOE_EDEVICE;
 }
+
+int moe_last_device_error_detail(const moe_ctx* ctx) { return ctx == nullptr ? 0 : ctx->c.last_detail; }
 
 moe_status moe_trace_fetch(moe_ctx* ctx, unsigned long long* host, int n, moe_stream stream) {
   if (ctx == nullptr || host == nullptr || n < 0) return MOE_EINVAL;

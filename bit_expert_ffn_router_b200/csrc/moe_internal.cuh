@@ -31,7 +31,8 @@ struct Ctx {
   unsigned long long timeout_ns = 200ull * 1000 * 1000;  // limit of every device-side wait
   unsigned long long* d_trace = nullptr;  // phase timestamps (MOE_TRACE), kTraceSlots per CTA
   void* static_scratch = nullptr;  // device address of the static scratch (first static call)
-  bool coop_pdl = false;           // a cooperative launch also takes programmatic serialization
+  bool coop_pdl = false;
+  int last_detail = 0;             // detail word of the last device error moe_check_device_status read           // a cooperative launch also takes programmatic serialization
 };
 constexpr int kTraceSlots = 32;
 constexpr int kTraceCtas = 1024;

@@ -81,6 +81,7 @@ _SIGS = {
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_last_cuda_error": (ctypes.c_char_p, []),
     "moe_check_device_status": (_I, [_P, _S]),
+    "moe_last_device_error_detail": (_I, [_P]),
     "moe_trace_fetch": (_I, [_P, ctypes.c_void_p, _I, _S]),
     "moe_expert_layout_get": (_I, [ctypes.POINTER(_Cfg), ctypes.POINTER(_Layout)]),
     "moe_workspace_bytes": (_Z, [ctypes.POINTER(_Cfg), _I]),
@@ -278,8 +279,16 @@ class Context:
             "n_uniq": view(g.n_uniq, 1, torch.int32),
         }
 
+    def prepare_stack_forward(self, cfg, L, T, w_router, slot_of, n_slots, pool, stride, shared, ws,
+                              stream=None) -> "PreparedStack":
+        """moe_stack_forward with every argument but x, the bias and y marshalled once (for launch loops)."""
+        return PreparedStack(self, cfg, L, T, w_router, slot_of, n_slots, pool, stride, shared, ws, stream)
+
     def check_device_status(self, stream=None) -> int:
         return self.lib.moe_check_device_status(self.h, _stream(stream))
+
+    def last_device_error_detail(self) -> int:
+        return self.lib.moe_last_device_error_detail(self.h)
 
     def trace_fetch(self, n_ctas: int, stream=None):
         """Phase timestamps of the last decode-layer launches (MOE_TRACE set at creation)."""
@@ -310,6 +319,29 @@ class PreparedLayer:
 
     def __call__(self, x, y) -> None:
         _check(self.status(x, y), "moe_layer_forward")
+
+
+class PreparedStack:
+    """A moe_stack_forward call whose fixed arguments (configuration, routers,
+    slot table, pool, shared experts, workspace, stream) are converted to
+    ctypes values once; each call marshals only x, the bias and y."""
+
+    def __init__(self, ctx, cfg, L, T, w_router, slot_of, n_slots, pool, stride, shared, ws, stream=None):
+        self._fn = ctx.lib.moe_stack_forward
+        self._cfg = cfg.c()
+        self._keep = (ctx, w_router, slot_of, pool, shared, ws)
+        self._head = (ctx.h, ctypes.byref(self._cfg), L)
+        self._T = T
+        self._mid = (_ptr(w_router),)
+        self._tail = (_ptr(slot_of), n_slots, _ptr(pool), stride, _ptr(shared), _ptr(ws),
+                      ws.numel() * ws.element_size())
+        self._stream = _stream(stream)
+
+    def status(self, x, bias, y) -> int:
+        return self._fn(*self._head, _ptr(x), self._T, *self._mid, _ptr(bias), *self._tail, _ptr(y), self._stream)
+
+    def __call__(self, x, bias, y) -> None:
+        _check(self.status(x, bias, y), "moe_stack_forward")
 
 
 # ------------------------------------------------------------------ buffers

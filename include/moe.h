@@ -148,6 +148,11 @@ MOE_API const char* moe_last_cuda_error(void);
  * MOE_ETIMEOUT (a bounded wait ran out). */
 MOE_API moe_status moe_check_device_status(moe_ctx* ctx, moe_stream stream);
 
+/* Diagnostics: the detail word a kernel recorded with the last device error
+ * that moe_check_device_status returned (for MOE_ETIMEOUT, the wait that gave
+ * up; for MOE_EDEVICE, the pair or expert index), 0 if none. */
+MOE_API int moe_last_device_error_detail(const moe_ctx* ctx);
+
 /* Diagnostics: when the environment variable MOE_TRACE is set at context
  * creation, the decode-layer kernel records the global-timer value (ns) at
  * its phase boundaries, 32 slots per CTA. This copies up to n values (CTA
