@@ -42,7 +42,7 @@ namespace moe {
 
 __host__ __device__ constexpr int ds_consumer_warps(int bits) { return bits == 2 ? 15 : 11; }
 constexpr int kDsNS = 12;       // weight ring slots (at most)
-constexpr int kDsNHS = 4;       // h staging slots of the gate/up epilogue
+constexpr int kDsMaxBlk = 40;   // gate/up channel blocks of one CTA in one layer (at most)
 constexpr int kDsCps = 16;      // gate/up channels per ring stage
 constexpr int kQW = 18;         // words per quantised 32-value block: 16 int16 pairs, scale, sum
 constexpr int kDsMaxCtas = 256;  // grid size limit (done words per layer parity)
@@ -53,6 +53,33 @@ constexpr int kDsPollNs = 64;      // back-off between polls of words that were 
 // the number of layers; tags of a launch are base + 1 .. base + L.
 __device__ unsigned int g_ds_epoch;
 __device__ unsigned int g_ds_exit;
+// Completion counters of the three exchanges of a layer (logits, h, layer
+// output), one per 128-byte line: every CTA adds 1 per layer once its part
+// is written, so after layer l of a launch with tag base `base` each holds
+// (base + l + 1) * G (mod 2^32). They advance in step with the tag counter.
+constexpr int kCntLogits = 0, kCntH = 32, kCntOut = 64;
+__device__ unsigned int g_ds_cnt[96];
+
+// Division by a runtime constant with one wide multiply: n / d for n < 2^31
+// and n < 2^32 / d, with m = floor(2^32 / d) + 1 (the remainder term stays
+// below one step of n / d in that range).
+struct FastDiv {
+  uint32_t d;
+  unsigned long long m;
+};
+
+__host__ __device__ inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  f.m = 0x100000000ull / d + 1;
+  return f;
+}
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  return static_cast<uint32_t>((static_cast<unsigned long long>(n) * f.m) >> 32);
+}
+
+__device__ __forceinline__ uint32_t fmod_(uint32_t n, const FastDiv& f) { return n - fdiv(n, f) * f.d; }
 
 // Offsets (bytes) of the arrays of one layer's routing record.
 struct RecOff {
@@ -79,18 +106,21 @@ struct DSParams {
   unsigned long long* logits_ll;  // [kDsLogitCopies, T, E]
   unsigned long long* h_ll;       // [n_rows, f/32, kQW]
   unsigned long long* y_ll;       // [2, T, d/2]
-  unsigned long long* done_ll;    // [2, kDsMaxCtas]
   int* status;
   unsigned long long timeout_ns;
   unsigned long long* trace;
   // geometry (host computed)
   int gu_lpr, dn_lpr, gran, n_units;
+  int gu_lsh, dn_lsh;           // log2 of gu_lpr, dn_lpr (both powers of two)
+  FastDiv fd_nb, fd_nbf, fd_ring, fd_gpd;  // d / 32, f / 32, ring slots, down stages per slot
+  FastDiv fd_hrow, fd_hp;  // 16-byte units of a quantised h row; rpc / 2
   int gu_row, gu_sc, dn_row, dn_sc;  // bytes per row: codes, scales
   int rpc;                      // output rows per CTA (at most)
   int n_ring, slot_bytes;       // weight ring: slots and bytes per slot
   int dn_stride, gpd;           // bytes per down stage, down stages per ring slot
   int hq_rows;
   int sm_wr, sm_x, sm_xq, sm_hs, sm_zs, sm_route, sm_xres, sm_ring, sm_shdn;
+  int max_blk;                  // gate/up blocks of one CTA in one layer (h staging slots)
 };
 
 struct DSShared {
@@ -100,9 +130,20 @@ struct DSShared {
   int abort_flag;
   unsigned base_tag;
   int n_uniq;
-  int hs_done[kDsNHS];  // channel tasks finished for the block staged in the slot
-  int hs_gen[kDsNHS];   // epilogues finished in the slot
+  int route_ok;  // this layer's routing in shared memory is complete (read behind route_bar)
+  // A copy of the launch parameters for the out-of-line helpers: they read
+  // it from shared memory instead of from a per-thread stack copy.
+  DSParams prm;
 };
+
+// Start of part b of n items split into G near-equal parts (n * G < 2^31,
+// which the launch checks).
+__device__ __forceinline__ int split_at(int n, int b, int G) {
+  return static_cast<int>(static_cast<unsigned>(n) * static_cast<unsigned>(b) / static_cast<unsigned>(G));
+}
+
+// The kernel's dynamic shared memory.
+extern __shared__ __align__(128) char ds_smem[];
 
 struct DSRoute {
   int32_t* idx;        // [np]  top-k of token t at t*k + j
@@ -181,6 +222,36 @@ __device__ __forceinline__ bool ds_aborted(const DSShared* S) {
   return *reinterpret_cast<const volatile int*>(&S->abort_flag) != 0;
 }
 
+// Counts this CTA's part of an exchange as written (the tagged words it
+// stored before the last CTA barrier); relaxed, fire and forget.
+__device__ __forceinline__ void cnt_add(int which) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(&g_ds_cnt[which]) : "memory");
+}
+
+// Polls an exchange counter (one thread) until it reaches `target`
+// (wrap-safe); false on timeout or abort.
+__device__ __forceinline__ bool cnt_wait(int which, unsigned target, DSShared* S, int* status, int where,
+                                         uint64_t deadline) {
+  while (true) {
+    unsigned v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(&g_ds_cnt[which]) : "memory");
+    if (static_cast<int>(v - target) >= 0) return true;
+    if (*reinterpret_cast<volatile int*>(&S->abort_flag) != 0) return false;
+    if (global_timer_ns() > deadline) {
+      report(status, kDevTimeout, where);
+      *reinterpret_cast<volatile int*>(&S->abort_flag) = 1;
+      return false;
+    }
+    __nanosleep(32);
+  }
+}
+
+// The same, agreed by the whole warp (call with the warp converged): code
+// that follows it may use full-warp collectives.
+__device__ __forceinline__ bool ds_aborted_warp(const DSShared* S) {
+  return __any_sync(0xffffffffu, ds_aborted(S));
+}
+
 // Warp-wide bounded mbarrier wait by lane 0 (false on timeout or abort).
 __device__ __forceinline__ bool ds_wait_warp(uint64_t* b, uint32_t parity, const DSShared* S, uint64_t deadline) {
   int ok = 1;
@@ -226,7 +297,7 @@ __device__ __forceinline__ void load_xq(const int* __restrict__ vec, int nb, int
 // c) and returns the word this lane owns (lanes 0..17), in the layout above.
 __device__ __forceinline__ uint32_t quant_block_warp(float v, int lane) {
   const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v))));
-  const float inv = m > 0.f ? 32767.f / m : 0.f;
+  const float inv = m > 0.f ? __fdividef(32767.f, m) : 0.f;
   constexpr float kMagic = 12582912.f;  // 1.5 * 2^23: rint(v * inv) in the low bits
   const int r = __float_as_int(fmaf(v, inv, kMagic));
   const int sum = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(r - 0x4B400000)));
@@ -247,12 +318,12 @@ __device__ __forceinline__ uint32_t quant_block_warp(float v, int lane) {
 // tag was not there yet, so a batch costs about one L2 round trip. Writes the
 // raw bf16 rows (xs, for the router), the quantised gate/up operand (xq) and
 // this CTA's residual rows (xres).
-constexpr int kXB = 4;
+constexpr int kXB = 1;
 
-template <int BITS>
+template <int BITS, int GBPL>
 __device__ void ds_read_x(const DSParams& P, int l, uint32_t tag, uint16_t* xs, int* xq, float* xres, int r0,
                           int r1, DSShared* S, uint64_t deadline, int CT) {
-  const int nb = P.d / kBlock, bpl = nb / P.gu_lpr;
+  const int nb = P.d / kBlock;
   const int words = kQW * nb;
   const int jobs = P.T * nb * 4;  // four threads per 32-value block
   const int tid = threadIdx.x;
@@ -267,9 +338,10 @@ __device__ void ds_read_x(const DSParams& P, int l, uint32_t tag, uint16_t* xs, 
       for (int i = 0; i < kXB; ++i) {
         const int j = tid + (k0 + i) * CT;
         const int job = j < jobs ? j >> 2 : 0, q = j & 3;
-        const int t = job / nb, blk = job % nb;
-        const uint4 raw =
-            __ldcg(reinterpret_cast<const uint4*>(P.x + static_cast<size_t>(t) * P.d + blk * kBlock + 8 * q));
+        const int t = fdiv(job, P.fd_nb), blk = job - t * nb;
+        const uint4 raw = j < jobs ? __ldcg(reinterpret_cast<const uint4*>(P.x + static_cast<size_t>(t) * P.d +
+                                                                           blk * kBlock + 8 * q))
+                                   : make_uint4(0u, 0u, 0u, 0u);
         w4[i][0] = raw.x;
         w4[i][1] = raw.y;
         w4[i][2] = raw.z;
@@ -282,17 +354,17 @@ __device__ void ds_read_x(const DSParams& P, int l, uint32_t tag, uint16_t* xs, 
       for (int i = 0; i < kXB; ++i) {
         const int j = tid + (k0 + i) * CT;
         const int job = j < jobs ? j >> 2 : 0, q = j & 3;
-        const int t = job / nb, blk = job % nb;
+        const int t = fdiv(job, P.fd_nb), blk = job - t * nb;
         src[i] = yl + static_cast<size_t>(t) * (P.d / 2) + blk * 16 + 4 * q;
-        ld_ll2(src[i], v[i][0], v[i][1]);
-        ld_ll2(src[i] + 2, v[i][2], v[i][3]);
+        if (j < jobs) {
+          ld_ll2(src[i], v[i][0], v[i][1]);
+          ld_ll2(src[i] + 2, v[i][2], v[i][3]);
+        } else {  // no load: a slot past the end counts as present
+          v[i][0] = v[i][1] = v[i][2] = v[i][3] = ll_word(0u, tag - 1);
+        }
       }
-      // every CTA's done word rides along in the first batch
-      const unsigned long long* dp = P.done_ll + static_cast<size_t>((l - 1) & 1) * kDsMaxCtas + tid;
-      const bool has_done = k0 == 0 && tid < static_cast<int>(gridDim.x);
-      unsigned long long dw = has_done ? ld_ll(dp) : ll_word(0u, tag - 1);
       while (true) {
-        bool all = tag_ok(dw, tag - 1);
+        bool all = true;
 #pragma unroll
         for (int i = 0; i < kXB; ++i)
 #pragma unroll
@@ -303,7 +375,6 @@ __device__ void ds_read_x(const DSParams& P, int l, uint32_t tag, uint16_t* xs, 
           break;
         }
         __nanosleep(kDsPollNs);
-        if (!tag_ok(dw, tag - 1)) dw = ld_ll(dp);
 #pragma unroll
         for (int i = 0; i < kXB; ++i)
 #pragma unroll
@@ -321,7 +392,7 @@ __device__ void ds_read_x(const DSParams& P, int l, uint32_t tag, uint16_t* xs, 
       const int j = tid + (k0 + i) * CT;
       const bool live = j < jobs;
       const int job = live ? j >> 2 : 0, q = j & 3;
-      const int t = job / nb, blk = job % nb;
+      const int t = fdiv(job, P.fd_nb), blk = job - t * nb;
       float v8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -337,8 +408,8 @@ __device__ void ds_read_x(const DSParams& P, int l, uint32_t tag, uint16_t* xs, 
         for (int e = 0; e < 8; ++e)
           if (c0 + e >= r0 && c0 + e < r1) xres[t * P.rpc + (c0 + e - r0)] = v8[e];
       }
-      const int gl = blk / bpl, bb = blk % bpl;
-      quant_quad_c2(v8, xq + t * words, nb, bb * P.gu_lpr + gl, q, live);
+      const int gl = blk / GBPL, bb = blk - gl * GBPL;
+      quant_quad_c2(v8, xq + t * words, nb, (bb << P.gu_lsh) + gl, q, live);
     }
   }
 }
@@ -360,143 +431,147 @@ __device__ __forceinline__ float ds_key_value(uint32_t k) {
   return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
 }
 
-// Warp t: polls token t's E <= 512 logit words (16 per lane), selects its k
-// experts and gates into R. Fast path: the k-th largest of the 32 lane maxima
-// bounds the k-th largest key from below; when at most 32 keys reach it they
-// are ranked against each other in one pass, otherwise k rounds of warp
-// maximum select them. The publishing CTA also writes the plain logits.
-__device__ void ds_topk(const DSParams& P, const DSRoute& R, int t, uint32_t tag, float* pub_logits,
-                        unsigned long long* scratch, DSShared* S, uint64_t deadline) {
-  constexpr int VPL = 16;
+constexpr int kDsMaxE = 512;  // experts a decode launch supports
+
+// Warp t: polls token t's E <= 512 logit words (all of a lane's 16 at once),
+// turns them into order keys held in registers, selects its k experts and
+// gates into R. Selection: k rounds of a warp maximum over the keys (ties go
+// to the lower expert index through a second, minimum reduction over the
+// indices that hold the maximum); lane j keeps the j-th pick. The publishing
+// CTA also writes the plain logits.
+__device__ __noinline__ void ds_topk(const DSParams& P, int t, uint32_t tag, float* pub_logits, uint32_t* kr,
+                                     DSShared* S, uint64_t deadline, unsigned long long* td) {
+  const DSRoute R = ds_route(ds_smem + P.sm_route, P.T * P.k);
+  constexpr int KPL = kDsMaxE / 32;  // keys a lane holds
   const int lane = threadIdx.x & 31;
   const unsigned long long* row =
       P.logits_ll + (static_cast<size_t>(blockIdx.x % kDsLogitCopies) * P.T + t) * P.E;
-  unsigned long long w[VPL];
+  unsigned long long w[KPL];
 #pragma unroll
-  for (int v = 0; v < VPL; ++v) w[v] = ld_ll(row + min(v * 32 + lane, P.E - 1));
+  for (int v = 0; v < KPL; ++v) w[v] = ll_word(0u, v * 32 + lane < P.E ? tag - 1 : tag);  // absent words count as there
   bool ok = true;
-  while (true) {  // re-poll only the words not there yet, all at once
+#pragma unroll 1
+  for (int pass = 0;; ++pass) {  // (re-)load only the words not there yet, all at once
+    if (pass > 0) {
+      if (ds_aborted(S) || global_timer_ns() > deadline) {
+        ok = false;
+        break;
+      }
+      __nanosleep(kDsPollNs);
+    }
+#pragma unroll
+    for (int v = 0; v < KPL; ++v)
+      if (!tag_ok(w[v], tag)) w[v] = ld_ll(row + v * 32 + lane);
     bool all = true;
 #pragma unroll
-    for (int v = 0; v < VPL; ++v) all = all && tag_ok(w[v], tag);
+    for (int v = 0; v < KPL; ++v) all = all && tag_ok(w[v], tag);
     if (all) break;
-    if (ds_aborted(S) || global_timer_ns() > deadline) {
-      ok = false;
-      break;
-    }
-    __nanosleep(kDsPollNs);
-#pragma unroll
-    for (int v = 0; v < VPL; ++v)
-      if (!tag_ok(w[v], tag)) w[v] = ld_ll(row + min(v * 32 + lane, P.E - 1));
   }
   if (!__all_sync(0xffffffffu, ok)) {
     if (lane == 0 && !ds_aborted(S)) ds_abort(S, P.status, 22);
     return;
   }
-  float lv[VPL];
+  uint32_t kv[KPL];  // order keys; 0 = absent (e >= E) or taken
 #pragma unroll
-  for (int v = 0; v < VPL; ++v) lv[v] = __uint_as_float(static_cast<uint32_t>(w[v]));
-  if (pub_logits != nullptr) {
-#pragma unroll
-    for (int v = 0; v < VPL; ++v)
-      if (v * 32 + lane < P.E) pub_logits[static_cast<size_t>(t) * P.E + v * 32 + lane] = lv[v];
+  for (int v = 0; v < KPL; ++v) {
+    const int e = v * 32 + lane;
+    const float lv = __uint_as_float(static_cast<uint32_t>(w[v]));
+    kv[v] = e < P.E ? ds_order_key(lv) : 0u;
+    if (e < P.E) kr[e] = kv[v];
   }
-  uint32_t key[VPL];
-#pragma unroll
-  for (int v = 0; v < VPL; ++v) key[v] = v * 32 + lane < P.E ? ds_order_key(lv[v]) : 0u;
+  if (pub_logits != nullptr) {  // the publishing CTA: the plain logits, from L2 again
+#pragma unroll 1
+    for (int e = lane; e < P.E; e += 32)
+      pub_logits[static_cast<size_t>(t) * P.E + e] = __uint_as_float(static_cast<uint32_t>(ld_ll(row + e)));
+  }
+  if (td && lane == 0) td[29] = global_timer_ns();
   uint32_t mine_key = 0u;
   int mine_e = 0;
-  uint32_t lmax = 0u;
-#pragma unroll
-  for (int v = 0; v < VPL; ++v) lmax = max(lmax, key[v]);
-  uint32_t srt = lmax;  // bitonic sort of the lane maxima, descending
-#pragma unroll
-  for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      const uint32_t o = __shfl_xor_sync(0xffffffffu, srt, stride);
-      const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0 || size == 32);
-      srt = keep_max ? max(srt, o) : min(srt, o);
-    }
-  }
-  const uint32_t Lk = __shfl_sync(0xffffffffu, srt, P.k - 1);
-  int cnt = 0;
-#pragma unroll
-  for (int v = 0; v < VPL; ++v) cnt += (Lk > 0u && key[v] >= Lk) ? 1 : 0;
-  const int C = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(cnt)));
-  if (Lk > 0u && C <= 32) {
-    int pos = cnt;  // exclusive prefix of cnt over the lanes
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, pos, o);
-      if (lane >= o) pos += n;
-    }
-    pos -= cnt;
-#pragma unroll
-    for (int v = 0; v < VPL; ++v)
-      if (Lk > 0u && key[v] >= Lk)  // larger word = larger key, then lower expert index
-        scratch[pos++] = (static_cast<unsigned long long>(key[v]) << 32) |
-                         (0xffffffffu - static_cast<uint32_t>(v * 32 + lane));
-    __syncwarp();
-    const unsigned long long mine = lane < C ? scratch[lane] : 0ull;
-    int rank = 0;
-    for (int j = 0; j < C; ++j) rank += scratch[j] > mine ? 1 : 0;
-    __syncwarp();
-    if (lane < C && rank < P.k) scratch[rank] = mine;
-    __syncwarp();
-    if (lane < P.k) {
-      const unsigned long long sel = scratch[lane];
-      mine_key = static_cast<uint32_t>(sel >> 32);
-      mine_e = static_cast<int>(0xffffffffu - static_cast<uint32_t>(sel & 0xffffffffu));
-    }
-    __syncwarp();
-  } else {
 #pragma unroll 1
-    for (int j = 0; j < P.k; ++j) {
-      uint32_t lm = 0u;
+  for (int j = 0; j < P.k; ++j) {
+    // lane maximum and the lowest register index holding the warp maximum,
+    // both as trees (short dependency chains)
+    uint32_t t[KPL];
 #pragma unroll
-      for (int v = 0; v < VPL; ++v) lm = max(lm, key[v]);
-      const uint32_t M = __reduce_max_sync(0xffffffffu, lm);
-      uint32_t my = 0xffffffffu;
+    for (int i = 0; i < KPL; ++i) t[i] = kv[i];
 #pragma unroll
-      for (int v = VPL - 1; v >= 0; --v)
-        if (key[v] == M) my = static_cast<uint32_t>(v * 32 + lane);
-      const int e = static_cast<int>(__reduce_min_sync(0xffffffffu, lm == M ? my : 0xffffffffu));
+    for (int h = KPL / 2; h > 0; h >>= 1)
 #pragma unroll
-      for (int v = 0; v < VPL; ++v) key[v] = (v * 32 + lane == e) ? 0u : key[v];
-      if (lane == j) {
-        mine_key = M;
-        mine_e = e;
-      }
+      for (int i = 0; i < h; ++i) t[i] = max(t[i], t[i + h]);
+    const uint32_t M = __reduce_max_sync(0xffffffffu, t[0]);
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) t[i] = kv[i] == M ? static_cast<uint32_t>(i) : 0xffffu;
+#pragma unroll
+    for (int h = KPL / 2; h > 0; h >>= 1)
+#pragma unroll
+      for (int i = 0; i < h; ++i) t[i] = min(t[i], t[i + h]);
+    const unsigned le = t[0] < 0xffffu ? static_cast<unsigned>(lane + 32 * static_cast<int>(t[0])) : 0x7fffffffu;
+    const int e = static_cast<int>(__reduce_min_sync(0xffffffffu, le));
+#pragma unroll
+    for (int i = 0; i < KPL; ++i)
+      if (lane + 32 * i == e) kv[i] = 0u;
+    if (lane == j) {
+      mine_key = M;
+      mine_e = e;
     }
   }
+  if (td && lane == 0) td[30] = global_timer_ns();
   const bool sel = lane < P.k;
   const float lj = sel ? ds_key_value(mine_key) : 0.f;
   const float l0 = __shfl_sync(0xffffffffu, lj, 0);
   const float ex = sel ? expf(lj - l0) : 0.f;
-  float denom;
-  if (P.renorm) {
-    denom = warp_sum(ex);
-  } else {
-    float s = 0.f;  // full-softmax denominator over every logit of the row
-#pragma unroll
-    for (int v = 0; v < VPL; ++v)
-      if (v * 32 + lane < P.E) s += expf(lv[v] - l0);
-    denom = warp_sum(s);
+  float sum = ex;
+  if (!P.renorm) {
+    // full-softmax denominator over the whole row (its keys in kr)
+    sum = 0.f;
+#pragma unroll 1
+    for (int e = lane; e < P.E; e += 32) sum += expf(ds_key_value(kr[e]) - l0);  // NaN logits make the sum NaN
   }
+  const float denom = warp_sum(sum);
   if (sel) {
     R.idx[t * P.k + lane] = mine_e;
     R.gate[t * P.k + lane] = ex / denom;
+  }
+  if (P.T == 1) {
+    // one token: its k experts are distinct, so the grouping is their order
+    // by expert index, found here by ranks instead of a CTA-wide sort
+    int pos = 0;
+#pragma unroll 4
+    for (int j = 0; j < 32; ++j) {
+      const int ej = __shfl_sync(0xffffffffu, mine_e, j);
+      pos += (j < P.k && ej < mine_e) ? 1 : 0;
+    }
+    if (sel) {
+      int slot = R.slot_s[min(max(mine_e, 0), P.E - 1)];
+      if (slot < 0 || slot >= P.n_slots) {
+        report(P.status, kDevBadSlot, mine_e);
+        slot = 0;
+      }
+      R.sorted_e[pos] = mine_e;
+      R.pair_token[pos] = 0;
+      R.pair_gate[pos] = ex / denom;
+      R.pair_pos[lane] = pos;
+      R.uniq_e[pos] = mine_e;
+      R.uniq_slot[pos] = slot;
+      R.uniq_off[pos] = pos;
+    }
+    if (lane == 0) {
+      R.uniq_off[P.k] = P.k;
+      S->n_uniq = P.k;
+    }
   }
 }
 
 // Stable sort of the T*k pairs by expert in shared memory, the unique
 // experts and their slots. Every consumer thread takes part.
-__device__ void ds_group(const DSParams& P, const DSRoute& R, DSShared* S, int np, int CT) {
+__device__ __noinline__ void ds_group(const DSParams& P, DSShared* S, int np, int CT) {
+  const DSRoute R = ds_route(ds_smem + P.sm_route, np);
   const int tid = threadIdx.x;
+#pragma unroll 1
   for (int p = tid; p < np; p += CT) {
     const int e = min(max(R.idx[p], 0), P.E - 1);
     int pos = 0;
+#pragma unroll 1
     for (int q = 0; q < np; ++q) {
       const int eq = min(max(R.idx[q], 0), P.E - 1);
       pos += (eq < e) || (eq == e && q < p);
@@ -509,6 +584,7 @@ __device__ void ds_group(const DSParams& P, const DSRoute& R, DSShared* S, int n
   named_sync(1, CT);
   if (tid < 32) {
     int base = 0;
+#pragma unroll 1
     for (int c = 0; c < np; c += 32) {
       const int i = c + tid;
       const bool first = i < np && (i == 0 || R.sorted_e[i - 1] != R.sorted_e[i]);
@@ -536,7 +612,8 @@ __device__ void ds_group(const DSParams& P, const DSRoute& R, DSShared* S, int n
 }
 
 // Writes layer l's routing record (the publishing CTA only).
-__device__ void ds_publish(const DSParams& P, const DSRoute& R, int l, int np, int nu, int CT) {
+__device__ __noinline__ void ds_publish(const DSParams& P, int l, int np, int nu, int CT) {
+  const DSRoute R = ds_route(ds_smem + P.sm_route, np);
   char* rec = P.rec + static_cast<size_t>(l) * P.rec_bytes;
   int32_t* idx = reinterpret_cast<int32_t*>(rec + P.ro.idx);
   float* gate = reinterpret_cast<float*>(rec + P.ro.gate);
@@ -551,6 +628,7 @@ __device__ void ds_publish(const DSParams& P, const DSRoute& R, int l, int np, i
   int32_t* ec = reinterpret_cast<int32_t*>(rec + P.ro.expert_count);
   int32_t* eo = reinterpret_cast<int32_t*>(rec + P.ro.expert_offset);
   const int tid = threadIdx.x;
+#pragma unroll 1
   for (int q = tid; q < np; q += CT) {
     const int pos = R.pair_pos[q];
     const int e = min(max(R.idx[q], 0), P.E - 1);
@@ -564,6 +642,7 @@ __device__ void ds_publish(const DSParams& P, const DSRoute& R, int l, int np, i
     pg[pos] = R.gate[q];
     ps[pos] = slot;
   }
+#pragma unroll 1
   for (int u = tid; u < nu; u += CT) {
     ue[u] = R.uniq_e[u];
     us[u] = R.uniq_slot[u];
@@ -573,6 +652,7 @@ __device__ void ds_publish(const DSParams& P, const DSRoute& R, int l, int np, i
     uo[nu] = np;
     *reinterpret_cast<int32_t*>(rec + P.ro.n_uniq) = nu;
   }
+#pragma unroll 1
   for (int e = tid; e < P.E; e += CT) {  // counts by binary search in the sorted experts
     int lo = 0, hi = np;
     while (lo < hi) {
@@ -602,7 +682,12 @@ __device__ void ds_router(const DSParams& P, int l, uint32_t tag, const float* w
   const float* bias = P.bias != nullptr ? P.bias + static_cast<size_t>(l) * P.T * P.E : nullptr;
 #pragma unroll 1
   for (int task = warp; task < nr * P.T; task += CW) {
-    const int e = e0 + task % nr, t = task / nr;
+    int t = 0, rem = task;  // task -> (token, row) without a division: at most T rows of nr
+    while (rem >= nr) {
+      rem -= nr;
+      ++t;
+    }
+    const int e = e0 + rem;
     const float4* w4 = reinterpret_cast<const float4*>(wrs + static_cast<size_t>(e - e0) * P.d);
     const uint2* x2 = reinterpret_cast<const uint2*>(xs + static_cast<size_t>(t) * P.d);
     const size_t o = static_cast<size_t>(t) * P.E + e;
@@ -631,14 +716,14 @@ struct GUBlock {
   int cb;              // channel block inside the expert
 };
 
-__device__ __forceinline__ void gu_block_of(int beta, int nsh, int sb0, int rb0, int nbf, GUBlock& gb) {
+__device__ __forceinline__ void gu_block_of(int beta, int nsh, int sb0, int rb0, const FastDiv& fd_nbf, GUBlock& gb) {
   if (beta < nsh) {
     gb.u = -1;
     gb.cb = sb0 + beta;
   } else {
     const int g = rb0 + beta - nsh;
-    gb.u = g / nbf;
-    gb.cb = g % nbf;
+    gb.u = fdiv(g, fd_nbf);
+    gb.cb = g - gb.u * fd_nbf.d;
   }
 }
 
@@ -657,82 +742,129 @@ __device__ __forceinline__ int h_row_token(const DSRoute& R, int u, int first, i
   return u < 0 ? i : R.pair_token[first + i];
 }
 
-// One gate/up channel task: channel c (of a 32-channel block) for every token
-// of the block's expert, the weights in ring stage `st`; h values -> hs.
-template <int BITS, int BPL>
-__device__ __forceinline__ void gu_task(const DSParams& P, const DSRoute& R, const uint8_t* st, int cl,
-                                        const int* xq, int u, int np, float* hs, int c, int& cur_t,
-                                        XR<BITS>* xr) {
-  const int lane = threadIdx.x & 31;
-  const int lpr = P.gu_lpr, gl = lane % lpr;
+// The gate/up + SwiGLU phase of one layer for one consumer warp: its channel
+// tasks (task j = channel j % 32 of block j / 32; blocks in order: this
+// CTA's shared-expert blocks, then its routed blocks), each for every token
+// of the block's expert, the weights in ring stage seq + j / 16; h -> hs.
+// Out of line on purpose: the loop gets the whole register budget instead of
+// sharing it with the live state of the kernel around it. The launch
+// parameters come from their shared-memory copy and are read into registers
+// once. Returns false when the phase gave up (abort or timeout).
+template <int BITS, int BPL, int CW>
+__device__ __noinline__ bool gu_phase(const DSParams& Q, DSShared* S, int nsh, int sb0, int rb0, int n_blk,
+                                      uint32_t seq, uint64_t deadline, unsigned long long* td) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int d = Q.d, T = Q.T, np = Q.T * Q.k, nb = Q.d / kBlock;
+  const int lpr = Q.gu_lpr, gl = lane & (lpr - 1);
   const bool active = lane < lpr;
-  const int nb = P.d / kBlock;
-  const uint8_t* cg = st + 2 * cl * P.gu_row;
-  const uint16_t* sg = reinterpret_cast<const uint16_t*>(st + 2 * kDsCps * P.gu_row) + 2 * cl * nb;
+  const int gu_row = Q.gu_row, slot_bytes = Q.slot_bytes, n_ring = Q.n_ring;
+  const FastDiv fd_ring = Q.fd_ring, fd_nbf = Q.fd_nbf;
+  int* status = Q.status;
+  const uint8_t* ring = reinterpret_cast<const uint8_t*>(ds_smem + Q.sm_ring);
+  float* hs = reinterpret_cast<float*>(ds_smem + Q.sm_hs);
+  const int* xq = reinterpret_cast<const int*>(ds_smem + Q.sm_xq);
+  const DSRoute R = ds_route(ds_smem + Q.sm_route, np);
+  XR<BITS> xr[BPL];
+  int cur_t = -1;
+  bool ok = true;
+#pragma unroll 1
+  for (int task = warp; task < n_blk * 32; task += CW) {
+    if (ds_aborted_warp(S)) {
+      ok = false;
+      break;
+    }
+    const int beta = task >> 5, c = task & 31;
+    GUBlock gb;
+    gu_block_of(beta, nsh, sb0, rb0, fd_nbf, gb);
+    const uint32_t sq = seq + beta * (32 / kDsCps) + c / kDsCps;
+    const uint32_t sqd = fdiv(sq, fd_ring);
+    const int slot = sq - sqd * n_ring;
+    if (!ds_wait_warp(&S->full[slot], sqd & 1, S, deadline)) {
+      if (lane == 0 && !ds_aborted(S)) ds_abort(S, status, 2);
+      ok = false;
+      break;
+    }
+    const int ti = (task - warp) / CW;  // this warp's task count
+    if (td && lane == 0) {
+      if (task == warp) td[22] = global_timer_ns();  // first stage in
+      if (ti < 16) td[32 + ti] = global_timer_ns();
+    }
+    const uint8_t* st = ring + static_cast<size_t>(slot) * slot_bytes;
+    const int cl = c % kDsCps;
+    const uint8_t* cg = st + 2 * cl * gu_row;
+    const uint16_t* sg = reinterpret_cast<const uint16_t*>(st + 2 * kDsCps * gu_row) + 2 * cl * nb;
+    float* hsl = hs + beta * T * 32;
+    int first, n;
+    expert_h_rows(R, gb.u, np, T, first, n);
+#pragma unroll 1
+    for (int i = 0; i < n; ++i) {
+      const int t = h_row_token(R, gb.u, first, i);
+      if (t != cur_t) {
+        load_xq<BITS, BPL>(xq + t * kQW * nb, nb, lpr, gl, xr);
+        cur_t = t;
+      }
+      float2 v = make_float2(0.f, 0.f);
+      if (active) v = row_dot2<BITS, BPL>(cg, sg, cg + gu_row, sg + nb, d, gl, xr);
+      v = group_sum2(v, lpr);
+      // fast exponential and division: h is requantised to 16 bits for the
+      // down rows, far coarser than their few-ulp error
+      if (lane == 0) hsl[i * 32 + c] = __fdividef(v.x, 1.f + __expf(-v.x)) * v.y;
+    }
+    if (td && lane == 0 && ti < 16) td[48 + ti] = global_timer_ns();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S->empty[slot]);
+  }
+  return ok;
+}
+
+// A gate/up block's 32 channels are in hs: requantise each token's 32
+// values and publish them as tagged words (one warp).
+__device__ __noinline__ void gu_publish(const DSParams& P, int u, int cb, int np, const float* hsl, uint32_t tag) {
+  const DSRoute R = ds_route(ds_smem + P.sm_route, np);
+  const int lane = threadIdx.x & 31;
+  const int nbf = P.f / kBlock;
   int first, n;
   expert_h_rows(R, u, np, P.T, first, n);
 #pragma unroll 1
   for (int i = 0; i < n; ++i) {
-    const int t = h_row_token(R, u, first, i);
-    if (t != cur_t) {
-      load_xq<BITS, BPL>(xq + t * kQW * nb, nb, lpr, gl, xr);
-      cur_t = t;
-    }
-    float2 v = make_float2(0.f, 0.f);
-    if (active) v = row_dot2<BITS, BPL>(cg, sg, cg + P.gu_row, sg + nb, P.d, gl, xr);
-    v = group_sum2(v, lpr);
-    // fast exponential and division: h is requantised to 16 bits for the
-    // down rows, far coarser than their few-ulp error
-    if (lane == 0) hs[i * 32 + c] = __fdividef(v.x, 1.f + __expf(-v.x)) * v.y;
+    const uint32_t wq = quant_block_warp(hsl[i * 32 + lane], lane);
+    if (lane < kQW) st_ll(P.h_ll + (static_cast<size_t>(first + i) * nbf + cb) * kQW + lane, ll_word(wq, tag));
   }
 }
 
 // ------------------------------------------------------------------ down
 // Stages the quantised h rows of DN stages [i0, i1) into hq (every consumer
-// thread takes part), in stage order. A thread loads up to kHB 16-byte units
-// at once and re-polls, together, only the words not there yet.
-constexpr int kHB = 8;
+// thread takes part). The round's rows, in stage order, are the shared
+// expert's T rows (when stage 0 is in the round) followed by the routed rows
+// [uniq_off[ua], uniq_off[ub]), one contiguous range of h. A thread loads up
+// to kHB 16-byte units at once and re-polls, together, only the words that
+// were not there yet.
+constexpr int kHB = 4;
 
-__device__ void ds_stage_h(const DSParams& P, const DSRoute& R, int np, int i0, int i1, bool sh_first, uint32_t tag,
+template <int DBPL>
+__device__ void ds_stage_h(const DSParams& P, const DSRoute& R, int np, int i0, int i1, int sh, uint32_t tag,
                            int* hq, DSShared* S, uint64_t deadline, int CT) {
-  const int nbf = P.f / kBlock, bpl = nbf / P.dn_lpr;
+  const int nbf = P.f / kBlock;
   const int units_per_row = nbf * (kQW / 2);  // 16-byte units
-  // rows of the round: stage order, each stage's rows contiguous in h
-  int n_rows = 0;
-  for (int i = i0; i < i1; ++i) {
-    const int u = (sh_first && i == 0) ? -1 : i - (sh_first ? 1 : 0);
-    int first, n;
-    expert_h_rows(R, u, np, P.T, first, n);
-    n_rows += n;
-  }
+  const FastDiv& fd_row = P.fd_hrow;
+  const int n_sh = (sh && i0 == 0) ? P.T : 0;
+  const int ua = max(i0 - sh, 0), ub = max(i1 - sh, 0);
+  const int rfirst = R.uniq_off[ua];
+  const int n_rows = n_sh + (ub > ua ? R.uniq_off[ub] - rfirst : 0);
   const int units = n_rows * units_per_row;
 #pragma unroll 1
   for (int j0 = threadIdx.x; j0 < units; j0 += kHB * CT) {
     unsigned long long v[kHB][2];
     const unsigned long long* src[kHB];
-    int dst_row[kHB], dst_col[kHB], dst_w[kHB];
 #pragma unroll
     for (int k = 0; k < kHB; ++k) {
       const int j = min(j0 + k * CT, units - 1);
-      const int r = j / units_per_row, rem = j % units_per_row;
-      // row r of the round -> its h row (walk the stages)
-      int base = 0, hrow = 0;
-      for (int i = i0; i < i1; ++i) {
-        const int u = (sh_first && i == 0) ? -1 : i - (sh_first ? 1 : 0);
-        int first, n;
-        expert_h_rows(R, u, np, P.T, first, n);
-        if (r < base + n) {
-          hrow = first + (r - base);
-          break;
-        }
-        base += n;
-      }
+      const int r = fdiv(j, fd_row), rem = j - r * units_per_row;
+      const int hrow = r < n_sh ? np + r : rfirst + (r - n_sh);
       const int blk = rem / (kQW / 2), w2 = rem % (kQW / 2);
       src[k] = P.h_ll + (static_cast<size_t>(hrow) * nbf + blk) * kQW + 2 * w2;
-      dst_row[k] = r;
-      dst_col[k] = (blk % bpl) * P.dn_lpr + blk / bpl;
-      dst_w[k] = 2 * w2;
-      ld_ll2(src[k], v[k][0], v[k][1]);
+      if (j0 + k * CT < units) ld_ll2(src[k], v[k][0], v[k][1]);
+      else v[k][0] = v[k][1] = ll_word(0u, tag);  // past the end: no load
     }
     while (true) {
       bool all = true;
@@ -752,10 +884,13 @@ __device__ void ds_stage_h(const DSParams& P, const DSRoute& R, int np, int i0, 
     }
 #pragma unroll
     for (int k = 0; k < kHB; ++k) {
-      if (j0 + k * CT < units) {
-        int* dst = hq + dst_row[k] * kQW * nbf;
-        dst[dst_w[k] * nbf + dst_col[k]] = static_cast<int>(static_cast<uint32_t>(v[k][0]));
-        dst[(dst_w[k] + 1) * nbf + dst_col[k]] = static_cast<int>(static_cast<uint32_t>(v[k][1]));
+      const int j = j0 + k * CT;
+      if (j < units) {
+        const int r = fdiv(j, fd_row), rem = j - r * units_per_row;
+        const int blk = rem / (kQW / 2), w2 = rem % (kQW / 2);
+        int* dst = hq + r * kQW * nbf + ((blk % DBPL) << P.dn_lsh) + blk / DBPL;
+        dst[(2 * w2) * nbf] = static_cast<int>(static_cast<uint32_t>(v[k][0]));
+        dst[(2 * w2 + 1) * nbf] = static_cast<int>(static_cast<uint32_t>(v[k][1]));
       }
     }
   }
@@ -767,8 +902,8 @@ template <int BITS, int BPL>
 __device__ __forceinline__ void dn_task(const DSParams& P, const DSRoute& R, const uint8_t* st, int u, int np,
                                         const int* hq, int hq_row0, int nrows_out, float* zs) {
   const int lane = threadIdx.x & 31;
-  const int lpr = P.dn_lpr, rpw = 32 / lpr;
-  const int rl = lane / lpr, gl = lane % lpr;
+  const int lpr = P.dn_lpr, rpw = 32 >> P.dn_lsh;
+  const int rl = lane >> P.dn_lsh, gl = lane & (lpr - 1);
   const int nb = P.f / kBlock;
   const uint8_t* codes = st;
   const uint16_t* scales = reinterpret_cast<const uint16_t*>(st + nrows_out * P.dn_row);
@@ -794,17 +929,13 @@ __device__ __forceinline__ void dn_task(const DSParams& P, const DSRoute& R, con
 // channels) and down group (the down rows of up to `gpd` routed experts) of
 // a layer; consumers free a slot with 16 arrivals. Down groups follow the
 // gate/up stages, so they stream in while gate/up is still computing.
-__device__ __forceinline__ bool ring_slot_free(uint64_t* empty, uint32_t seq, int n) {
-  return seq < static_cast<uint32_t>(n) || mbar_test(&empty[seq % n], ((seq / n) - 1) & 1);
-}
-
 __device__ __forceinline__ void mbar_arrive_cnt(uint64_t* b, uint32_t count) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
 }
 
-__device__ __forceinline__ void issue_gu(const DSParams& P, DSShared* S, uint8_t* ring, uint32_t seq,
+__device__ __noinline__ void issue_gu(const DSParams& P, DSShared* S, uint8_t* ring, uint32_t seq,
                                          const uint8_t* rec, int ch0) {
-  const int slot = seq % P.n_ring;
+  const int slot = fmod_(seq, P.fd_ring);
   uint8_t* dst = ring + static_cast<size_t>(slot) * P.slot_bytes;
   const uint32_t cb = 2 * kDsCps * P.gu_row, sb = 2 * kDsCps * P.gu_sc;
   mbar_arrive_expect_tx(&S->full[slot], cb + sb);
@@ -813,20 +944,11 @@ __device__ __forceinline__ void issue_gu(const DSParams& P, DSShared* S, uint8_t
 }
 
 // Down rows [r0, r1) of one record into dst (codes, then scales).
-__device__ __forceinline__ void copy_dn(const DSParams& P, uint8_t* dst, const uint8_t* rec, int r0, int r1,
+__device__ __noinline__ void copy_dn(const DSParams& P, uint8_t* dst, const uint8_t* rec, int r0, int r1,
                                         uint64_t* bar) {
   const uint32_t cb = (r1 - r0) * P.dn_row, sb = (r1 - r0) * P.dn_sc;
   bulk_g2s(dst, rec + P.lay.dn_codes + static_cast<size_t>(r0) * P.dn_row, cb, bar);
   bulk_g2s(dst + cb, rec + P.lay.dn_scales + static_cast<size_t>(r0) * P.dn_sc, sb, bar);
-}
-
-// Waits (bounded) until ring slot `seq` may be reused.
-__device__ __forceinline__ bool wait_slot(DSShared* S, uint64_t* empty, uint32_t seq, int n, uint64_t deadline) {
-  while (!ring_slot_free(empty, seq, n)) {
-    if (ds_aborted(S) || global_timer_ns() > deadline) return false;
-    __nanosleep(32);
-  }
-  return true;
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -834,7 +956,7 @@ template <int BITS, int GBPL, int DBPL, bool ROUTE>
 __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_stack_kernel(const DSParams P) {
   constexpr int CW = ds_consumer_warps(BITS);
   constexpr int CT = CW * 32;
-  extern __shared__ __align__(128) char smem[];
+  char* smem = ds_smem;
   DSShared* S = reinterpret_cast<DSShared*>(smem);
   const int np = P.T * P.k;
   const DSRoute R = ds_route(smem + P.sm_route, np);
@@ -854,10 +976,10 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
 
   // static splits: router rows, output rows (units of `gran` rows) and the
   // shared expert's channel blocks of this CTA
-  const int e0 = static_cast<int>((static_cast<long long>(P.E) * b) / G);
-  const int e1 = static_cast<int>((static_cast<long long>(P.E) * (b + 1)) / G);
-  const int r0 = P.gran * static_cast<int>((static_cast<long long>(P.n_units) * b) / G);
-  const int r1 = P.gran * static_cast<int>((static_cast<long long>(P.n_units) * (b + 1)) / G);
+  const int e0 = split_at(P.E, b, G);
+  const int e1 = split_at(P.E, b + 1, G);
+  const int r0 = P.gran * split_at(P.n_units, b, G);
+  const int r1 = P.gran * split_at(P.n_units, b + 1, G);
   const int sb0 = P.has_shared ? (b * nbf + G - 1) / G : 0;
   const int sb1 = P.has_shared ? ((b + 1) * nbf + G - 1) / G : 0;
   const int nsh = sb1 - sb0;
@@ -877,10 +999,9 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
     mbar_init(&S->wr_empty, CW);
     mbar_init(&S->route_bar, 1);
     S->abort_flag = 0;
-    for (int i = 0; i < kDsNHS; ++i) {
-      S->hs_done[i] = 0;
-      S->hs_gen[i] = 0;
-    }
+    S->n_uniq = 0;
+    S->route_ok = 0;
+    S->prm = P;
     fence_mbar_init();
   }
   __syncthreads();
@@ -895,121 +1016,185 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
   const uint64_t deadline = t_start + P.timeout_ns;
   unsigned long long* trace = P.trace != nullptr && b < kTraceCtas ? P.trace + b * kTraceSlots : nullptr;
   const int dl = P.L > 1 ? 1 : 0;
+  const DSParams& Q = S->prm;  // what the out-of-line helpers get
 
   if (warp == CW) {
     // ============================================================ producer
-    if (lane == 0) {
-      uint32_t seq = 0, wr_count = 0, shdn_count = 0;
-      bool ok = true;
-      auto issue_wr = [&](int l) {
-        const uint32_t bytes = static_cast<uint32_t>((e1 - e0) * P.d * 4);
-        mbar_arrive_expect_tx(&S->wr_full, bytes);
-        bulk_g2s(wrs, P.wr + (static_cast<size_t>(l) * P.E + e0) * P.d, bytes, &S->wr_full);
-        ++wr_count;
-      };
-      // layer l's shared-expert down rows: buffer l & 1, its (l >> 1)-th use
-      auto issue_shdn = [&](int l) {
-        const int j = l & 1;
-        if (l >= 2) {
-          while (!mbar_try_wait(&S->shdn_empty[j], ((l >> 1) - 1) & 1, 20000u)) {
+    // Lane i of the warp issues item i of each window of n_ring ring items (a
+    // gate/up stage or a down group), after waiting, on its own, for its
+    // slot's previous item to be consumed: copies issued from many lanes at
+    // once overlap their issue latency. A window never holds two items of
+    // one slot, so every wait is for the phase right after the one the
+    // previous window saw complete (mbarrier parity cannot tell phase k
+    // from phase k - 2).
+    uint32_t seq = 0, wr_count = 0, shdn_count = 0;
+    bool ok = true;
+    // waits (lane-local, bounded) until ring slot `q` may be reused
+    auto slot_ready = [&](uint32_t q) -> bool {
+      if (q < static_cast<uint32_t>(P.n_ring)) return true;
+      const uint32_t qd = fdiv(q, P.fd_ring);
+      const uint32_t parity = (qd - 1) & 1;
+      while (!mbar_try_wait(&S->empty[q - qd * P.n_ring], parity, 100000u)) {
+        if (ds_aborted(S) || global_timer_ns() > deadline) return false;
+      }
+      return true;
+    };
+    auto issue_wr = [&](int l) {
+      const uint32_t bytes = static_cast<uint32_t>((e1 - e0) * P.d * 4);
+      mbar_arrive_expect_tx(&S->wr_full, bytes);
+      bulk_g2s(wrs, P.wr + (static_cast<size_t>(l) * P.E + e0) * P.d, bytes, &S->wr_full);
+    };
+    // layer l's shared-expert down rows: buffer l & 1, its (l >> 1)-th use
+    auto issue_shdn = [&](int l) -> bool {
+      const int j = l & 1;
+      if (l >= 2) {
+        while (!mbar_try_wait(&S->shdn_empty[j], ((l >> 1) - 1) & 1, 100000u)) {
+          if (ds_aborted(S) || global_timer_ns() > deadline) return false;
+        }
+      }
+      const uint8_t* rec = P.shared + static_cast<size_t>(l) * P.stride;
+      mbar_arrive_expect_tx(&S->shdn_full[j], (r1 - r0) * (P.dn_row + P.dn_sc));
+      copy_dn(Q, shdn + j * P.dn_stride, rec, r0, r1, &S->shdn_full[j]);
+      return true;
+    };
+    // the shared expert's gate/up stages of layer l: ring items, one per lane
+    auto issue_shgu = [&](int l) -> bool {
+      const int n = nsh * (32 / kDsCps);
+      bool all = true;
+#pragma unroll 1
+      for (int w0 = 0; w0 < n && all; w0 += P.n_ring) {  // windows of n_ring items, as below
+        const int it = w0 + lane;
+        bool mine = true;
+        if (lane < P.n_ring && it < n) {
+          const uint32_t q = seq + it;
+          mine = slot_ready(q);
+          if (mine)
+            issue_gu(Q, S, ring, q, P.shared + static_cast<size_t>(l) * P.stride,
+                     (sb0 + it / (32 / kDsCps)) * 32 + (it % (32 / kDsCps)) * kDsCps);
+        }
+        all = __all_sync(0xffffffffu, mine);
+      }
+      seq += n;
+      return all;
+    };
+    const bool sh_dn = P.has_shared && has_rows;
+    // Iteration l issues layer l's routed items (l >= 0), then layer l + 1's
+    // inputs that do not depend on its x: router rows, shared-expert down
+    // rows and gate/up stages. wr_count (lane 0) and shdn_count (lane 1)
+    // count the copies each lane actually issued.
+#pragma unroll 1
+    for (int l = -1; l < P.L && ok; ++l) {
+      if (ds_aborted_warp(S)) break;
+      if (l >= 0) {
+        // routing of layer l is in shared memory once route_bar completes
+        int got = 1;
+        if (lane == 0) {
+          while (!mbar_try_wait(&S->route_bar, l & 1, 100000u)) {
             if (ds_aborted(S) || global_timer_ns() > deadline) {
-              ok = false;
-              return;
+              got = 0;
+              break;
             }
           }
         }
-        const uint8_t* rec = P.shared + static_cast<size_t>(l) * P.stride;
-        mbar_arrive_expect_tx(&S->shdn_full[j], (r1 - r0) * (P.dn_row + P.dn_sc));
-        copy_dn(P, shdn + j * P.dn_stride, rec, r0, r1, &S->shdn_full[j]);
-        ++shdn_count;
-      };
-      auto issue_shgu = [&](int l) {
-        const uint8_t* rec = P.shared + static_cast<size_t>(l) * P.stride;
-        for (int blk = sb0; blk < sb1 && ok; ++blk)
-          for (int q = 0; q < 32 / kDsCps && ok; ++q) {
-            if (!(ok = wait_slot(S, S->empty, seq, P.n_ring, deadline))) break;
-            issue_gu(P, S, ring, seq++, rec, blk * 32 + q * kDsCps);
-          }
-      };
-      if (!ds_aborted(S)) {
-        if (wr_rows) issue_wr(0);
-        if (P.has_shared && has_rows) issue_shdn(0);
-        if (P.has_shared) issue_shgu(0);
-      }
-      for (int l = 0; l < P.L && ok && !ds_aborted(S); ++l) {
-        // routing of layer l is in shared memory once route_bar completes
-        while (!mbar_try_wait(&S->route_bar, l & 1, 20000u)) {
-          if (ds_aborted(S) || global_timer_ns() > deadline) {
-            ok = false;
-            break;
-          }
+        if (!__shfl_sync(0xffffffffu, got, 0)) {
+          ok = false;
+          break;
         }
-        if (!ok) break;
-        unsigned long long* td = (trace != nullptr && l == dl) ? trace : nullptr;
+        if (S->route_ok == 0) {  // the consumers gave the layer up
+          ok = false;
+          break;
+        }
+        unsigned long long* td = (trace != nullptr && l == dl && lane == 0) ? trace : nullptr;
         if (td) td[16] = global_timer_ns();
-        const int nu = S->n_uniq;
+        const int nu = min(max(S->n_uniq, 0), min(np, P.E));
         const int tot = nu * nbf;
-        const int rb0 = static_cast<int>((static_cast<long long>(tot) * b) / G);
-        const int rb1 = static_cast<int>((static_cast<long long>(tot) * (b + 1)) / G);
-        for (int ig = 0; ig < (rb1 - rb0) * (32 / kDsCps) && ok; ++ig) {
-          const int blk = rb0 + ig / (32 / kDsCps);
-          const int u = blk / nbf, cb = blk % nbf;
-          if (!(ok = wait_slot(S, S->empty, seq, P.n_ring, deadline))) break;
-          issue_gu(P, S, ring, seq++, P.pool + static_cast<size_t>(R.uniq_slot[u]) * P.stride,
-                   cb * 32 + (ig % (32 / kDsCps)) * kDsCps);
-          if (td && ig == 0) td[17] = global_timer_ns();
-        }
-        if (td) td[18] = global_timer_ns();
+        const int rb0 = split_at(tot, b, G);
+        const int rb1 = split_at(tot, b + 1, G);
+        const int n_gu = (rb1 - rb0) * (32 / kDsCps);
         const int n_grp = has_rows ? (nu + P.gpd - 1) / P.gpd : 0;
-        for (int g = 0; g < n_grp && ok; ++g) {
-          if (!(ok = wait_slot(S, S->empty, seq, P.n_ring, deadline))) break;
-          const int u0 = g * P.gpd, u1 = min(nu, u0 + P.gpd);
-          const int slot = seq % P.n_ring;
-          uint8_t* dst = ring + static_cast<size_t>(slot) * P.slot_bytes;
-          mbar_arrive_expect_tx(&S->full[slot], (u1 - u0) * (r1 - r0) * (P.dn_row + P.dn_sc));
-          for (int u = u0; u < u1; ++u)
-            copy_dn(P, dst + (u - u0) * P.dn_stride, P.pool + static_cast<size_t>(R.uniq_slot[u]) * P.stride, r0, r1,
-                    &S->full[slot]);
-          ++seq;
+        const int n_items = n_gu + n_grp;
+#pragma unroll 1
+        for (int w0 = 0; w0 < n_items && ok; w0 += P.n_ring) {
+          const int it = w0 + lane;
+          bool mine = true;
+          if (lane < P.n_ring && it < n_items) {
+            const uint32_t q = seq + it;
+            mine = slot_ready(q);
+            if (mine) {
+              if (it < n_gu) {
+                const int blk = rb0 + it / (32 / kDsCps);
+                const int u = fdiv(blk, P.fd_nbf), cb = blk - u * nbf;
+                issue_gu(Q, S, ring, q, P.pool + static_cast<size_t>(R.uniq_slot[u]) * P.stride,
+                         cb * 32 + (it % (32 / kDsCps)) * kDsCps);
+              } else {
+                const int g = it - n_gu;
+                const int u0 = g * P.gpd, u1 = min(nu, u0 + P.gpd);
+                const int slot = fmod_(q, P.fd_ring);
+                uint8_t* dst = ring + static_cast<size_t>(slot) * P.slot_bytes;
+                mbar_arrive_expect_tx(&S->full[slot], (u1 - u0) * (r1 - r0) * (P.dn_row + P.dn_sc));
+#pragma unroll 1
+                for (int u = u0; u < u1; ++u)
+                  copy_dn(Q, dst + (u - u0) * P.dn_stride, P.pool + static_cast<size_t>(R.uniq_slot[u]) * P.stride,
+                          r0, r1, &S->full[slot]);
+              }
+            }
+          }
+          ok = __all_sync(0xffffffffu, mine);
+          if (td && w0 == 0) td[17] = global_timer_ns();
         }
-        if (td) td[19] = global_timer_ns();
+        seq += n_items;
+        if (td) td[18] = global_timer_ns();
         if (!ok) break;
-        if (l + 1 < P.L) {
-          // the next layer's inputs that do not depend on x
-          if (wr_rows) {
-            while (!mbar_try_wait(&S->wr_empty, l & 1, 20000u)) {
+      }
+      if (l + 1 < P.L) {
+        const int ln = l + 1;
+        int okn = 1;
+        if (wr_rows && lane == 0) {
+          if (ln > 0) {
+            while (!mbar_try_wait(&S->wr_empty, l & 1, 100000u)) {
               if (ds_aborted(S) || global_timer_ns() > deadline) {
-                ok = false;
+                okn = 0;
                 break;
               }
             }
-            if (!ok) break;
-            issue_wr(l + 1);
           }
-          if (P.has_shared && has_rows) issue_shdn(l + 1);
-          if (P.has_shared && ok) issue_shgu(l + 1);
+          if (okn) {
+            issue_wr(ln);
+            ++wr_count;
+          }
         }
+        if (sh_dn && lane == 1) {
+          okn = issue_shdn(ln) ? 1 : 0;
+          shdn_count += okn;
+        }
+        ok = __all_sync(0xffffffffu, okn != 0);
+        if (ok && P.has_shared) ok = issue_shgu(ln);
       }
-      if (!ok && !ds_aborted(S)) ds_abort(S, P.status, 10);
-      // every issued copy lands before the CTA may exit (they take
-      // microseconds; the 100 ms bound only guards against the impossible)
-      const uint64_t d2 = global_timer_ns() + 100000000ull;
+    }
+    if (lane == 0 && !ok && !ds_aborted(S)) ds_abort(S, P.status, 10);
+    // every issued copy lands before the CTA may exit; copies take
+    // microseconds, so after an abort (when a counted ring item may never
+    // have been issued) the waits give up after 2 ms in all
+    const uint64_t d2 = global_timer_ns() + 2000000ull;
+    if (lane == 0) {
+#pragma unroll 1
       for (uint32_t q = seq > static_cast<uint32_t>(P.n_ring) ? seq - P.n_ring : 0; q < seq; ++q)
         while (!mbar_try_wait(&S->full[q % P.n_ring], (q / P.n_ring) & 1, 20000u) && global_timer_ns() < d2) {
-        }
-      for (uint32_t q = shdn_count > 2u ? shdn_count - 2u : 0u; q < shdn_count; ++q)
-        while (!mbar_try_wait(&S->shdn_full[q & 1], (q >> 1) & 1, 20000u) && global_timer_ns() < d2) {
         }
       if (wr_count > 0)
         while (!mbar_try_wait(&S->wr_full, (wr_count - 1) & 1, 20000u) && global_timer_ns() < d2) {
         }
     }
+    if (lane == 1)
+#pragma unroll 1
+      for (uint32_t q = shdn_count > 2u ? shdn_count - 2u : 0u; q < shdn_count; ++q)
+        while (!mbar_try_wait(&S->shdn_full[q & 1], (q >> 1) & 1, 20000u) && global_timer_ns() < d2) {
+        }
     __syncwarp();
   } else {
     // ============================================================ consumers
     const int tid = threadIdx.x;
-    uint32_t seq = 0, blk_seq = 0;
-    XR<BITS> xr[GBPL];
+    uint32_t seq = 0;
 #pragma unroll 1
     for (int l = 0; l < P.L; ++l) {
       const uint32_t tag = base + 1 + static_cast<uint32_t>(l);
@@ -1018,10 +1203,17 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
       const bool traced = trace != nullptr && l < 2 && tid == 0;
       unsigned long long* tdet = (trace != nullptr && l == dl) ? trace : nullptr;
       if (traced) trace[8 * l] = global_timer_ns();
-      // ---- x of this layer
-      if (!ds_aborted(S))
-        ds_read_x<BITS>(P, ROUTE ? l : 0, tag, wr_rows ? xs : nullptr, xq, xres, r0, r1, S, deadline, CT);
+      // ---- x of this layer: layer l > 0 waits until every CTA has written
+      // its part of layer l - 1's output (and so has read all of layer l - 1)
+      if (ROUTE && l > 0) {
+        if (tid == 0 && !ds_aborted(S)) cnt_wait(kCntOut, (base + l) * G, S, P.status, 20, deadline);
+        named_sync(1, CT);
+        if (tdet && tid == 0) tdet[31] = global_timer_ns();
+      }
+      if (!ds_aborted_warp(S))
+        ds_read_x<BITS, GBPL>(P, ROUTE ? l : 0, tag, wr_rows ? xs : nullptr, xq, xres, r0, r1, S, deadline, CT);
       if (ROUTE) {
+#pragma unroll 1
         for (int e = tid; e < P.E; e += CT) R.slot_s[e] = __ldg(P.slot_of + static_cast<size_t>(l) * P.E + e);
       }
       named_sync(1, CT);
@@ -1031,37 +1223,57 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
         // ---- router rows of this CTA
         if (wr_rows) {
           if (ds_wait_warp(&S->wr_full, l & 1, S, deadline)) {
-            if (!ds_aborted(S)) ds_router(P, l, tag, wrs, xs, e0, e1, CW);
+            if (!ds_aborted_warp(S)) ds_router(P, l, tag, wrs, xs, e0, e1, CW);
           } else if (lane == 0 && !ds_aborted(S)) {
             ds_abort(S, P.status, 1);
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&S->wr_empty);
         }
+        // every CTA counts its logit rows as written, then waits for all
+        named_sync(1, CT);
+        if (tid == 0) {
+          cnt_add(kCntLogits);
+          if (!ds_aborted(S)) cnt_wait(kCntLogits, (base + l + 1) * G, S, P.status, 22, deadline);
+        }
+        named_sync(1, CT);
         if (traced) trace[8 * l + 2] = global_timer_ns();
         // ---- top-k (warp t) and grouping (all)
         const bool publisher = b == l % G;
         float* pub = publisher ? reinterpret_cast<float*>(P.rec + static_cast<size_t>(l) * P.rec_bytes + P.ro.logits)
                                : nullptr;
-        if (warp < P.T && !ds_aborted(S))
-          ds_topk(P, R, warp, tag, pub, reinterpret_cast<unsigned long long*>(hs) + warp * 32, S, deadline);
+        if (warp < P.T && !ds_aborted_warp(S))
+          ds_topk(Q, warp, tag, pub, reinterpret_cast<uint32_t*>(smem + P.sm_x) + warp * P.E, S, deadline,
+                  (tdet && warp == 0) ? tdet : nullptr);
         if (tdet && tid == 0) tdet[20] = global_timer_ns();
         named_sync(1, CT);
-        if (!ds_aborted(S)) ds_group(P, R, S, np, CT);
-        else named_sync(1, CT), named_sync(1, CT);
-        nu = S->n_uniq;
+        if (P.T > 1) {  // (one token: the top-k warp has grouped its pairs)
+          if (!ds_aborted_warp(S)) ds_group(Q, S, np, CT);
+          else named_sync(1, CT), named_sync(1, CT);
+        }
+        // the routing is complete unless some thread gave up: one decision
+        // for every consumer thread, which the producer reads behind route_bar
+        const bool route_bad = named_sync_or(1, CT, ds_aborted(S));
+        nu = route_bad ? 0 : min(max(S->n_uniq, 0), min(np, P.E));
         if (tdet && tid == 0) tdet[21] = global_timer_ns();
-        if (tid == 0) mbar_arrive(&S->route_bar);
-        if (publisher && !ds_aborted(S)) ds_publish(P, R, l, np, nu, CT);
+        if (tid == 0) {
+          S->route_ok = route_bad ? 0 : 1;
+          mbar_arrive(&S->route_bar);
+        }
+        if (route_bad) break;  // every consumer thread leaves the layer loop here
+        if (publisher) ds_publish(Q, l, np, nu, CT);
       } else {
         // the grouping was written by moe_group_tokens
         const int nug = min(max(__ldcg(P.g.n_uniq), 0), min(np, P.E));
+#pragma unroll 1
         for (int p = tid; p < np; p += CT) {
           R.pair_token[p] = min(max(__ldcg(P.g.pair_token + p), 0), P.T - 1);
           R.pair_gate[p] = __ldcg(P.g.pair_gate + p);
           R.pair_pos[p] = min(max(__ldcg(P.g.pair_pos + p), 0), np - 1);
         }
+#pragma unroll 1
         for (int u = tid; u <= nug; u += CT) R.uniq_off[u] = min(max(__ldcg(P.g.uniq_offset + u), 0), np);
+#pragma unroll 1
         for (int u = tid; u < nug; u += CT) {
           int slot = __ldcg(P.g.uniq_slot + u);
           if (slot < 0 || slot >= P.n_slots) {
@@ -1070,84 +1282,45 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
           }
           R.uniq_slot[u] = slot;
         }
-        if (tid == 0) S->n_uniq = nug;
-        named_sync(1, CT);
-        nu = nug;
-        if (tid == 0) mbar_arrive(&S->route_bar);
+        if (tid == 0) {
+          S->n_uniq = nug;
+          cnt_add(kCntLogits);  // no logits here, but the counters advance in step
+        }
+        const bool route_bad = named_sync_or(1, CT, ds_aborted(S));
+        nu = route_bad ? 0 : nug;
+        if (tid == 0) {
+          S->route_ok = route_bad ? 0 : 1;
+          mbar_arrive(&S->route_bar);
+        }
+        if (route_bad) break;  // every consumer thread leaves the layer loop here
       }
       if (traced) trace[8 * l + 3] = global_timer_ns();
 
       // ---- gate/up + SwiGLU: 32 channel tasks per block, blocks in order
       const int tot = nu * nbf;
-      const int rb0 = static_cast<int>((static_cast<long long>(tot) * b) / G);
-      const int rb1 = static_cast<int>((static_cast<long long>(tot) * (b + 1)) / G);
+      const int rb0 = split_at(tot, b, G);
+      const int rb1 = split_at(tot, b + 1, G);
       const int n_blk = nsh + (rb1 - rb0);
-      int cur_t = -1;
-#pragma unroll 1
-      for (int task = warp; task < n_blk * 32; task += CW) {
-        if (ds_aborted(S)) break;
-        const int beta = task >> 5, c = task & 31;
-        GUBlock gb;
-        gu_block_of(beta, nsh, sb0, rb0, nbf, gb);
-        const uint32_t sq = seq + beta * (32 / kDsCps) + c / kDsCps;
-        const int slot = sq % P.n_ring;
-        const uint32_t bid = blk_seq + beta;
-        const int hslot = bid % kDsNHS;
-        const int gen = bid / kDsNHS;
-        // the slot's previous block must have been published
-        bool ok = true;
-        if (lane == 0) {
-          while (*reinterpret_cast<volatile int*>(&S->hs_gen[hslot]) != gen) {
-            if (ds_aborted(S) || global_timer_ns() > deadline) {
-              ok = false;
-              break;
-            }
-            __nanosleep(20);
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok || !ds_wait_warp(&S->full[slot], (sq / P.n_ring) & 1, S, deadline)) {
-          if (lane == 0 && !ds_aborted(S)) ds_abort(S, P.status, 2);
-          break;
-        }
-        if (tdet && tid == 0) {
-          const int it = task / CW;
-          if (it == 0) tdet[22] = global_timer_ns();
-          if (it < 8) tdet[24 + it] = global_timer_ns();
-        }
-        float* hsl = hs + hslot * P.T * 32;
-        gu_task<BITS, GBPL>(P, R, ring + static_cast<size_t>(slot) * P.slot_bytes, c % kDsCps, xq, gb.u, np, hsl,
-                            c, cur_t, xr);
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) {
-          mbar_arrive(&S->empty[slot]);
-          __threadfence_block();
-          last = atomicAdd(&S->hs_done[hslot], 1) == 31;
-        }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-          // the block's 32 channels are in hs: requantise each token's 32
-          // values and publish them as tagged words
-          __threadfence_block();
-          int first, n;
-          expert_h_rows(R, gb.u, np, P.T, first, n);
-          for (int i = 0; i < n; ++i) {
-            const uint32_t wq = quant_block_warp(hsl[i * 32 + lane], lane);
-            if (lane < kQW)
-              st_ll(P.h_ll + (static_cast<size_t>(first + i) * nbf + gb.cb) * kQW + lane, ll_word(wq, tag));
-          }
-          __syncwarp();
-          if (lane == 0) {
-            S->hs_done[hslot] = 0;
-            __threadfence_block();
-            *reinterpret_cast<volatile int*>(&S->hs_gen[hslot]) = gen + 1;
-          }
-        }
-      }
+      if (!ds_aborted_warp(S))
+        gu_phase<BITS, GBPL, CW>(Q, S, nsh, sb0, rb0, n_blk, seq, deadline, (tdet && warp == 0) ? tdet : nullptr);
       if (tdet && tid == 0) tdet[23] = global_timer_ns();
       seq += n_blk * (32 / kDsCps);
-      blk_seq += n_blk;
+      named_sync(1, CT);
+      // every block's 32 channels are in hs: requantise and publish them
+      if (!ds_aborted(S)) {
+#pragma unroll 1
+        for (int beta = warp; beta < n_blk; beta += CW) {
+          GUBlock gb;
+          gu_block_of(beta, nsh, sb0, rb0, P.fd_nbf, gb);
+          gu_publish(Q, gb.u, gb.cb, np, hs + beta * P.T * 32, tag);
+        }
+      }
+      named_sync(1, CT);
+      // every CTA counts its h blocks as written, then waits for all
+      if (tid == 0) {
+        cnt_add(kCntH);
+        if (!ds_aborted(S)) cnt_wait(kCntH, (base + l + 1) * G, S, P.status, 23, deadline);
+      }
       named_sync(1, CT);
       if (traced) trace[8 * l + 4] = global_timer_ns();
 
@@ -1167,7 +1340,7 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
           const int u = i1 - sh;
           if (u >= 0 && i1 > i0) {
             const int ua = max(i0 - sh, 0);
-            if (u / P.gpd - ua / P.gpd >= P.n_ring) break;
+            if (static_cast<int>(fdiv(u, P.fd_gpd) - fdiv(ua, P.fd_gpd)) >= P.n_ring) break;
           }
           int first, n;
           expert_h_rows(R, u, np, P.T, first, n);
@@ -1175,21 +1348,23 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
           rows += n;
           ++i1;
         }
-        if (!ds_aborted(S)) ds_stage_h(P, R, np, i0, i1, sh != 0, tag, hq, S, deadline, CT);
+        if (i1 == i0) {  // a stage larger than the staging area: cannot happen with valid routing
+          if (tid == 0) ds_abort(S, P.status, 24);
+          break;
+        }
+        if (!ds_aborted(S)) ds_stage_h<DBPL>(P, R, np, i0, i1, sh, tag, hq, S, deadline, CT);
         named_sync(1, CT);
         if (traced && i0 == 0) trace[8 * l + 5] = global_timer_ns();
         // each warp takes whole stages; the hq row of stage i is the rows of
         // the stages before it in this round
 #pragma unroll 1
         for (int i = i0 + warp; i < i1; i += CW) {
-          if (ds_aborted(S)) break;
-          int row0 = 0;
-          for (int j = i0; j < i; ++j) {
-            int fj, nj;
-            expert_h_rows(R, j - sh, np, P.T, fj, nj);
-            row0 += nj;
-          }
+          if (ds_aborted_warp(S)) break;
           const int u = i - sh;
+          // hq row of the stage's first row: the round's shared rows, then
+          // the routed rows before it
+          const int n_sh = (sh && i0 == 0) ? P.T : 0;
+          const int row0 = u < 0 ? 0 : n_sh + R.uniq_off[u] - R.uniq_off[max(i0 - sh, 0)];
           const uint8_t* st;
           uint64_t* full;
           uint32_t parity;
@@ -1199,11 +1374,13 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
             full = &S->shdn_full[l & 1];
             parity = (l >> 1) & 1;
           } else {
-            const uint32_t sq = grp0 + u / P.gpd;
-            slot = sq % P.n_ring;
-            st = ring + static_cast<size_t>(slot) * P.slot_bytes + (u % P.gpd) * P.dn_stride;
+            const int g = fdiv(u, P.fd_gpd);
+            const uint32_t sq = grp0 + g;
+            const uint32_t sqd = fdiv(sq, P.fd_ring);
+            slot = sq - sqd * P.n_ring;
+            st = ring + static_cast<size_t>(slot) * P.slot_bytes + (u - g * P.gpd) * P.dn_stride;
             full = &S->full[slot];
-            parity = (sq / P.n_ring) & 1;
+            parity = sqd & 1;
           }
           if (!ds_wait_warp(full, parity, S, deadline)) {
             if (lane == 0 && !ds_aborted(S)) ds_abort(S, P.status, 3);
@@ -1217,8 +1394,9 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
             } else {
               // the group's 16 arrivals: its first expert brings the ones the
               // group has no expert for
-              const int m = min(nu - (u / P.gpd) * P.gpd, P.gpd);
-              mbar_arrive_cnt(&S->empty[slot], (u % P.gpd) == 0 ? kDsCps - (m - 1) : 1);
+              const int g0 = fdiv(u, P.fd_gpd) * P.gpd;
+              const int m = min(nu - g0, P.gpd);
+              mbar_arrive_cnt(&S->empty[slot], u == g0 ? kDsCps - (m - 1) : 1);
             }
           }
         }
@@ -1226,19 +1404,19 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
         i0 = i1;
       }
       seq += has_rows ? (nu + P.gpd - 1) / P.gpd : 0;
-      // this CTA has read everything of layer l that other CTAs wrote
-      if (tid == 0 && ROUTE && l + 1 < P.L)
-        st_ll(P.done_ll + static_cast<size_t>(l & 1) * kDsMaxCtas + b, ll_word(0u, tag));
       if (traced) trace[8 * l + 6] = global_timer_ns();
 
       // ---- combine: y[t, r] = sum_j gate[t,j] z[(t,j)][r] + z_shared[t][r] (+ x)
       if (!ds_aborted(S) && has_rows) {
-        const int npairs = nr_out / 2;
+        const int hp = P.rpc / 2;  // row pairs of the widest CTA
         char* yl = static_cast<char*>(P.y) + static_cast<size_t>(l) * P.T * P.d * (P.out_f32 ? 4 : 2);
         unsigned long long* yll = P.y_ll + static_cast<size_t>(l & 1) * P.T * (P.d / 2);
-        for (int i = tid; i < P.T * npairs; i += CT) {
-          const int t = i / npairs, rr = 2 * (i % npairs);
+#pragma unroll 1
+        for (int i = tid; i < P.T * hp; i += CT) {
+          const int t = fdiv(i, P.fd_hp), rr = 2 * (i - t * hp);
+          if (rr >= nr_out) continue;
           float a0 = 0.f, a1 = 0.f;
+#pragma unroll 1
           for (int j = 0; j < P.k; ++j) {
             const int p = R.pair_pos[t * P.k + j];
             const float g = R.pair_gate[p];
@@ -1266,6 +1444,9 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
       }
       if (l + 2 == P.L && tid == 0) grid_dep_launch();
       named_sync(1, CT);
+      // this CTA's output rows are written and it has read everything of
+      // layer l that other CTAs wrote
+      if (tid == 0) cnt_add(kCntOut);
       if (traced) trace[8 * l + 7] = global_timer_ns();
     }
     if (P.L == 1 && tid == 0) grid_dep_launch();
@@ -1284,9 +1465,13 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
 
 // Moves the tag counter far past every tag an interrupted launch may have
 // written, so that none of its words can match a later launch.
-__global__ void ds_skip_tags_kernel() {
-  atomicAdd(&g_ds_epoch, 1u << 20);
+__global__ void ds_skip_tags_kernel(int G) {
+  const unsigned e = atomicAdd(&g_ds_epoch, 1u << 20) + (1u << 20);
   atomicExch(&g_ds_exit, 0u);
+  // the exchange counters restart in step with the new tag counter
+  atomicExch(&g_ds_cnt[kCntLogits], e * G);
+  atomicExch(&g_ds_cnt[kCntH], e * G);
+  atomicExch(&g_ds_cnt[kCntOut], e * G);
 }
 
 // ------------------------------------------------------------------ host side
@@ -1336,8 +1521,7 @@ size_t decode_exchange_bytes(const moe_layer_cfg& c, int T) {
   const size_t lg = ds_align(static_cast<size_t>(kDsLogitCopies) * T * c.E * 8, 256);
   const size_t h = ds_align(n_rows * (c.f / kBlock) * kQW * 8, 256);
   const size_t y = ds_align(2 * static_cast<size_t>(T) * (c.d / 2) * 8, 256);
-  const size_t dn = 2 * kDsMaxCtas * 8;
-  return lg + h + y + dn;
+  return lg + h + y;
 }
 
 __global__ void ds_probe_kernel() {}
@@ -1361,6 +1545,10 @@ cudaError_t decode_init(Ctx& ctx) {
     const unsigned start = (static_cast<unsigned>(rd()) & 0xfff00000u) | 0x00010000u;
     e = cudaMemcpyToSymbol(g_ds_epoch, &start, sizeof(start));
     if (e != cudaSuccess) return e;
+    unsigned cnt[96] = {};
+    cnt[kCntLogits] = cnt[kCntH] = cnt[kCntOut] = start * static_cast<unsigned>(ctx.num_sms);
+    e = cudaMemcpyToSymbol(g_ds_cnt, cnt, sizeof(cnt));
+    if (e != cudaSuccess) return e;
   }
   // whether a cooperative launch also takes programmatic serialization here
   // (probed once, outside any stream capture, with an empty kernel)
@@ -1379,8 +1567,8 @@ cudaError_t decode_init(Ctx& ctx) {
   return cudaSuccess;
 }
 
-cudaError_t decode_skip_tags(cudaStream_t s) {
-  ds_skip_tags_kernel<<<1, 1, 0, s>>>();
+cudaError_t decode_skip_tags(const Ctx& ctx, cudaStream_t s) {
+  ds_skip_tags_kernel<<<1, 1, 0, s>>>(ctx.num_sms);
   return cudaGetLastError();
 }
 
@@ -1441,13 +1629,16 @@ cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const St
     P.logits_ll = reinterpret_cast<unsigned long long*>(ex);
     P.h_ll = reinterpret_cast<unsigned long long*>(ex + lg);
     P.y_ll = reinterpret_cast<unsigned long long*>(ex + lg + h);
-    P.done_ll = reinterpret_cast<unsigned long long*>(ex + lg + h + y);
   }
   P.status = ctx.d_status;
   P.timeout_ns = ctx.timeout_ns;
   P.trace = ctx.d_trace;
   P.gu_lpr = gg.lpr;
   P.dn_lpr = gd.lpr;
+  P.gu_lsh = __builtin_ctz(static_cast<unsigned>(gg.lpr));
+  P.dn_lsh = __builtin_ctz(static_cast<unsigned>(gd.lpr));
+  P.fd_nb = make_fastdiv(nbd);
+  P.fd_nbf = make_fastdiv(nbf);
   P.gu_row = c.d * c.bits / 8;
   P.gu_sc = nbd * 2;
   P.dn_row = c.f * c.bits / 8;
@@ -1476,9 +1667,15 @@ cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const St
   P.sm_xres = static_cast<int>(o);
   o = ds_align(o + static_cast<size_t>(T) * P.rpc * 4, 128);
   P.sm_hs = static_cast<int>(o);
-  const size_t hs_bytes = static_cast<size_t>(kDsNHS) * T * 32 * 4;
-  const size_t tk_bytes = static_cast<size_t>(MOE_DECODE_MAX_T) * 32 * 8;  // top-k scratch (aliases hs)
-  o = ds_align(o + (hs_bytes > tk_bytes ? hs_bytes : tk_bytes), 128);
+  const int nu_max0 = np < c.E ? np : c.E;
+  // the kernel splits items among the CTAs in 32-bit arithmetic
+  if (static_cast<long long>(nu_max0) * nbf * G >= (1ll << 31) ||
+      static_cast<long long>(c.E > P.n_units ? c.E : P.n_units) * G >= (1ll << 31))
+    return cudaErrorNotSupported;
+  P.max_blk = (nu_max0 * nbf + G - 1) / G + (nbf + G - 1) / G;
+  if (P.max_blk > kDsMaxBlk) return cudaErrorNotSupported;
+  const size_t hs_bytes = static_cast<size_t>(P.max_blk) * T * 32 * 4;
+  o = ds_align(o + hs_bytes, 128);
   P.sm_xq = static_cast<int>(o);
   o = ds_align(o + static_cast<size_t>(T) * kQW * nbd * 4, 128);
   P.sm_wr = static_cast<int>(o);
@@ -1487,23 +1684,34 @@ cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const St
   o = ds_align(o + 2 * static_cast<size_t>(P.dn_stride), 128);
   P.sm_x = static_cast<int>(o);
   const size_t fixed = o;
-  // the staging area: raw x for the router, then the quantised h rows of a
-  // round of down stages (all rows if they fit in 48 KB, else 48 KB worth,
-  // at least T rows); at least three ring slots
+  // the staging area: raw x for the router, the top-k key rows, then the
+  // quantised h rows of a round of down stages (all rows if they fit in
+  // 48 KB, else 48 KB worth, at least T rows); at least three ring slots,
+  // for which the h rows give way down to their minimum
   const size_t xs_bytes = a.route ? static_cast<size_t>(T) * c.d * 2 : 0;
   const size_t hq_row = static_cast<size_t>(kQW) * nbf * 4;
+  const size_t keys_bytes = static_cast<size_t>(T) * c.E * 4;  // top-k key rows (after the router)
+  size_t x_min = xs_bytes > keys_bytes ? xs_bytes : keys_bytes;
+  if (x_min < T * hq_row) x_min = T * hq_row;
   size_t hq_bytes = static_cast<size_t>(n_rows) * hq_row;
-  const size_t hq_cap = 48 * 1024 > T * hq_row ? 48 * 1024 : T * hq_row;
-  if (hq_bytes > hq_cap) hq_bytes = hq_cap;
-  const size_t x_bytes = ds_align(xs_bytes > hq_bytes ? xs_bytes : hq_bytes, 128);
+  if (hq_bytes > 48 * 1024) hq_bytes = 48 * 1024;
+  size_t x_bytes = ds_align(x_min > hq_bytes ? x_min : hq_bytes, 128);
+  auto ring_slots = [&](size_t xb) {
+    const long long r = static_cast<long long>(kDsSmemMax) - static_cast<long long>(ds_align(fixed + xb, 128));
+    return r > 0 ? static_cast<int>(r / P.slot_bytes) : 0;
+  };
+  if (ring_slots(x_bytes) < 3) x_bytes = ds_align(x_min, 128);
   P.hq_rows = static_cast<int>(x_bytes / hq_row);
   if (P.hq_rows > n_rows) P.hq_rows = n_rows;
   o = ds_align(fixed + x_bytes, 128);
-  const long long rem = static_cast<long long>(kDsSmemMax) - static_cast<long long>(o);
-  int n_ring = static_cast<int>(rem / P.slot_bytes);
+  int n_ring = ring_slots(x_bytes);
   if (n_ring > kDsNS) n_ring = kDsNS;
   if (n_ring < 3) return cudaErrorNotSupported;
   P.n_ring = n_ring;
+  P.fd_ring = make_fastdiv(n_ring);
+  P.fd_hrow = make_fastdiv(nbf * (kQW / 2));
+  P.fd_hp = make_fastdiv(P.rpc / 2);
+  P.fd_gpd = make_fastdiv(P.gpd);
   P.sm_ring = static_cast<int>(o);
   o += static_cast<size_t>(n_ring) * P.slot_bytes;
   if (o > static_cast<size_t>(kDsSmemMax)) return cudaErrorNotSupported;

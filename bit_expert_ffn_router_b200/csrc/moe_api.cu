@@ -350,7 +350,7 @@ moe_status moe_check_device_status(moe_ctx* ctx, moe_stream stream) {
   ctx->c.last_detail = h[1];
   // clear the status word, and move the decode kernel's tag counter past any
   // tag an interrupted launch may have written
-  if (cudaMemsetAsync(ctx->c.d_status, 0, 64, s) != cudaSuccess || decode_skip_tags(s) != cudaSuccess ||
+  if (cudaMemsetAsync(ctx->c.d_status, 0, 64, s) != cudaSuccess || decode_skip_tags(ctx->c, s) != cudaSuccess ||
       cudaStreamSynchronize(s) != cudaSuccess)
     return MOE_ECUDA;
   return h[0] == kDevTimeout ? MOE_ETIMEOUT : MOE_EDEVICE;

@@ -34,7 +34,7 @@ struct Ctx {
   bool coop_pdl = false;
   int last_detail = 0;             // detail word of the last device error moe_check_device_status read           // a cooperative launch also takes programmatic serialization
 };
-constexpr int kTraceSlots = 32;
+constexpr int kTraceSlots = 64;
 constexpr int kTraceCtas = 1024;
 
 }  // namespace moe
@@ -187,7 +187,7 @@ struct StackArgs {
 cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const StackArgs& a, cudaStream_t s);
 size_t decode_exchange_bytes(const moe_layer_cfg& c, int T);
 // Moves the decode kernel's tag counter past an interrupted launch's tags.
-cudaError_t decode_skip_tags(cudaStream_t s);
+cudaError_t decode_skip_tags(const Ctx& ctx, cudaStream_t s);
 bool decode_geometry_ok(int d, int f);
 
 // FFN arguments of the prefill path

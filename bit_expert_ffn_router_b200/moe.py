@@ -293,7 +293,7 @@ class Context:
     def trace_fetch(self, n_ctas: int, stream=None):
         """Phase timestamps of the last decode-layer launches (MOE_TRACE set at creation)."""
         import numpy as np
-        buf = np.zeros((n_ctas, 32), dtype=np.uint64)
+        buf = np.zeros((n_ctas, 64), dtype=np.uint64)
         _check(self.lib.moe_trace_fetch(self.h, buf.ctypes.data, buf.size, _stream(stream)), "moe_trace_fetch")
         return buf
 

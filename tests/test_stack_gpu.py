@@ -153,3 +153,37 @@ def test_stack_argument_errors():
     assert c.stack_forward_status(**{**args, "ws": ws[:ws.numel() // 2]}) == M.ENOSPACE
     assert c.stack_forward_status(**{**args, "L": 0}) == M.EINVAL
     assert c.check_device_status() == M.OK
+
+
+@pytest.mark.parametrize("limit_us", [1, 5, 20])
+def test_stack_wait_limits_report_timeout_and_recover(monkeypatch, limit_us):
+    """Short wait limits make the stack kernel give up at different points
+    (an exchange, a weight stage, the routing of a later layer): every launch
+    ends, reports MOE_ETIMEOUT (or finishes), and the same context then gives
+    the exact results of an unlimited one."""
+    cfg = M.FULL.replace(bits=2, out_fp32=0, residual=1)
+    st = Stack(cfg, 3, 4, seed=610)
+    ref, _ = st.forward()
+    torch.cuda.synchronize()
+    dv = st.dev
+    monkeypatch.setenv("MOE_TIMEOUT_US", str(limit_us))
+    short = M.Context(torch.cuda.current_device())
+    monkeypatch.delenv("MOE_TIMEOUT_US")
+    ws = M.stack_workspace(cfg, st.L, st.T)
+    seen = set()
+    for _ in range(4):
+        y = st.out()
+        assert short.stack_forward_status(cfg, st.L, dv["x"], st.T, dv["wr"], dv["bias"], dv["slot_of"], st.n_slots,
+                                          dv["pool"], st.stride, dv["shared"], ws, y) == M.OK
+        s = short.check_device_status()
+        assert s in (M.OK, M.ETIMEOUT)
+        seen.add(s)
+        assert short.check_device_status() == M.OK
+        if s == M.OK:
+            assert torch.equal(y, ref)
+    if limit_us == 1:
+        assert M.ETIMEOUT in seen
+    short.close()
+    y2, _ = st.forward()
+    torch.cuda.synchronize()
+    assert torch.equal(y2, ref)
