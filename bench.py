@@ -477,8 +477,9 @@ def layer_call_record(st, steps, world):
     M, cfg, p = st.M, st.cfg, st.p
     ws = M.workspace(cfg, st.T)
     bias = st.bias[0]
+    s = torch.cuda.Stream()  # the calls launch on the stream the graph captures
     calls = [st.ctx.prepare_layer_forward(cfg, st.T, p["wr"][l], bias[l], p["slot_of"][l * cfg.E:(l + 1) * cfg.E],
-                                          p["n_slots"], p["pool"], p["stride"], p["shared"][l], ws)
+                                          p["n_slots"], p["pool"], p["stride"], p["shared"][l], ws, stream=s)
              for l in range(st.L)]
 
     def run():
@@ -487,14 +488,13 @@ def layer_call_record(st, steps, world):
             c(x, st.y[l])
             x = st.y[l]
 
-    s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
         run()
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
+    with torch.cuda.graph(g, stream=s):
         run()
     for _ in range(3):
         g.replay()

@@ -43,7 +43,9 @@ namespace moe {
 __host__ __device__ constexpr int ds_consumer_warps(int bits) { return bits == 2 ? 15 : 11; }
 constexpr int kDsNS = 12;       // weight ring slots (at most)
 constexpr int kDsMaxBlk = 40;   // gate/up channel blocks of one CTA in one layer (at most)
-constexpr int kDsCps = 16;      // gate/up channels per ring stage
+constexpr int kDsArr = 16;      // arrivals that release a ring slot (one down group)
+constexpr int kDsGuDepth = 4;   // gate/up tasks a consumer warp has in flight
+constexpr int kDsGpd = 6;       // routed experts per down group (ring slot)
 constexpr int kQW = 18;         // words per quantised 32-value block: 16 int16 pairs, scale, sum
 constexpr int kDsMaxCtas = 256;  // grid size limit (done words per layer parity)
 constexpr int kDsLogitCopies = 4;  // copies of the logit words: CTA b reads copy b % 4
@@ -120,6 +122,7 @@ struct DSParams {
   int dn_stride, gpd;           // bytes per down stage, down stages per ring slot
   int hq_rows;
   int sm_wr, sm_x, sm_xq, sm_hs, sm_zs, sm_route, sm_xres, sm_ring, sm_shdn;
+  int sm_gub, gu_task_bytes, gu_depth;  // per-warp gate/up buffers: gu_depth tasks of gu_task_bytes each
   int max_blk;                  // gate/up blocks of one CTA in one layer (h staging slots)
 };
 
@@ -477,12 +480,10 @@ __device__ __noinline__ void ds_topk(const DSParams& P, int t, uint32_t tag, flo
     const int e = v * 32 + lane;
     const float lv = __uint_as_float(static_cast<uint32_t>(w[v]));
     kv[v] = e < P.E ? ds_order_key(lv) : 0u;
-    if (e < P.E) kr[e] = kv[v];
-  }
-  if (pub_logits != nullptr) {  // the publishing CTA: the plain logits, from L2 again
-#pragma unroll 1
-    for (int e = lane; e < P.E; e += 32)
-      pub_logits[static_cast<size_t>(t) * P.E + e] = __uint_as_float(static_cast<uint32_t>(ld_ll(row + e)));
+    if (e < P.E) {
+      kr[e] = kv[v];
+      if (pub_logits != nullptr) pub_logits[static_cast<size_t>(t) * P.E + e] = lv;  // the publishing CTA
+    }
   }
   if (td && lane == 0) td[29] = global_timer_ns();
   uint32_t mine_key = 0u;
@@ -742,63 +743,149 @@ __device__ __forceinline__ int h_row_token(const DSRoute& R, int u, int first, i
   return u < 0 ? i : R.pair_token[first + i];
 }
 
-// The gate/up + SwiGLU phase of one layer for one consumer warp: its channel
-// tasks (task j = channel j % 32 of block j / 32; blocks in order: this
-// CTA's shared-expert blocks, then its routed blocks), each for every token
-// of the block's expert, the weights in ring stage seq + j / 16; h -> hs.
-// Out of line on purpose: the loop gets the whole register budget instead of
-// sharing it with the live state of the kernel around it. The launch
-// parameters come from their shared-memory copy and are read into registers
-// once. Returns false when the phase gave up (abort or timeout).
+// ---- gate/up data path: every consumer warp streams the rows of its own
+// channel tasks (task j = channel j % 32 of block j / 32; blocks in order:
+// this CTA's shared-expert blocks, then its routed blocks; warp w takes
+// tasks w, w + CW, ...) into a private buffer of kDsGuDepth task slots with
+// 16-byte cp.async, one commit group per task (gu_depth <= kDsGuDepth slots,
+// chosen at launch to fit shared memory). Many warps issuing at once
+// keep the copies' issue cost off one thread, and no slot is shared.
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// waits until at most n (clamped to 0..kDsGuDepth-1) of this thread's newest groups are pending
+__device__ __forceinline__ void cp_async_wait_pending(int n) {
+  if (n <= 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
+  else if (n == 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
+  else if (n == 2) asm volatile("cp.async.wait_group 2;" ::: "memory");
+  else asm volatile("cp.async.wait_group 3;" ::: "memory");
+}
+static_assert(kDsGuDepth == 4, "cp_async_wait_pending covers depths up to 4");
+
+// First routed gate/up block (index u * nbf + cb over the unique experts)
+// whose work offset sh_w + nbf * uniq_off[u] + cb * n_u is at least x.
+__device__ __forceinline__ int routed_block_at(const DSRoute& R, int nu, int nbf, int sh_w, int x) {
+  if (nu <= 0) return 0;
+  int lo = 0, hi = nu - 1;  // the last u whose first block starts at or before x
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (sh_w + nbf * R.uniq_off[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  const int base = sh_w + nbf * R.uniq_off[lo];
+  if (x <= base) return lo * nbf;
+  const int n = max(R.uniq_off[lo + 1] - R.uniq_off[lo], 1);
+  const int cb = (x - base + n - 1) / n;
+  return cb >= nbf ? (lo + 1) * nbf : lo * nbf + cb;
+}
+
+// Record (byte address) and channel of task j of layer l, or false past the
+// CTA's blocks.
+__device__ __forceinline__ const uint8_t* gu_task_rec(const DSParams& P, const int32_t* uniq_slot, int l, int j,
+                                                      int nsh, int sb0, int rb0, int& ch, int& u) {
+  const int beta = j >> 5;
+  if (beta < nsh) {
+    u = -1;
+    ch = (sb0 + beta) * 32 + (j & 31);
+    return P.shared + static_cast<size_t>(l) * P.stride;
+  }
+  const int g = rb0 + beta - nsh;
+  u = static_cast<int>(fdiv(g, P.fd_nbf));
+  ch = (g - u * static_cast<int>(P.fd_nbf.d)) * 32 + (j & 31);
+  return P.pool + static_cast<size_t>(uniq_slot[u]) * P.stride;
+}
+
+// One task's rows (gate and up of channel ch: codes, then scales) into a
+// buffer slot; the warp's lanes split the 16-byte pieces. Commits one group
+// (empty when there is no task) so that group counts stay per task.
+__device__ __forceinline__ void gu_load(const DSParams& P, const uint8_t* rec, int ch, uint8_t* dst, bool valid) {
+  const int lane = threadIdx.x & 31;
+  if (valid) {
+    const int cbytes = 2 * P.gu_row, sbytes = 2 * P.gu_sc;
+    const uint8_t* cs = rec + P.lay.gu_codes + static_cast<size_t>(2 * ch) * P.gu_row;
+    const uint8_t* ss = rec + P.lay.gu_scales + static_cast<size_t>(2 * ch) * P.gu_sc;
+#pragma unroll 1
+    for (int o = lane * 16; o < cbytes; o += 32 * 16) cp_async16(dst + o, cs + o);
+#pragma unroll 1
+    for (int o = lane * 16; o < sbytes; o += 32 * 16) cp_async16(dst + cbytes + o, ss + o);
+  }
+  cp_async_commit();
+}
+
+// Issues this warp's shared-expert tasks of layer l (the first ones of its
+// list) before the layer's routing is known. Returns how many were issued.
+template <int CW>
+__device__ __noinline__ int gu_prefetch_shared(const DSParams& Q, int l, int nsh, int sb0) {
+  const int warp = threadIdx.x >> 5;
+  uint8_t* wbuf = reinterpret_cast<uint8_t*>(ds_smem + Q.sm_gub) +
+                  static_cast<size_t>(warp) * Q.gu_depth * Q.gu_task_bytes;
+  int n = 0;
+#pragma unroll 1
+  for (int j = warp; j < nsh * 32 && n < Q.gu_depth; j += CW, ++n) {
+    int ch, u;
+    const uint8_t* rec = gu_task_rec(Q, nullptr, l, j, nsh, sb0, 0, ch, u);
+    gu_load(Q, rec, ch, wbuf + static_cast<size_t>(n) * Q.gu_task_bytes, true);
+  }
+  return n;
+}
+
+// The gate/up + SwiGLU phase of layer l for one consumer warp: streams and
+// computes its tasks (the first n_pre of them were issued already), each for
+// every token of the block's expert; h -> hs. Out of line on purpose: the
+// loop gets the whole register budget instead of sharing it with the live
+// state of the kernel around it. The launch parameters come from their
+// shared-memory copy and are read into registers once. Returns false when
+// the phase gave up (abort).
 template <int BITS, int BPL, int CW>
-__device__ __noinline__ bool gu_phase(const DSParams& Q, DSShared* S, int nsh, int sb0, int rb0, int n_blk,
-                                      uint32_t seq, uint64_t deadline, unsigned long long* td) {
+__device__ __noinline__ bool gu_phase(const DSParams& Q, DSShared* S, int l, int nsh, int sb0, int rb0, int n_blk,
+                                      int n_pre, unsigned long long* td) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int d = Q.d, T = Q.T, np = Q.T * Q.k, nb = Q.d / kBlock;
   const int lpr = Q.gu_lpr, gl = lane & (lpr - 1);
   const bool active = lane < lpr;
-  const int gu_row = Q.gu_row, slot_bytes = Q.slot_bytes, n_ring = Q.n_ring;
-  const FastDiv fd_ring = Q.fd_ring, fd_nbf = Q.fd_nbf;
-  int* status = Q.status;
-  const uint8_t* ring = reinterpret_cast<const uint8_t*>(ds_smem + Q.sm_ring);
+  const int gu_row = Q.gu_row, tb = Q.gu_task_bytes;
   float* hs = reinterpret_cast<float*>(ds_smem + Q.sm_hs);
   const int* xq = reinterpret_cast<const int*>(ds_smem + Q.sm_xq);
+  const int depth = Q.gu_depth;
+  uint8_t* wbuf = reinterpret_cast<uint8_t*>(ds_smem + Q.sm_gub) + static_cast<size_t>(warp) * depth * tb;
   const DSRoute R = ds_route(ds_smem + Q.sm_route, np);
+  const int n_task = warp < n_blk * 32 ? (n_blk * 32 - warp + CW - 1) / CW : 0;
+  int issued = n_pre;
+  // fill the pipeline
+#pragma unroll 1
+  for (; issued < n_task && issued < depth; ++issued) {
+    int ch, u;
+    const uint8_t* rec = gu_task_rec(Q, R.uniq_slot, l, warp + issued * CW, nsh, sb0, rb0, ch, u);
+    gu_load(Q, rec, ch, wbuf + static_cast<size_t>(issued) * tb, true);
+  }
   XR<BITS> xr[BPL];
-  int cur_t = -1;
+  int cur_t = -1, rs = 0;  // rs: the slot of task i (task i + depth refills it)
   bool ok = true;
 #pragma unroll 1
-  for (int task = warp; task < n_blk * 32; task += CW) {
+  for (int i = 0; i < n_task; ++i) {
     if (ds_aborted_warp(S)) {
       ok = false;
       break;
     }
+    const int task = warp + i * CW;
     const int beta = task >> 5, c = task & 31;
-    GUBlock gb;
-    gu_block_of(beta, nsh, sb0, rb0, fd_nbf, gb);
-    const uint32_t sq = seq + beta * (32 / kDsCps) + c / kDsCps;
-    const uint32_t sqd = fdiv(sq, fd_ring);
-    const int slot = sq - sqd * n_ring;
-    if (!ds_wait_warp(&S->full[slot], sqd & 1, S, deadline)) {
-      if (lane == 0 && !ds_aborted(S)) ds_abort(S, status, 2);
-      ok = false;
-      break;
-    }
-    const int ti = (task - warp) / CW;  // this warp's task count
+    const int u = beta < nsh ? -1 : static_cast<int>(fdiv(rb0 + beta - nsh, Q.fd_nbf));
+    cp_async_wait_pending(issued - i - 1);
+    __syncwarp();
     if (td && lane == 0) {
-      if (task == warp) td[22] = global_timer_ns();  // first stage in
-      if (ti < 16) td[32 + ti] = global_timer_ns();
+      if (i == 0) td[22] = global_timer_ns();  // first task's rows in
+      if (i < 8) td[32 + i] = global_timer_ns();
     }
-    const uint8_t* st = ring + static_cast<size_t>(slot) * slot_bytes;
-    const int cl = c % kDsCps;
-    const uint8_t* cg = st + 2 * cl * gu_row;
-    const uint16_t* sg = reinterpret_cast<const uint16_t*>(st + 2 * kDsCps * gu_row) + 2 * cl * nb;
+    const uint8_t* st = wbuf + static_cast<size_t>(rs) * tb;
+    const uint8_t* cg = st;
+    const uint16_t* sg = reinterpret_cast<const uint16_t*>(st + 2 * gu_row);
     float* hsl = hs + beta * T * 32;
     int first, n;
-    expert_h_rows(R, gb.u, np, T, first, n);
+    expert_h_rows(R, u, np, T, first, n);
 #pragma unroll 1
-    for (int i = 0; i < n; ++i) {
-      const int t = h_row_token(R, gb.u, first, i);
+    for (int k = 0; k < n; ++k) {
+      const int t = h_row_token(R, u, first, k);
       if (t != cur_t) {
         load_xq<BITS, BPL>(xq + t * kQW * nb, nb, lpr, gl, xr);
         cur_t = t;
@@ -808,12 +895,19 @@ __device__ __noinline__ bool gu_phase(const DSParams& Q, DSShared* S, int nsh, i
       v = group_sum2(v, lpr);
       // fast exponential and division: h is requantised to 16 bits for the
       // down rows, far coarser than their few-ulp error
-      if (lane == 0) hsl[i * 32 + c] = __fdividef(v.x, 1.f + __expf(-v.x)) * v.y;
+      if (lane == 0) hsl[k * 32 + c] = __fdividef(v.x, 1.f + __expf(-v.x)) * v.y;
     }
-    if (td && lane == 0 && ti < 16) td[48 + ti] = global_timer_ns();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&S->empty[slot]);
+    if (td && lane == 0 && i < 8) td[48 + i] = global_timer_ns();
+    __syncwarp();  // the slot is read: refill it with task i + depth
+    if (issued < n_task) {
+      int ch, uu;
+      const uint8_t* rec = gu_task_rec(Q, R.uniq_slot, l, warp + issued * CW, nsh, sb0, rb0, ch, uu);
+      gu_load(Q, rec, ch, wbuf + static_cast<size_t>(rs) * tb, true);
+      ++issued;
+    }
+    rs = rs + 1 == depth ? 0 : rs + 1;
   }
+  asm volatile("cp.async.wait_all;" ::: "memory");  // nothing of this layer stays in flight
   return ok;
 }
 
@@ -925,22 +1019,12 @@ __device__ __forceinline__ void dn_task(const DSParams& P, const DSRoute& R, con
 }
 
 // ------------------------------------------------------------------ producer
-// One ring of fixed-size slots carries, in order, every gate/up stage (16
-// channels) and down group (the down rows of up to `gpd` routed experts) of
-// a layer; consumers free a slot with 16 arrivals. Down groups follow the
-// gate/up stages, so they stream in while gate/up is still computing.
+// One ring of fixed-size slots carries the down groups of a layer (the down
+// rows, this CTA's output rows, of up to `gpd` routed experts each), issued
+// as soon as the routing is known, so they stream in while gate/up computes;
+// consumers free a slot with 16 arrivals.
 __device__ __forceinline__ void mbar_arrive_cnt(uint64_t* b, uint32_t count) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
-}
-
-__device__ __noinline__ void issue_gu(const DSParams& P, DSShared* S, uint8_t* ring, uint32_t seq,
-                                         const uint8_t* rec, int ch0) {
-  const int slot = fmod_(seq, P.fd_ring);
-  uint8_t* dst = ring + static_cast<size_t>(slot) * P.slot_bytes;
-  const uint32_t cb = 2 * kDsCps * P.gu_row, sb = 2 * kDsCps * P.gu_sc;
-  mbar_arrive_expect_tx(&S->full[slot], cb + sb);
-  bulk_g2s(dst, rec + P.lay.gu_codes + static_cast<size_t>(2 * ch0) * P.gu_row, cb, &S->full[slot]);
-  bulk_g2s(dst + cb, rec + P.lay.gu_scales + static_cast<size_t>(2 * ch0) * P.gu_sc, sb, &S->full[slot]);
 }
 
 // Down rows [r0, r1) of one record into dst (codes, then scales).
@@ -962,7 +1046,9 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
   const DSRoute R = ds_route(smem + P.sm_route, np);
   float* wrs = reinterpret_cast<float*>(smem + P.sm_wr);
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem + P.sm_x);
-  int* hq = reinterpret_cast<int*>(smem + P.sm_x);  // the same region after the router
+  // quantised h rows of a round of down stages: the gate/up buffers and the
+  // x staging area behind them (both idle during the down phase)
+  int* hq = reinterpret_cast<int*>(smem + P.sm_gub);
   int* xq = reinterpret_cast<int*>(smem + P.sm_xq);
   float* hs = reinterpret_cast<float*>(smem + P.sm_hs);
   float* zs = reinterpret_cast<float*>(smem + P.sm_zs);
@@ -980,8 +1066,16 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
   const int e1 = split_at(P.E, b + 1, G);
   const int r0 = P.gran * split_at(P.n_units, b, G);
   const int r1 = P.gran * split_at(P.n_units, b + 1, G);
-  const int sb0 = P.has_shared ? (b * nbf + G - 1) / G : 0;
-  const int sb1 = P.has_shared ? ((b + 1) * nbf + G - 1) / G : 0;
+  // gate/up blocks are split among the CTAs by work (h rows x channels):
+  // the shared expert's blocks first (T rows each), then routed expert u's
+  // (n_u rows each); CTA b takes the blocks whose work offset falls in
+  // [W b / G, W (b + 1) / G). W does not depend on the routing, so the
+  // shared-expert share is known before it.
+  const int gu_w = nbf * P.T * (P.k + (P.has_shared ? 1 : 0));
+  const int gu_lo = split_at(gu_w, b, G), gu_hi = split_at(gu_w, b + 1, G);
+  const int sh_w = P.has_shared ? nbf * P.T : 0;
+  const int sb0 = P.has_shared ? min(nbf, (gu_lo + P.T - 1) / P.T) : 0;
+  const int sb1 = P.has_shared ? min(nbf, (gu_hi + P.T - 1) / P.T) : 0;
   const int nsh = sb1 - sb0;
   const bool has_rows = r1 > r0;
   const bool wr_rows = ROUTE && e1 > e0;
@@ -989,7 +1083,7 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
   if (threadIdx.x == 0) {
     for (int i = 0; i < kDsNS; ++i) {
       mbar_init(&S->full[i], 1);
-      mbar_init(&S->empty[i], kDsCps);
+      mbar_init(&S->empty[i], kDsArr);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S->shdn_full[i], 1);
@@ -1057,26 +1151,6 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
       copy_dn(Q, shdn + j * P.dn_stride, rec, r0, r1, &S->shdn_full[j]);
       return true;
     };
-    // the shared expert's gate/up stages of layer l: ring items, one per lane
-    auto issue_shgu = [&](int l) -> bool {
-      const int n = nsh * (32 / kDsCps);
-      bool all = true;
-#pragma unroll 1
-      for (int w0 = 0; w0 < n && all; w0 += P.n_ring) {  // windows of n_ring items, as below
-        const int it = w0 + lane;
-        bool mine = true;
-        if (lane < P.n_ring && it < n) {
-          const uint32_t q = seq + it;
-          mine = slot_ready(q);
-          if (mine)
-            issue_gu(Q, S, ring, q, P.shared + static_cast<size_t>(l) * P.stride,
-                     (sb0 + it / (32 / kDsCps)) * 32 + (it % (32 / kDsCps)) * kDsCps);
-        }
-        all = __all_sync(0xffffffffu, mine);
-      }
-      seq += n;
-      return all;
-    };
     const bool sh_dn = P.has_shared && has_rows;
     // Iteration l issues layer l's routed items (l >= 0), then layer l + 1's
     // inputs that do not depend on its x: router rows, shared-expert down
@@ -1107,12 +1181,7 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
         unsigned long long* td = (trace != nullptr && l == dl && lane == 0) ? trace : nullptr;
         if (td) td[16] = global_timer_ns();
         const int nu = min(max(S->n_uniq, 0), min(np, P.E));
-        const int tot = nu * nbf;
-        const int rb0 = split_at(tot, b, G);
-        const int rb1 = split_at(tot, b + 1, G);
-        const int n_gu = (rb1 - rb0) * (32 / kDsCps);
-        const int n_grp = has_rows ? (nu + P.gpd - 1) / P.gpd : 0;
-        const int n_items = n_gu + n_grp;
+        const int n_items = has_rows ? (nu + P.gpd - 1) / P.gpd : 0;  // down groups
 #pragma unroll 1
         for (int w0 = 0; w0 < n_items && ok; w0 += P.n_ring) {
           const int it = w0 + lane;
@@ -1120,25 +1189,19 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
           if (lane < P.n_ring && it < n_items) {
             const uint32_t q = seq + it;
             mine = slot_ready(q);
+            if (trace != nullptr && l == dl && w0 == 0 && lane < 8) trace[56 + lane] = global_timer_ns();
             if (mine) {
-              if (it < n_gu) {
-                const int blk = rb0 + it / (32 / kDsCps);
-                const int u = fdiv(blk, P.fd_nbf), cb = blk - u * nbf;
-                issue_gu(Q, S, ring, q, P.pool + static_cast<size_t>(R.uniq_slot[u]) * P.stride,
-                         cb * 32 + (it % (32 / kDsCps)) * kDsCps);
-              } else {
-                const int g = it - n_gu;
-                const int u0 = g * P.gpd, u1 = min(nu, u0 + P.gpd);
-                const int slot = fmod_(q, P.fd_ring);
-                uint8_t* dst = ring + static_cast<size_t>(slot) * P.slot_bytes;
-                mbar_arrive_expect_tx(&S->full[slot], (u1 - u0) * (r1 - r0) * (P.dn_row + P.dn_sc));
+              const int u0 = it * P.gpd, u1 = min(nu, u0 + P.gpd);
+              const int slot = fmod_(q, P.fd_ring);
+              uint8_t* dst = ring + static_cast<size_t>(slot) * P.slot_bytes;
+              mbar_arrive_expect_tx(&S->full[slot], (u1 - u0) * (r1 - r0) * (P.dn_row + P.dn_sc));
 #pragma unroll 1
-                for (int u = u0; u < u1; ++u)
-                  copy_dn(Q, dst + (u - u0) * P.dn_stride, P.pool + static_cast<size_t>(R.uniq_slot[u]) * P.stride,
-                          r0, r1, &S->full[slot]);
-              }
+              for (int u = u0; u < u1; ++u)
+                copy_dn(Q, dst + (u - u0) * P.dn_stride, P.pool + static_cast<size_t>(R.uniq_slot[u]) * P.stride,
+                        r0, r1, &S->full[slot]);
             }
           }
+          if (trace != nullptr && l == dl && w0 == 0 && lane < 8) trace[40 + lane] = global_timer_ns();
           ok = __all_sync(0xffffffffu, mine);
           if (td && w0 == 0) td[17] = global_timer_ns();
         }
@@ -1168,7 +1231,6 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
           shdn_count += okn;
         }
         ok = __all_sync(0xffffffffu, okn != 0);
-        if (ok && P.has_shared) ok = issue_shgu(ln);
       }
     }
     if (lane == 0 && !ok && !ds_aborted(S)) ds_abort(S, P.status, 10);
@@ -1195,9 +1257,12 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
     // ============================================================ consumers
     const int tid = threadIdx.x;
     uint32_t seq = 0;
+    // this warp's shared-expert gate/up rows of the next layer, issued ahead
+    int n_pre = (P.has_shared && !ds_aborted(S)) ? gu_prefetch_shared<CW>(Q, 0, nsh, sb0) : 0;
 #pragma unroll 1
     for (int l = 0; l < P.L; ++l) {
       const uint32_t tag = base + 1 + static_cast<uint32_t>(l);
+      const bool publisher = ROUTE && b == l % G;
       // trace slots: 8 phase stamps for layers 0 and 1, then details of
       // layer dl (the second one when there is one)
       const bool traced = trace != nullptr && l < 2 && tid == 0;
@@ -1239,7 +1304,7 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
         named_sync(1, CT);
         if (traced) trace[8 * l + 2] = global_timer_ns();
         // ---- top-k (warp t) and grouping (all)
-        const bool publisher = b == l % G;
+        // (publisher: the CTA that writes this layer's routing record)
         float* pub = publisher ? reinterpret_cast<float*>(P.rec + static_cast<size_t>(l) * P.rec_bytes + P.ro.logits)
                                : nullptr;
         if (warp < P.T && !ds_aborted_warp(S))
@@ -1261,7 +1326,6 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
           mbar_arrive(&S->route_bar);
         }
         if (route_bad) break;  // every consumer thread leaves the layer loop here
-        if (publisher) ds_publish(Q, l, np, nu, CT);
       } else {
         // the grouping was written by moe_group_tokens
         const int nug = min(max(__ldcg(P.g.n_uniq), 0), min(np, P.E));
@@ -1297,14 +1361,14 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
       if (traced) trace[8 * l + 3] = global_timer_ns();
 
       // ---- gate/up + SwiGLU: 32 channel tasks per block, blocks in order
-      const int tot = nu * nbf;
-      const int rb0 = split_at(tot, b, G);
-      const int rb1 = split_at(tot, b + 1, G);
+      const int rb0 = routed_block_at(R, nu, nbf, sh_w, max(gu_lo, sh_w));
+      const int rb1 = routed_block_at(R, nu, nbf, sh_w, max(gu_hi, sh_w));
       const int n_blk = nsh + (rb1 - rb0);
       if (!ds_aborted_warp(S))
-        gu_phase<BITS, GBPL, CW>(Q, S, nsh, sb0, rb0, n_blk, seq, deadline, (tdet && warp == 0) ? tdet : nullptr);
+        gu_phase<BITS, GBPL, CW>(Q, S, l, nsh, sb0, rb0, n_blk, n_pre, (tdet && warp == 0) ? tdet : nullptr);
+      else
+        asm volatile("cp.async.wait_all;" ::: "memory");
       if (tdet && tid == 0) tdet[23] = global_timer_ns();
-      seq += n_blk * (32 / kDsCps);
       named_sync(1, CT);
       // every block's 32 channels are in hs: requantise and publish them
       if (!ds_aborted(S)) {
@@ -1316,11 +1380,11 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
         }
       }
       named_sync(1, CT);
-      // every CTA counts its h blocks as written, then waits for all
-      if (tid == 0) {
-        cnt_add(kCntH);
-        if (!ds_aborted(S)) cnt_wait(kCntH, (base + l + 1) * G, S, P.status, 23, deadline);
-      }
+      // every CTA counts its h blocks as written, then waits for all; the
+      // publishing CTA writes the layer's routing record meanwhile
+      if (tid == 0) cnt_add(kCntH);
+      if (publisher) ds_publish(Q, l, np, nu, CT);
+      if (tid == 0 && !ds_aborted(S)) cnt_wait(kCntH, (base + l + 1) * G, S, P.status, 23, deadline);
       named_sync(1, CT);
       if (traced) trace[8 * l + 4] = global_timer_ns();
 
@@ -1396,7 +1460,7 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
               // group has no expert for
               const int g0 = fdiv(u, P.fd_gpd) * P.gpd;
               const int m = min(nu - g0, P.gpd);
-              mbar_arrive_cnt(&S->empty[slot], u == g0 ? kDsCps - (m - 1) : 1);
+              mbar_arrive_cnt(&S->empty[slot], u == g0 ? kDsArr - (m - 1) : 1);
             }
           }
         }
@@ -1405,6 +1469,9 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
       }
       seq += has_rows ? (nu + P.gpd - 1) / P.gpd : 0;
       if (traced) trace[8 * l + 6] = global_timer_ns();
+      // the down phase is done with the buffers: this warp's shared-expert
+      // gate/up rows of the next layer go in now
+      n_pre = (l + 1 < P.L && P.has_shared && !ds_aborted_warp(S)) ? gu_prefetch_shared<CW>(Q, l + 1, nsh, sb0) : 0;
 
       // ---- combine: y[t, r] = sum_j gate[t,j] z[(t,j)][r] + z_shared[t][r] (+ x)
       if (!ds_aborted(S) && has_rows) {
@@ -1450,6 +1517,7 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
       if (traced) trace[8 * l + 7] = global_timer_ns();
     }
     if (P.L == 1 && tid == 0) grid_dep_launch();
+    asm volatile("cp.async.wait_all;" ::: "memory");  // a layer given up may leave copies in flight
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -1652,12 +1720,11 @@ cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const St
   P.n_units = c.d / gran;
   P.rpc = gran * ((P.n_units + G - 1) / G);
   const int wr_rows = a.route ? (c.E + G - 1) / G : 0;
-  // ring slots hold one gate/up stage (16 channels) or a group of down
-  // stages (this CTA's output rows of up to gpd experts)
-  const size_t gu_stage = static_cast<size_t>(2 * kDsCps) * (P.gu_row + P.gu_sc);
+  // ring slots hold a group of down stages (this CTA's output rows of up to
+  // kDsGpd experts); a gate/up task is the two rows of one channel
   P.dn_stride = static_cast<int>(ds_align(static_cast<size_t>(P.rpc) * (P.dn_row + P.dn_sc), 16));
-  P.slot_bytes = static_cast<int>(ds_align(gu_stage > static_cast<size_t>(P.dn_stride) ? gu_stage : P.dn_stride, 128));
-  P.gpd = P.slot_bytes / P.dn_stride;
+  P.gu_task_bytes = static_cast<int>(ds_align(2 * static_cast<size_t>(P.gu_row + P.gu_sc), 128));
+  if ((2 * P.gu_row) % 16 != 0 || (2 * P.gu_sc) % 16 != 0) return cudaErrorNotSupported;
   // shared-memory map
   size_t o = ds_align(sizeof(DSShared), 128);
   P.sm_route = static_cast<int>(o);
@@ -1668,11 +1735,13 @@ cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const St
   o = ds_align(o + static_cast<size_t>(T) * P.rpc * 4, 128);
   P.sm_hs = static_cast<int>(o);
   const int nu_max0 = np < c.E ? np : c.E;
-  // the kernel splits items among the CTAs in 32-bit arithmetic
-  if (static_cast<long long>(nu_max0) * nbf * G >= (1ll << 31) ||
+  // gate/up work (h rows x channel blocks) split among the CTAs in 32-bit
+  // arithmetic; a CTA's blocks start at distinct work offsets of its share
+  const long long gu_w = static_cast<long long>(nbf) * T * (c.k + (a.shared != nullptr ? 1 : 0));
+  if (static_cast<long long>(nu_max0) * nbf * G >= (1ll << 31) || gu_w * G >= (1ll << 31) ||
       static_cast<long long>(c.E > P.n_units ? c.E : P.n_units) * G >= (1ll << 31))
     return cudaErrorNotSupported;
-  P.max_blk = (nu_max0 * nbf + G - 1) / G + (nbf + G - 1) / G;
+  P.max_blk = static_cast<int>((gu_w + G - 1) / G);
   if (P.max_blk > kDsMaxBlk) return cudaErrorNotSupported;
   const size_t hs_bytes = static_cast<size_t>(P.max_blk) * T * 32 * 4;
   o = ds_align(o + hs_bytes, 128);
@@ -1682,31 +1751,45 @@ cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const St
   o = ds_align(o + static_cast<size_t>(wr_rows) * c.d * 4, 128);
   P.sm_shdn = static_cast<int>(o);
   o = ds_align(o + 2 * static_cast<size_t>(P.dn_stride), 128);
-  P.sm_x = static_cast<int>(o);
-  const size_t fixed = o;
-  // the staging area: raw x for the router, the top-k key rows, then the
-  // quantised h rows of a round of down stages (all rows if they fit in
-  // 48 KB, else 48 KB worth, at least T rows); at least three ring slots,
-  // for which the h rows give way down to their minimum
+  const size_t before_gub = o;
+  // then the per-warp gate/up buffers, the staging area and the ring. The
+  // staging area holds raw x for the router, then the top-k key rows; the
+  // gate/up buffers and the staging area together hold the quantised h rows
+  // of a round of down stages (at least T rows). The first of (gate/up
+  // depth, experts per down group) from (4, 6) down to (2, 1) that leaves
+  // room for two ring slots wins.
   const size_t xs_bytes = a.route ? static_cast<size_t>(T) * c.d * 2 : 0;
   const size_t hq_row = static_cast<size_t>(kQW) * nbf * 4;
-  const size_t keys_bytes = static_cast<size_t>(T) * c.E * 4;  // top-k key rows (after the router)
+  const size_t keys_bytes = static_cast<size_t>(T) * c.E * 4;
   size_t x_min = xs_bytes > keys_bytes ? xs_bytes : keys_bytes;
   if (x_min < T * hq_row) x_min = T * hq_row;
-  size_t hq_bytes = static_cast<size_t>(n_rows) * hq_row;
-  if (hq_bytes > 48 * 1024) hq_bytes = 48 * 1024;
-  size_t x_bytes = ds_align(x_min > hq_bytes ? x_min : hq_bytes, 128);
-  auto ring_slots = [&](size_t xb) {
-    const long long r = static_cast<long long>(kDsSmemMax) - static_cast<long long>(ds_align(fixed + xb, 128));
-    return r > 0 ? static_cast<int>(r / P.slot_bytes) : 0;
-  };
-  if (ring_slots(x_bytes) < 3) x_bytes = ds_align(x_min, 128);
-  P.hq_rows = static_cast<int>(x_bytes / hq_row);
+  int n_ring = 0;
+  size_t fixed = 0, x_bytes = 0;
+  for (int depth = kDsGuDepth; depth >= 2 && n_ring < 2; --depth) {
+    for (int gpd : {kDsGpd, 4, 2, 1}) {
+      const int slot_bytes = static_cast<int>(ds_align(static_cast<size_t>(gpd) * P.dn_stride, 128));
+      fixed = ds_align(before_gub + static_cast<size_t>(CW) * depth * P.gu_task_bytes, 128);
+      auto ring_slots = [&](size_t xb) {
+        const long long r = static_cast<long long>(kDsSmemMax) - static_cast<long long>(ds_align(fixed + xb, 128));
+        return r > 0 ? static_cast<int>(r / slot_bytes) : 0;
+      };
+      x_bytes = ds_align(x_min, 128);
+      n_ring = ring_slots(x_bytes);
+      if (n_ring >= 2) {
+        P.gu_depth = depth;
+        P.slot_bytes = slot_bytes;
+        P.gpd = slot_bytes / P.dn_stride;
+        break;
+      }
+    }
+  }
+  if (n_ring < 2) return cudaErrorNotSupported;
+  if (n_ring > kDsNS) n_ring = kDsNS;
+  P.sm_gub = static_cast<int>(before_gub);
+  P.sm_x = static_cast<int>(fixed);
+  P.hq_rows = static_cast<int>((fixed - before_gub + x_bytes) / hq_row);
   if (P.hq_rows > n_rows) P.hq_rows = n_rows;
   o = ds_align(fixed + x_bytes, 128);
-  int n_ring = ring_slots(x_bytes);
-  if (n_ring > kDsNS) n_ring = kDsNS;
-  if (n_ring < 3) return cudaErrorNotSupported;
   P.n_ring = n_ring;
   P.fd_ring = make_fastdiv(n_ring);
   P.fd_hrow = make_fastdiv(nbf * (kQW / 2));
