@@ -154,8 +154,8 @@ MOE_API moe_status moe_check_device_status(moe_ctx* ctx, moe_stream stream);
 MOE_API int moe_last_device_error_detail(const moe_ctx* ctx);
 
 /* Diagnostics: when the environment variable MOE_TRACE is set at context
- * creation, the decode-layer kernel records the global-timer value (ns) at
- * its phase boundaries, 32 slots per CTA. This copies up to n values (CTA
+ * creation, the decode kernel records the global-timer value (ns) at its
+ * phase boundaries, 64 slots per CTA. This copies up to n values (CTA
  * major) into host memory, synchronising `stream`, and clears the record.
  * Returns MOE_EINVAL if tracing is off. */
 MOE_API moe_status moe_trace_fetch(moe_ctx* ctx, unsigned long long* host, int n, moe_stream stream);
@@ -180,7 +180,13 @@ MOE_API moe_status moe_router_topk(moe_ctx* ctx, const moe_layer_cfg* cfg, const
                            const float* w_router, const float* logit_bias, int T,
                            float* logits, int32_t* idx, float* gate, moe_stream stream);
 
-/* Top-k and gates from given fp32 logits [T, E] (the selection step alone). */
+/* Top-k and gates from given fp32 logits [T, E] (the selection step alone):
+ * each token keeps the k largest of its E logits, 10 of 512 at full size
+ * (news.blueqat.app/post/3262, first section Strataとは; geekoyaji.com
+ * "freetoken-vs-strata-moe-offload", section 共通の仕組み). Ties go to the
+ * lower expert index; NaN ranks below every number. idx [T, k] int32 in
+ * descending-logit order, gate [T, k] fp32 (softmax over the k chosen, or the
+ * full softmax when cfg->renorm == 0). T = 0 is a no-op. */
 MOE_API moe_status moe_topk(moe_ctx* ctx, const moe_layer_cfg* cfg, const float* logits, int T,
                     int32_t* idx, float* gate, moe_stream stream);
 
@@ -195,7 +201,12 @@ MOE_API moe_status moe_group_tokens(moe_ctx* ctx, const moe_layer_cfg* cfg, cons
                             void* ws, size_t ws_bytes, moe_grouping* out, moe_stream stream);
 
 /* Expert FFN over 2-bit (q2) or 3-bit (q3) records: for every sorted pair and
- * every shared-expert row, h = silu(W_g x) * (W_u x) and z = W_d h.
+ * every shared-expert row, h = silu(W_g x) * (W_u x) and z = W_d h, with the
+ * weights dequantised inside the kernels. The pages put the experts at 2 to
+ * 3 bits per weight (news.blueqat.app/post/3262, section 量子化の種類とサイズ)
+ * and run the shared expert on the GPU for every token (same page, section
+ * GPU・CPU・RAM・SSDの分担); the SwiGLU form is the one the pages' model family
+ * uses and is not printed there.
  * slot_pool: base of the pool (256-byte aligned), slot_stride: bytes between
  * slots (a multiple of 256, >= the record size); shared_expert: one record or
  * NULL when cfg->n_shared == 0; ws: the workspace the grouping came from.
@@ -220,9 +231,14 @@ MOE_API moe_status moe_expert_ffn_q3(moe_ctx* ctx, const moe_layer_cfg* cfg, con
 MOE_API moe_status moe_combine(moe_ctx* ctx, const moe_layer_cfg* cfg, const moe_grouping* grouping,
                        const float* z_rows, const void* x, int T, void* y, moe_stream stream);
 
-/* The whole step: router -> top-k -> grouping -> experts -> combine. Picks the
- * decode path for T <= MOE_DECODE_MAX_T and the tensor-core grouped GEMM path
- * otherwise. Arguments as above; ws must hold moe_workspace_bytes(cfg, T). */
+/* The whole step: router -> top-k -> grouping -> experts -> combine, the
+ * per-layer expert step of the pages' engine (news.blueqat.app/post/3262,
+ * sections Strataとは and GPU・CPU・RAM・SSDの分担). Picks the decode path for
+ * T <= MOE_DECODE_MAX_T (decode passes of up to 4 tokens: vramglass.com,
+ * section その3) and the tensor-core grouped GEMM path otherwise (prefill
+ * chunks of up to 8,192 tokens: news.blueqat.app, section
+ * GPU・CPU・RAM・SSDの分担). Arguments as above; ws must hold
+ * moe_workspace_bytes(cfg, T). */
 MOE_API moe_status moe_layer_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, const void* x, int T,
                              const float* w_router, const float* logit_bias,
                              const int32_t* slot_of, int n_slots, const uint8_t* slot_pool,
