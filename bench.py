@@ -470,6 +470,48 @@ def stack_record(st, ms_total, steps, first, hbm, world):
     }
 
 
+def residency_record(st, pool, every=32, max_swaps=256):
+    """The hot set under the drifting T=4 stream: moe_usage_count after every
+    step, and every `every` steps the plan_swaps exchanges (at most
+    max_swaps) carried out by moe_slot_swap; the share of routed pairs whose
+    expert sits in the pool's first `hot` slots, static table vs adapted, and
+    the exchange cost. Counts halve at each adaptation (a sliding window)."""
+    import torch
+    from bit_expert_ffn_router_b200 import residency as R
+    M, cfg, ctx = st.M, st.cfg, st.ctx
+    L, E, T, n_hot = st.L, cfg.E, st.T, pool["hot"]
+    table = pool["slot_of"].view(-1)
+    static = table.cpu().numpy().copy()
+    cur = static.copy()
+    counts = torch.zeros(L * E, dtype=torch.int32, device="cuda")
+    hit_s = hit_a = 0.0
+    n_sw, sw_ms = 0, 0.0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for s in range(st.S):
+        st.step(s)
+        ctx.usage_count(cfg, L, T, st.ws, counts)
+        ex = [st.sets[s, l].reshape(-1) for l in range(L)]
+        hit_s += R.hot_hit_rate(ex, static, E, n_hot)
+        hit_a += R.hot_hit_rate(ex, cur, E, n_hot)
+        if s % every == every - 1:
+            a, b = R.plan_swaps(counts.cpu().numpy(), cur, n_hot, max_swaps=max_swaps)
+            e0.record()
+            ctx.slot_swap(cfg, pool["pool"], pool["stride"], table, pool["n_slots"], a, b)
+            e1.record()
+            torch.cuda.synchronize()
+            sw_ms += e0.elapsed_time(e1)
+            n_sw += a.size
+            cur = R.apply_swaps(cur, a, b)
+            counts //= 2
+    assert ctx.check_device_status() == M.OK
+    assert np.array_equal(table.cpu().numpy(), cur)
+    rec = pool["lay"]["bytes"]
+    return {"hot_slots": int(n_hot), "steps": int(st.S), "adapt_every": every,
+            "hot_hit_rate_static": round(hit_s / st.S, 4), "hot_hit_rate_adaptive": round(hit_a / st.S, 4),
+            "swaps": int(n_sw), "swap_us_each": round(sw_ms * 1e3 / max(n_sw, 1), 2),
+            "swap_gbs": round(4 * rec * n_sw / max(sw_ms, 1e-9) / 1e6, 1)}
+
+
 def layer_call_record(st, steps, world):
     """The same stack as L separate moe_layer_forward launches (one CUDA graph
     per step): the single-layer entry point's speed."""
@@ -610,6 +652,7 @@ def run_extras(args, pool2, st1, world, local, hbm, tf):
     st4 = DecodeStack(pool2, T=4, steps=256, keep=7)
     ms, clk = time_steps(st4, 256, 3, world, local)
     out["stack_t4_correlated_q2"] = {**stack_record(st4, ms, 256, 3, hbm, world), "steps": 256, "clocks": clk}
+    out["residency_t4_correlated_q2"] = residency_record(st4, pool2)
     del st4, st1
     torch.cuda.empty_cache()
     for k in ("pool", "shared", "wr"):

@@ -17,7 +17,7 @@ LIB = os.path.join(LIBDIR, "libmoe.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 SOURCES = ["moe_api.cu", "router.cu", "router_tc.cu", "group.cu", "decode_stack.cu", "ffn_prefill.cu",
-           "combine.cu", "noalloc.cu"]
+           "combine.cu", "noalloc.cu", "residency.cu"]
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -1,8 +1,10 @@
 // C ABI of libmoe: argument checks, workspace carving and kernel launches.
 // Every compute entry point is asynchronous on the caller's stream and
 // allocates nothing; see include/moe.h for the contract of each call.
+#include <algorithm>
 #include <cstdlib>
 #include <new>
+#include <vector>
 
 #include "moe_internal.cuh"
 
@@ -420,6 +422,61 @@ moe_status moe_stack_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, int L, cons
   if ((st = check_pool(*cfg, slot_pool, slot_stride, shared_experts)) != MOE_OK) return st;
   return run_stack(ctx, *cfg, L, x, T, w_router, logit_bias, slot_of, n_slots, slot_pool, slot_stride,
                    shared_experts, ws, y, stream);
+}
+
+moe_status moe_usage_count(moe_ctx* ctx, const moe_layer_cfg* cfg, int L, int T, const void* ws, size_t ws_bytes,
+                           int32_t* counts, moe_stream stream) {
+  if (ctx == nullptr) return MOE_EINVAL;
+  DeviceGuard dg(ctx->c.device);
+  if (!dg.ok) return MOE_ECUDA;
+  const moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (L < 1 || T < 0 || (L > 1 && T > MOE_DECODE_MAX_T)) return MOE_EINVAL;
+  if (ws == nullptr || !aligned(ws, 256) || counts == nullptr || !aligned(counts, 4)) return MOE_EINVAL;
+  const WsLayout w = ws_layout(*cfg, T);
+  if (ws_bytes < static_cast<size_t>(L - 1) * w.rec_bytes + w.rec_bytes) return MOE_ENOSPACE;
+  if (T == 0) return MOE_OK;
+  return from_cuda(launch_usage_count(ctx->c, static_cast<const char*>(ws), w.rec_bytes, w.expert_count, L,
+                                      cfg->E, counts, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_slot_swap(moe_ctx* ctx, const moe_layer_cfg* cfg, uint8_t* slot_pool, size_t slot_stride,
+                         int32_t* slot_of, int n_entries, int n_slots, const int32_t* a, const int32_t* b, int n,
+                         moe_stream stream) {
+  if (ctx == nullptr) return MOE_EINVAL;
+  DeviceGuard dg(ctx->c.device);
+  if (!dg.ok) return MOE_ECUDA;
+  const moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (n < 0 || n_entries <= 0 || n_slots <= 0) return MOE_EINVAL;
+  if (n == 0) return MOE_OK;
+  if (slot_pool == nullptr || slot_of == nullptr || a == nullptr || b == nullptr) return MOE_EINVAL;
+  const size_t rec = layout_of(*cfg).bytes;
+  if (!aligned(slot_pool, 256) || !aligned(slot_of, 4) || slot_stride % 256 != 0 || slot_stride < rec)
+    return MOE_EINVAL;
+  // every entry in range, the 2n entries distinct (each exchange owns its two slots)
+  std::vector<int32_t> all;
+  all.reserve(2 * static_cast<size_t>(n));
+  for (int i = 0; i < n; ++i) {
+    if (a[i] < 0 || a[i] >= n_entries || b[i] < 0 || b[i] >= n_entries) return MOE_EINVAL;
+    all.push_back(a[i]);
+    all.push_back(b[i]);
+  }
+  std::sort(all.begin(), all.end());
+  if (std::adjacent_find(all.begin(), all.end()) != all.end()) return MOE_EINVAL;
+  for (int i0 = 0; i0 < n; i0 += kSwapBatch) {
+    SwapBatch batch;
+    const int m = std::min(kSwapBatch, n - i0);
+    for (int i = 0; i < m; ++i) {
+      batch.a[i] = a[i0 + i];
+      batch.b[i] = b[i0 + i];
+    }
+    for (int i = m; i < kSwapBatch; ++i) batch.a[i] = batch.b[i] = 0;
+    const cudaError_t e = launch_slot_swaps(ctx->c, slot_pool, slot_stride, rec, slot_of, n_slots, batch, m,
+                                            static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  return MOE_OK;
 }
 
 moe_status moe_expert_layout_get(const moe_layer_cfg* cfg, moe_expert_layout* out) {

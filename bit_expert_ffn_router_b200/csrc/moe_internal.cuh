@@ -215,6 +215,16 @@ cudaError_t launch_combine(const Ctx& ctx, const moe_layer_cfg& c, const int32_t
                            int n_pairs, const float* z_rows, const uint16_t* x, int T, void* y,
                            cudaStream_t s);
 
+// residency.cu: usage tallies and slot exchanges
+constexpr int kSwapBatch = 64;  // exchanges per launch (passed by value)
+struct SwapBatch {
+  int32_t a[kSwapBatch], b[kSwapBatch];  // slot-table entries whose slots trade places
+};
+cudaError_t launch_usage_count(const Ctx& ctx, const char* ws, size_t rec_bytes, size_t count_off, int L, int E,
+                               int32_t* counts, cudaStream_t s);
+cudaError_t launch_slot_swaps(const Ctx& ctx, uint8_t* pool, size_t stride, size_t record_bytes, int32_t* slot_of,
+                              int n_slots, const SwapBatch& batch, int n, cudaStream_t s);
+
 // kernel attribute set-up, once per context
 cudaError_t decode_init(Ctx& ctx);
 cudaError_t router_init(const Ctx& ctx);

@@ -101,6 +101,8 @@ _SIGS = {
     "moe_stack_forward": (_I, [_P, ctypes.POINTER(_Cfg), _I, _P, _I, _P, _P, _P, _I, _P, _Z, _P, _P, _Z, _P, _S]),
     "moe_stack_routing": (_I, [ctypes.POINTER(_Cfg), _I, _I, _P, _Z, _I, ctypes.POINTER(Routing)]),
     "moe_layer_forward_static": (_I, [_P, ctypes.POINTER(_Cfg), _P, _I, _P, _P, _P, _I, _P, _Z, _P, _P, _S]),
+    "moe_usage_count": (_I, [_P, ctypes.POINTER(_Cfg), _I, _I, _P, _Z, _P, _S]),
+    "moe_slot_swap": (_I, [_P, ctypes.POINTER(_Cfg), _P, _Z, _P, _I, _I, _P, _P, _I, _S]),
 }
 
 _lib = None
@@ -238,6 +240,30 @@ class Context:
                               stream=None) -> "PreparedLayer":
         """moe_layer_forward with every argument but x and y marshalled once (for launch loops)."""
         return PreparedLayer(self, cfg, T, w_router, bias, slot_of, n_slots, pool, stride, shared, ws, stream)
+
+    def usage_count_status(self, cfg, L, T, ws, counts, stream=None) -> int:
+        return self.lib.moe_usage_count(self.h, ctypes.byref(cfg.c()), L, T, _ptr(ws),
+                                        ws.numel() * ws.element_size(), _ptr(counts), _stream(stream))
+
+    def usage_count(self, cfg, L, T, ws, counts, stream=None) -> None:
+        """moe_usage_count: counts [L*E] int32 (device) += pairs routed to each expert by the call that
+        used ws (L = 1 for a single-layer workspace)."""
+        _check(self.usage_count_status(cfg, L, T, ws, counts, stream), "moe_usage_count")
+
+    def slot_swap_status(self, cfg, pool, stride, slot_of, n_slots, a, b, stream=None) -> int:
+        import numpy as np
+        a = np.ascontiguousarray(a, dtype=np.int32)
+        b = np.ascontiguousarray(b, dtype=np.int32)
+        if a.shape != b.shape or a.ndim != 1:
+            return EINVAL
+        return self.lib.moe_slot_swap(self.h, ctypes.byref(cfg.c()), _ptr(pool), stride, _ptr(slot_of),
+                                      slot_of.numel(), n_slots, a.ctypes.data, b.ctypes.data, a.size,
+                                      _stream(stream))
+
+    def slot_swap(self, cfg, pool, stride, slot_of, n_slots, a, b, stream=None) -> None:
+        """moe_slot_swap: the records at slots slot_of[a[i]] and slot_of[b[i]] trade places, and so
+        do the two table entries (a, b: host index arrays into the flat device table slot_of)."""
+        _check(self.slot_swap_status(cfg, pool, stride, slot_of, n_slots, a, b, stream), "moe_slot_swap")
 
     def layer_routing(self, cfg, T, ws, stack_layers=None, layer=0) -> dict:
         """The routing a whole-step call with workspace `ws` computed (moe_layer_routing; with

@@ -300,6 +300,39 @@ MOE_API moe_status moe_stack_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, int
 MOE_API moe_status moe_stack_routing(const moe_layer_cfg* cfg, int L, int T, void* ws, size_t ws_bytes,
                                      int layer, moe_routing* out);
 
+/* ---- expert residency --------------------------------------------------- */
+
+/* The pages' engine keeps its most used experts in GPU memory, picked from
+ * usage statistics and swapped as a conversation goes on (vramglass.com,
+ * section その1：よく使うエキスパートを選んでGPUに置く; news.blueqat.app/post/3262,
+ * section GPU・CPU・RAM・SSDの分担). Here the pool's first slots stand for that
+ * hot set; these two calls tally usage and move records between slots.
+ *
+ * moe_usage_count: counts[l * E + e] += the number of (token, j) pairs routed
+ * to expert e in layer l by the call whose workspace is ws, once that call
+ * has completed on `stream`'s order: L = 1 for a moe_layer_forward (or
+ * moe_router_topk + moe_group_tokens) workspace at T tokens, L layers for a
+ * moe_stack_forward workspace (T <= MOE_DECODE_MAX_T). counts: [L, E] int32
+ * device array; integer adds in a fixed owner per element, so the tallies are
+ * exact and deterministic.
+ *
+ * moe_slot_swap: for i < n, the records at slots slot_of[a[i]] and
+ * slot_of[b[i]] trade places in the pool and the two slot-table entries trade
+ * values, so every entry still names its own expert's record and later calls
+ * give the same results bit for bit. a, b: HOST arrays of n indices into the
+ * device slot table slot_of (n_entries entries, e.g. L * E); the 2n indices
+ * must be distinct and in range (MOE_EINVAL otherwise), and the slots they
+ * name distinct as well (true when no two entries share a slot, as in a pool
+ * with one record per layer and expert; not checked). A slot outside
+ * [0, n_slots) found on the device is reported as MOE_EDEVICE and that pair is
+ * left alone. Calls that read the pool or the table must be ordered after this
+ * one (same stream). */
+MOE_API moe_status moe_usage_count(moe_ctx* ctx, const moe_layer_cfg* cfg, int L, int T, const void* ws,
+                                   size_t ws_bytes, int32_t* counts, moe_stream stream);
+MOE_API moe_status moe_slot_swap(moe_ctx* ctx, const moe_layer_cfg* cfg, uint8_t* slot_pool, size_t slot_stride,
+                                 int32_t* slot_of, int n_entries, int n_slots, const int32_t* a, const int32_t* b,
+                                 int n, moe_stream stream);
+
 /* moe_layer_forward without a workspace argument: the step's scratch is a
  * static device array of MOE_STATIC_SCRATCH_BYTES inside the library image,
  * reserved on each device when the library's module loads there, so the call
