@@ -470,6 +470,43 @@ def stack_record(st, ms_total, steps, first, hbm, world):
     }
 
 
+def skip_record(st, pool, skip_from, steps=20):
+    """The stack with low-ranked non-resident pairs left out (rank >= skip_from,
+    slot >= the pool's hot slots): time per layer, the share of pairs left out,
+    and the drift of the layer outputs from the plain stack's (relative L2 per
+    token of y[l] = x_l + moe(x_l); layer 0 shows one step's effect, the last
+    layer the effect compounded over the stack)."""
+    import torch
+    M, L, T = st.M, st.L, st.T
+    cfg = st.cfg.replace(skip_from=skip_from, hot_slots=pool["hot"])
+    call = st.ctx.prepare_stack_forward(cfg, L, T, pool["wr"], pool["slot_of"], pool["n_slots"], pool["pool"],
+                                        pool["stride"], pool["shared"], st.ws)
+    plain = st.step(0).clone().float()
+    y = torch.empty_like(st.y)
+    for _ in range(3):
+        call(st.x0, st.bias[0], y)
+    torch.cuda.synchronize()
+    left = [float((st.ctx.layer_routing(cfg, T, st.ws, stack_layers=L, layer=l)["pair_pos"] < 0).float().mean())
+            for l in range(L)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        call(st.x0, st.bias[0], y)
+    e1.record()
+    torch.cuda.synchronize()
+    assert st.ctx.check_device_status() == M.OK
+    ms = e0.elapsed_time(e1) / steps
+    d = ((y.float() - plain).norm(dim=-1) / plain.norm(dim=-1)).cpu().numpy()  # [L, T]
+    fin = np.isfinite(plain.cpu().numpy()).all(axis=(1, 2))
+    n_fin = int(np.argmin(fin)) if not fin.all() else L  # the synthetic stream may overflow deep in the stack
+    last = max(n_fin - 1, 0)
+    return {"skip_from": skip_from, "hot_slots": int(pool["hot"]), "layer_us": round(ms * 1e3 / L, 3),
+            "pairs_left_out": round(float(np.mean(left)), 4), "finite_layers": n_fin,
+            "rel_drift_layer0": float(f"{d[0].max():.3g}"),
+            "rel_drift_last_finite_layer": float(f"{d[last].max():.3g}"),
+            "rel_drift_max_finite": float(f"{d[:max(n_fin, 1)].max():.3g}")}
+
+
 def residency_record(st, pool, every=32, max_swaps=256):
     """The hot set under the drifting T=4 stream: moe_usage_count after every
     step, and every `every` steps the plan_swaps exchanges (at most
@@ -649,6 +686,7 @@ def run_extras(args, pool2, st1, world, local, hbm, tf):
     import torch
     out = {}
     out["layer_calls_t1"] = layer_call_record(st1, 20, world)
+    out["skip_t1_q2"] = skip_record(st1, pool2, skip_from=6)
     st4 = DecodeStack(pool2, T=4, steps=256, keep=7)
     ms, clk = time_steps(st4, 256, 3, world, local)
     out["stack_t4_correlated_q2"] = {**stack_record(st4, ms, 256, 3, hbm, world), "steps": 256, "clocks": clk}

@@ -92,6 +92,7 @@ struct RecOff {
 struct DSParams {
   const uint16_t* x;            // [T, d] bf16: layer 0's input
   int T, d, f, E, k, L, renorm, residual, has_shared, out_f32;
+  int skip_from, hot_slots;  // pairs of rank >= skip_from on a slot >= hot_slots are left out (skip_from > 0)
   const float* wr;              // route: [L, E, d]
   const float* bias;            // route: null or [L, T, E]
   const int32_t* slot_of;       // route: [L, E]
@@ -534,48 +535,65 @@ __device__ __noinline__ void ds_topk(const DSParams& P, int t, uint32_t tag, flo
     R.gate[t * P.k + lane] = ex / denom;
   }
   if (P.T == 1) {
-    // one token: its k experts are distinct, so the grouping is their order
-    // by expert index, found here by ranks instead of a CTA-wide sort
-    int pos = 0;
-#pragma unroll 4
-    for (int j = 0; j < 32; ++j) {
-      const int ej = __shfl_sync(0xffffffffu, mine_e, j);
-      pos += (j < P.k && ej < mine_e) ? 1 : 0;
-    }
+    // one token: its k experts are distinct, so the grouping is the order of
+    // the kept ones by expert index, found here by ranks instead of a
+    // CTA-wide sort
+    int slot = 0;
     if (sel) {
-      int slot = R.slot_s[min(max(mine_e, 0), P.E - 1)];
+      slot = R.slot_s[min(max(mine_e, 0), P.E - 1)];
       if (slot < 0 || slot >= P.n_slots) {
         report(P.status, kDevBadSlot, mine_e);
         slot = 0;
       }
+    }
+    const bool keep = sel && !(P.skip_from > 0 && lane >= P.skip_from && slot >= P.hot_slots);
+    const unsigned kept = __ballot_sync(0xffffffffu, keep);
+    int pos = 0;
+#pragma unroll 4
+    for (int j = 0; j < 32; ++j) {
+      const int ej = __shfl_sync(0xffffffffu, mine_e, j);
+      pos += (((kept >> j) & 1u) != 0u && ej < mine_e) ? 1 : 0;
+    }
+    if (sel) R.pair_pos[lane] = keep ? pos : -1;
+    if (keep) {
       R.sorted_e[pos] = mine_e;
       R.pair_token[pos] = 0;
       R.pair_gate[pos] = ex / denom;
-      R.pair_pos[lane] = pos;
       R.uniq_e[pos] = mine_e;
       R.uniq_slot[pos] = slot;
       R.uniq_off[pos] = pos;
     }
     if (lane == 0) {
-      R.uniq_off[P.k] = P.k;
-      S->n_uniq = P.k;
+      const int n = __popc(kept);
+      R.uniq_off[n] = n;
+      S->n_uniq = n;
     }
   }
 }
 
 // Stable sort of the T*k pairs by expert in shared memory, the unique
 // experts and their slots. Every consumer thread takes part.
+// Pair p = t * k + j stays unless skipping is on, its rank j >= skip_from
+// and its expert's slot is not resident.
+__device__ __forceinline__ bool ds_keep_pair(const DSParams& P, const DSRoute& R, int p, int e) {
+  return P.skip_from == 0 || p % P.k < P.skip_from || R.slot_s[e] < P.hot_slots;
+}
+
 __device__ __noinline__ void ds_group(const DSParams& P, DSShared* S, int np, int CT) {
   const DSRoute R = ds_route(ds_smem + P.sm_route, np);
   const int tid = threadIdx.x;
 #pragma unroll 1
   for (int p = tid; p < np; p += CT) {
     const int e = min(max(R.idx[p], 0), P.E - 1);
+    if (!ds_keep_pair(P, R, p, e)) {
+      R.pair_pos[p] = -1;
+      continue;
+    }
     int pos = 0;
 #pragma unroll 1
     for (int q = 0; q < np; ++q) {
       const int eq = min(max(R.idx[q], 0), P.E - 1);
-      pos += (eq < e) || (eq == e && q < p);
+      pos += ((eq < e) || (eq == e && q < p)) && ds_keep_pair(P, R, q, eq);
     }
     R.sorted_e[pos] = e;
     R.pair_token[pos] = p / P.k;
@@ -584,11 +602,18 @@ __device__ __noinline__ void ds_group(const DSParams& P, DSShared* S, int np, in
   }
   named_sync(1, CT);
   if (tid < 32) {
-    int base = 0;
+    int n_kept = 0;  // the sorted pairs
 #pragma unroll 1
     for (int c = 0; c < np; c += 32) {
+      const int q = c + tid;
+      const bool k = q < np && ds_keep_pair(P, R, q, min(max(R.idx[q], 0), P.E - 1));
+      n_kept += __popc(__ballot_sync(0xffffffffu, k));
+    }
+    int base = 0;
+#pragma unroll 1
+    for (int c = 0; c < n_kept; c += 32) {
       const int i = c + tid;
-      const bool first = i < np && (i == 0 || R.sorted_e[i - 1] != R.sorted_e[i]);
+      const bool first = i < n_kept && (i == 0 || R.sorted_e[i - 1] != R.sorted_e[i]);
       const unsigned m = __ballot_sync(0xffffffffu, first);
       if (first) {
         const int u = base + __popc(m & ((1u << tid) - 1u));
@@ -605,7 +630,7 @@ __device__ __noinline__ void ds_group(const DSParams& P, DSShared* S, int np, in
       base += __popc(m);
     }
     if (tid == 0) {
-      R.uniq_off[base] = np;
+      R.uniq_off[base] = n_kept;
       S->n_uniq = base;
     }
   }
@@ -631,13 +656,14 @@ __device__ __noinline__ void ds_publish(const DSParams& P, int l, int np, int nu
   const int tid = threadIdx.x;
 #pragma unroll 1
   for (int q = tid; q < np; q += CT) {
-    const int pos = R.pair_pos[q];
+    const int pos = R.pair_pos[q];  // -1: a pair left out
     const int e = min(max(R.idx[q], 0), P.E - 1);
     int slot = R.slot_s[e];
     if (slot < 0 || slot >= P.n_slots) slot = 0;
     idx[q] = R.idx[q];
     gate[q] = R.gate[q];
     pp[q] = pos;
+    if (pos < 0) continue;
     pt[pos] = q / P.k;
     pj[pos] = q % P.k;
     pg[pos] = R.gate[q];
@@ -649,25 +675,26 @@ __device__ __noinline__ void ds_publish(const DSParams& P, int l, int np, int nu
     us[u] = R.uniq_slot[u];
     uo[u] = R.uniq_off[u];
   }
+  const int n_kept = R.uniq_off[nu];  // the sorted pairs (all T * k unless some were left out)
   if (tid == 0) {
-    uo[nu] = np;
+    uo[nu] = n_kept;
     *reinterpret_cast<int32_t*>(rec + P.ro.n_uniq) = nu;
   }
 #pragma unroll 1
   for (int e = tid; e < P.E; e += CT) {  // counts by binary search in the sorted experts
-    int lo = 0, hi = np;
+    int lo = 0, hi = n_kept;
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
       if (R.sorted_e[mid] < e) lo = mid + 1; else hi = mid;
     }
-    int lo2 = lo, hi2 = np;
+    int lo2 = lo, hi2 = n_kept;
     while (lo2 < hi2) {
       const int mid = (lo2 + hi2) >> 1;
       if (R.sorted_e[mid] <= e) lo2 = mid + 1; else hi2 = mid;
     }
     ec[e] = lo2 - lo;
     eo[e] = lo;
-    if (e == P.E - 1) eo[P.E] = np;
+    if (e == P.E - 1) eo[P.E] = n_kept;
   }
 }
 
@@ -1486,6 +1513,7 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
 #pragma unroll 1
           for (int j = 0; j < P.k; ++j) {
             const int p = R.pair_pos[t * P.k + j];
+            if (p < 0) continue;  // left out
             const float g = R.pair_gate[p];
             a0 = fmaf(g, zs[p * P.rpc + rr], a0);
             a1 = fmaf(g, zs[p * P.rpc + rr + 1], a1);
@@ -1662,6 +1690,8 @@ cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const St
   P.renorm = c.renorm;
   P.residual = c.residual;
   P.has_shared = a.shared != nullptr;
+  P.skip_from = c.skip_from;
+  P.hot_slots = c.hot_slots;
   P.out_f32 = c.out_fp32;
   P.wr = a.wr;
   P.bias = a.bias;

@@ -86,9 +86,17 @@ static moe_status check_cfg(const moe_layer_cfg* c) {
   if (c->k > c->E || c->k > kMaxK) return MOE_EINVAL;
   if (c->E > kMaxE) return MOE_EUNSUPPORTED;
   if (c->n_shared != 0 && c->n_shared != 1) return MOE_EUNSUPPORTED;
+  if (c->skip_from < 0 || c->skip_from > c->k || c->hot_slots < 0) return MOE_EINVAL;
   if (c->d % 128 != 0 || c->f % 64 != 0 || c->d > 4096 || c->f > 4096) return MOE_EUNSUPPORTED;
   if (!decode_geometry_ok(c->d, c->f)) return MOE_EUNSUPPORTED;
   return MOE_OK;
+}
+
+// The entry points outside the fused decode kernel do not skip experts.
+static moe_status check_cfg_unskipped(const moe_layer_cfg* c) {
+  const moe_status st = check_cfg(c);
+  if (st != MOE_OK) return st;
+  return c->skip_from != 0 ? MOE_EUNSUPPORTED : MOE_OK;
 }
 
 static bool aligned(const void* p, size_t a) {
@@ -177,7 +185,7 @@ static moe_status run_ffn(moe_ctx* ctx, const moe_layer_cfg* cfg, int bits, cons
   if (ctx == nullptr || grp == nullptr) return MOE_EINVAL;
   DeviceGuard dg(ctx->c.device);
   if (!dg.ok) return MOE_ECUDA;
-  moe_status st = check_cfg(cfg);
+  moe_status st = check_cfg_unskipped(cfg);
   if (st != MOE_OK) return st;
   if (cfg->bits != bits) return MOE_EINVAL;
   const int T = grp->T;
@@ -498,7 +506,7 @@ moe_status moe_router_topk(moe_ctx* ctx, const moe_layer_cfg* cfg, const void* x
   if (ctx == nullptr) return MOE_EINVAL;
   DeviceGuard dg(ctx->c.device);
   if (!dg.ok) return MOE_ECUDA;
-  moe_status st = check_cfg(cfg);
+  moe_status st = check_cfg_unskipped(cfg);
   if (st != MOE_OK) return st;
   if (T < 0) return MOE_EINVAL;
   if (T == 0) return MOE_OK;
@@ -517,7 +525,7 @@ moe_status moe_topk(moe_ctx* ctx, const moe_layer_cfg* cfg, const float* logits,
   if (ctx == nullptr) return MOE_EINVAL;
   DeviceGuard dg(ctx->c.device);
   if (!dg.ok) return MOE_ECUDA;
-  moe_status st = check_cfg(cfg);
+  moe_status st = check_cfg_unskipped(cfg);
   if (st != MOE_OK) return st;
   if (T < 0) return MOE_EINVAL;
   if (T == 0) return MOE_OK;
@@ -531,7 +539,7 @@ moe_status moe_group_tokens(moe_ctx* ctx, const moe_layer_cfg* cfg, const int32_
   if (ctx == nullptr || out == nullptr) return MOE_EINVAL;
   DeviceGuard dg(ctx->c.device);
   if (!dg.ok) return MOE_ECUDA;
-  moe_status st = check_cfg(cfg);
+  moe_status st = check_cfg_unskipped(cfg);
   if (st != MOE_OK) return st;
   if (T < 0 || n_slots <= 0) return MOE_EINVAL;
   if (ws == nullptr || !aligned(ws, 256)) return MOE_EINVAL;
@@ -565,7 +573,7 @@ moe_status moe_combine(moe_ctx* ctx, const moe_layer_cfg* cfg, const moe_groupin
   if (ctx == nullptr || grouping == nullptr) return MOE_EINVAL;
   DeviceGuard dg(ctx->c.device);
   if (!dg.ok) return MOE_ECUDA;
-  moe_status st = check_cfg(cfg);
+  moe_status st = check_cfg_unskipped(cfg);
   if (st != MOE_OK) return st;
   if (T < 0 || grouping->T != T || grouping->k != cfg->k) return MOE_EINVAL;
   if (T == 0) return MOE_OK;
@@ -601,6 +609,7 @@ moe_status moe_layer_forward(moe_ctx* ctx, const moe_layer_cfg* cfg, const void*
   if (T <= MOE_DECODE_MAX_T && cfg->E <= 512)  // one fused kernel: router, top-k, grouping, experts, combine
     return run_stack(ctx, *cfg, 1, x, T, w_router, logit_bias, slot_of, n_slots, slot_pool, slot_stride,
                      shared_expert, ws, y, stream);
+  if (cfg->skip_from != 0) return MOE_EUNSUPPORTED;  // skipping lives in the fused decode kernel only
   if ((st = moe_router_topk(ctx, cfg, x, w_router, logit_bias, T, logits, idx, gate, stream)) != MOE_OK)
     return st;
   moe_grouping g;

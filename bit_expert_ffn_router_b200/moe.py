@@ -29,7 +29,8 @@ class MoeError(RuntimeError):
 
 class _Cfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in
-                ("d", "f", "E", "k", "n_shared", "bits", "block", "renorm", "out_fp32", "residual")]
+                ("d", "f", "E", "k", "n_shared", "bits", "block", "renorm", "out_fp32", "residual",
+                 "skip_from", "hot_slots")]
 
 
 class _Layout(ctypes.Structure):
@@ -62,6 +63,8 @@ class LayerCfg:
     renorm: int = 1
     out_fp32: int = 1
     residual: int = 0
+    skip_from: int = 0  # 0: off; else pairs of rank >= skip_from on a slot >= hot_slots are left out (decode)
+    hot_slots: int = 0
 
     def c(self) -> _Cfg:
         return _Cfg(*(getattr(self, f.name) for f in dataclasses.fields(self)))

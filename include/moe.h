@@ -101,6 +101,19 @@ typedef struct {
   int renorm;    /* 1: gates = softmax over the k chosen logits; 0: full softmax read at them */
   int out_fp32;  /* 1: y is fp32; 0: y is bf16 (round to nearest even) */
   int residual;  /* 1: y = x + moe(x) */
+  /* Skipping low-ranked experts that are not resident (the pages' engine, on
+   * NVIDIA GPUs, by default leaves out low-ranked experts that are not in GPU
+   * memory and documents the small output change: news.blueqat.app/post/3262,
+   * section どう見るか). skip_from = 0: off. Else, in the fused decode calls
+   * (moe_layer_forward with T <= MOE_DECODE_MAX_T and E <= 512,
+   * moe_stack_forward), the pair of rank j >= skip_from of a token whose
+   * expert's slot is >= hot_slots is left out: it adds nothing to y, the
+   * other gates keep their values (no renormalisation), and an expert left
+   * with no pair is not read at all. The routing views then group the kept
+   * pairs only (uniq_offset[n_uniq] = their number; pair_pos = -1 for a pair
+   * left out). Other paths reject skip_from != 0 with MOE_EUNSUPPORTED. */
+  int skip_from; /* 0..k */
+  int hot_slots; /* slots [0, hot_slots) count as resident */
 } moe_layer_cfg;
 
 typedef struct {

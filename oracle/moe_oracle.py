@@ -233,20 +233,23 @@ def route(x_bits, w_router, k, bias=None, renorm=True):
 
 # ------------------------------------------------------------------ grouping
 
-def group(idx: np.ndarray, gate: np.ndarray, E: int, slot_of=None) -> dict:
+def group(idx: np.ndarray, gate: np.ndarray, E: int, slot_of=None, keep=None) -> dict:
     """Token -> expert grouping: a stable sort of the pairs p = t*k + j by expert.
 
     The result is in (expert, token, j) order. slot_of maps an expert to its
     slot in the expert pool, the indirection that stands for the pages' hot
     expert cache (vramglass.com, section その1：よく使うエキスパートを選んでGPUに置く).
+    keep (from kept_pairs) restricts the sort to the kept pairs; a pair left
+    out has pair_pos -1.
     """
     idx = np.asarray(idx, dtype=np.int64)
     T, k = idx.shape
     flat = idx.reshape(-1)
-    order = np.argsort(flat, kind="stable")
-    count = np.bincount(flat, minlength=E)
+    cand = np.arange(flat.size) if keep is None else np.nonzero(np.asarray(keep).reshape(-1))[0]
+    order = cand[np.argsort(flat[cand], kind="stable")]
+    count = np.bincount(flat[cand], minlength=E)
     offset = np.concatenate([[0], np.cumsum(count)])
-    pos = np.empty_like(order)
+    pos = np.full(flat.size, -1, dtype=np.int64)
     pos[order] = np.arange(order.size)
     uniq = np.nonzero(count)[0]
     g = {
@@ -293,8 +296,23 @@ class ExpertCache:
         return self.cache[key]
 
 
+def kept_pairs(idx: np.ndarray, slot_of, skip_from: int, hot_slots: int) -> np.ndarray:
+    """Which (token, j) pairs a step that skips low-ranked non-resident
+    experts keeps: all when skip_from == 0; else pair (t, j) is left out when
+    j >= skip_from and its expert's slot is >= hot_slots. The pages' engine
+    leaves out low-ranked experts that are not in GPU memory (news.blueqat.app
+    /post/3262, section どう見るか); "low-ranked" is read as rank >= skip_from
+    of the token's k, "not in GPU memory" as a slot outside the hot set, and
+    the remaining gates keep their values."""
+    keep = np.ones(idx.shape, dtype=bool)
+    if skip_from:
+        slots = np.asarray(slot_of)[idx]
+        keep[:, skip_from:] = slots[:, skip_from:] < hot_slots
+    return keep
+
+
 def layer_forward(x_bits, w_router, k, experts, shared=None, bias=None, renorm=True,
-                  residual=False, tokens=None):
+                  residual=False, tokens=None, skip_from=0, hot_slots=0, slot_of=None):
     """One MoE layer in fp64.
 
     experts(e) -> (W_g, W_u, W_d) of routed expert e; shared -> the shared
@@ -303,16 +321,20 @@ def layer_forward(x_bits, w_router, k, experts, shared=None, bias=None, renorm=T
     experts of each layer between GPU and CPU and wait for both before the next
     layer: vramglass.com, section その2：GPUとCPUで同時に計算する).
     residual=True returns x + y. `tokens` restricts the FFN to a subset of the
-    tokens (routing is still computed for all).
-    Returns dict(logits, idx, gate, y) with y fp64 [len(tokens), d].
+    tokens (routing is still computed for all). skip_from > 0 leaves out the
+    pairs kept_pairs() drops (slot_of: the layer's slot table).
+    Returns dict(logits, idx, gate, y, keep) with y fp64 [len(tokens), d].
     """
     l, idx, g = route(x_bits, w_router, k, bias, renorm)
+    keep = kept_pairs(idx, slot_of, skip_from, hot_slots)
     xd = bf16_to_f64(x_bits)
     toks = range(xd.shape[0]) if tokens is None else tokens
     ys = []
     for t in toks:
         y = np.zeros(xd.shape[1])
         for j in range(k):
+            if not keep[t, j]:
+                continue
             wg, wu, wd = experts(int(idx[t, j]))
             y = y + g[t, j] * expert_forward(xd[t], wg, wu, wd)
         if shared is not None:
@@ -320,4 +342,4 @@ def layer_forward(x_bits, w_router, k, experts, shared=None, bias=None, renorm=T
         if residual:
             y = xd[t] + y
         ys.append(y)
-    return {"logits": l, "idx": idx, "gate": g, "y": np.array(ys).reshape(len(ys), xd.shape[1])}
+    return {"logits": l, "idx": idx, "gate": g, "keep": keep, "y": np.array(ys).reshape(len(ys), xd.shape[1])}

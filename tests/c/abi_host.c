@@ -22,7 +22,7 @@ static unsigned char ws_raw[(1 << 20) + 256];
 
 int main(int argc, char** argv) {
   const int use_gpu = argc > 1 && strcmp(argv[1], "gpu") == 0;
-  moe_layer_cfg cfg = {2048, 768, 512, 10, 1, 2, 32, 1, 1, 0};
+  moe_layer_cfg cfg = {2048, 768, 512, 10, 1, 2, 32, 1, 1, 0, 0, 0};
   moe_expert_layout lay;
   moe_routing r;
   moe_ctx* ctx = NULL;

@@ -61,7 +61,8 @@ class Layer:
         cache = O.ExpertCache(lambda e: self.sections[e], self.cfg.d, self.cfg.f, self.cfg.bits)
         sh = O.expert_weights(self.shared, self.cfg.d, self.cfg.f, self.cfg.bits) if self.shared else None
         return O.layer_forward(self.x, self.wr, self.cfg.k, cache, sh, bias=self.bias, renorm=bool(self.cfg.renorm),
-                               residual=bool(self.cfg.residual), tokens=tokens)
+                               residual=bool(self.cfg.residual), tokens=tokens, skip_from=self.cfg.skip_from,
+                               hot_slots=self.cfg.hot_slots, slot_of=self.slot_of)
 
     # ---- device side
     def device(self):

@@ -410,3 +410,41 @@ def test_brute_force_tiny_layer(bits):
         y = [a + b for a, b in zip(acc, y)]
         assert list(out["idx"][t]) == order
         assert np.allclose(out["y"][t], y, rtol=1e-11, atol=1e-13)
+
+
+def test_skipping_low_ranked_non_resident_pairs():
+    """Leaving out pairs of rank >= skip_from on non-resident slots: the cases
+    that reduce to no skipping (every slot resident; skip_from = k), the case
+    that keeps only the top expert (skip_from = 1, nothing resident), and the
+    general case against the full layer minus the dropped pairs' terms."""
+    d, f, E, k, bits = 256, 128, 16, 4, 2
+    secs, shared = _tiny_layer(d, f, E, bits, seed=40)
+    x = synth.activations(5, d, seed=41)
+    wr = synth.router_weights(E, d, seed=42)
+    cache = O.ExpertCache(lambda e: secs[e], d, f, bits)
+    sh = O.expert_weights(shared, d, f, bits)
+    slot_of = synth.rng(43).permutation(E)
+    full = O.layer_forward(x, wr, k, cache, sh)
+    same = O.layer_forward(x, wr, k, cache, sh, skip_from=1, hot_slots=E, slot_of=slot_of)
+    assert np.array_equal(same["y"], full["y"]) and same["keep"].all()
+    same = O.layer_forward(x, wr, k, cache, sh, skip_from=k, hot_slots=0, slot_of=slot_of)
+    assert np.array_equal(same["y"], full["y"])
+    top = O.layer_forward(x, wr, k, cache, sh, skip_from=1, hot_slots=0, slot_of=slot_of)
+    xd = O.bf16_to_f64(x)
+    for t in range(5):
+        e0 = int(full["idx"][t, 0])
+        want = full["gate"][t, 0] * O.expert_forward(xd[t], *cache(e0)) + O.expert_forward(xd[t], *sh)
+        assert np.allclose(top["y"][t], want, rtol=1e-12, atol=1e-14)
+    part = O.layer_forward(x, wr, k, cache, sh, skip_from=2, hot_slots=E // 2, slot_of=slot_of)
+    keep = part["keep"]
+    assert keep[:, :2].all()
+    assert np.array_equal(keep[:, 2:], slot_of[full["idx"][:, 2:]] < E // 2)
+    for t in range(5):
+        drop = sum(full["gate"][t, j] * O.expert_forward(xd[t], *cache(int(full["idx"][t, j])))
+                   for j in range(k) if not keep[t, j])
+        assert np.allclose(part["y"][t], full["y"][t] - drop, rtol=1e-10, atol=1e-12)
+    g = O.group(full["idx"], full["gate"], E, slot_of, keep=keep)
+    assert g["expert_count"].sum() == keep.sum()
+    assert np.all(g["pair_pos"][~keep] == -1)
+    kept_pos = np.sort(g["pair_pos"][keep])
+    assert np.array_equal(kept_pos, np.arange(keep.sum()))

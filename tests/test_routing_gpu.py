@@ -54,22 +54,26 @@ def check_published_routing(L, ws=None, check_fp64=True, ws_routing=None):
         scale = np.abs(l_ref).max(axis=1, keepdims=True)
         assert np.all(np.abs(logits - l_ref) <= 1e-5 * scale)
         H.assert_routing_matches(r["idx"], idx_ref, l_ref)
-    # grouping of the published selection, every array
-    ref = O.group(r["idx"], r["gate"], cfg.E, L.slot_of)
-    n_pairs = T * cfg.k
+    # grouping of the published selection, every array (of the kept pairs,
+    # when low-ranked non-resident ones are left out)
+    keep = O.kept_pairs(r["idx"].astype(np.int64), L.slot_of, cfg.skip_from, cfg.hot_slots)
+    ref = O.group(r["idx"], r["gate"], cfg.E, L.slot_of, keep=keep)
+    n = int(keep.sum())
     nu = int(r["n_uniq"][0])
     assert nu == ref["n_uniq"]
     assert np.array_equal(r["expert_count"], ref["expert_count"])
     assert np.array_equal(r["expert_offset"], ref["expert_offset"])
-    assert np.array_equal(r["pair_token"], ref["pair_token"])
-    assert np.array_equal(r["pair_j"], ref["pair_j"])
-    assert np.array_equal(r["pair_gate"], ref["pair_gate"].astype(np.float32), equal_nan=True)
+    assert np.array_equal(r["pair_token"][:n], ref["pair_token"])
+    assert np.array_equal(r["pair_j"][:n], ref["pair_j"])
+    assert np.array_equal(r["pair_gate"][:n], ref["pair_gate"].astype(np.float32), equal_nan=True)
     assert np.array_equal(r["pair_pos"], ref["pair_pos"].reshape(-1))
-    order = np.argsort(r["idx"].reshape(-1), kind="stable")
-    assert np.array_equal(r["pair_slot"], L.slot_of[r["idx"].reshape(-1)[order]])
+    flat = r["idx"].reshape(-1)
+    kept_idx = np.nonzero(keep.reshape(-1))[0]
+    order = kept_idx[np.argsort(flat[kept_idx], kind="stable")]
+    assert np.array_equal(r["pair_slot"][:n], L.slot_of[flat[order]])
     assert np.array_equal(r["uniq_expert"][:nu], ref["uniq_expert"])
     assert np.array_equal(r["uniq_slot"][:nu], ref["uniq_slot"])
-    assert np.array_equal(r["uniq_offset"][:nu + 1], np.append(ref["expert_offset"][ref["uniq_expert"]], n_pairs))
+    assert np.array_equal(r["uniq_offset"][:nu + 1], np.append(ref["expert_offset"][ref["uniq_expert"]], n))
     return r
 
 

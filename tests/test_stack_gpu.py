@@ -187,3 +187,35 @@ def test_stack_wait_limits_report_timeout_and_recover(monkeypatch, limit_us):
     y2, _ = st.forward()
     torch.cuda.synchronize()
     assert torch.equal(y2, ref)
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("T", [1, 4])
+def test_stack_leaves_out_low_ranked_non_resident_pairs(bits, T):
+    """skip_from / hot_slots: every layer against the oracle that leaves the
+    same pairs out (routing views of the kept pairs, outputs within the usual
+    bound); with every slot resident the bits equal the plain stack's."""
+    base = M.FULL.replace(bits=bits, out_fp32=0, residual=1)
+    st = Stack(base, 3, T, seed=740 + 10 * bits + T)
+    plain, _ = st.forward()
+    st.cfg = base.replace(skip_from=4, hot_slots=st.n_slots)
+    same, _ = st.forward()
+    torch.cuda.synchronize()
+    assert torch.equal(same, plain)
+    cfg = base.replace(skip_from=4, hot_slots=st.n_slots // 2)
+    st.cfg = cfg
+    y, ws = st.forward()
+    torch.cuda.synchronize()
+    assert H.ctx().check_device_status() == M.OK
+    x = st.x
+    dropped = 0
+    for l in range(st.L):
+        Lv = st.layer_view(l, x)
+        r = {k: v.cpu().numpy() for k, v in H.ctx().layer_routing(cfg, T, ws, stack_layers=st.L, layer=l).items()}
+        check_published_routing(Lv, ws_routing=r)
+        ref = Lv.oracle()
+        dropped += int((~ref["keep"]).sum())
+        H.assert_close_rows(H.y_as_f64(y[l]), ref["y"], bf16=True)
+        x = _bits(y[l])
+    assert dropped > 0
+    assert not torch.equal(y, plain)
