@@ -51,9 +51,10 @@ def bf16_bits_to_f32(b) -> np.ndarray:
     return (b.astype(np.uint32) << 16).view(np.float32)
 
 
-def activations(T: int, d: int, seed: int) -> np.ndarray:
-    """x [T, d] as raw bf16 bits, N(0,1)."""
-    return f32_to_bf16_bits(rng(seed).standard_normal((T, d), dtype=np.float32))
+def activations(T: int, d: int, seed: int, scale: float = 1.0) -> np.ndarray:
+    """x [T, d] as raw bf16 bits, N(0, scale^2) (a power-of-two scale only
+    moves the exponent of the N(0,1) draw)."""
+    return f32_to_bf16_bits(rng(seed).standard_normal((T, d), dtype=np.float32) * np.float32(scale))
 
 
 def router_weights(E: int, d: int, seed: int, std: float = 0.02) -> np.ndarray:
