@@ -2,6 +2,9 @@
 // order, rows already multiplied by their gates) + z_rows[n_pairs + t] (the
 // shared expert), plus x[t] when the layer adds its residual.
 //
+// A pair the grouping left out (pair_pos -1: its expert is not held on this
+// device) adds nothing.
+//
 // The pages join each layer's routed experts (computed partly on the GPU and
 // partly on the CPU) before moving to the next layer (vramglass.com, section
 // その2：GPUとCPUで同時に計算する); here every expert runs on the GPU and the
@@ -22,6 +25,7 @@ combine_kernel(const int32_t* __restrict__ pair_pos, int n_pairs, int k, int has
   for (int c4 = threadIdx.x; c4 < n4; c4 += blockDim.x) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < k; ++j) {
+      if (pos[j] < 0) continue;
       const float4 v = __ldcs(reinterpret_cast<const float4*>(z + static_cast<size_t>(pos[j]) * d) + c4);
       acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }

@@ -539,14 +539,16 @@ __device__ __noinline__ void ds_topk(const DSParams& P, int t, uint32_t tag, flo
     // the kept ones by expert index, found here by ranks instead of a
     // CTA-wide sort
     int slot = 0;
+    bool held = true;
     if (sel) {
       slot = R.slot_s[min(max(mine_e, 0), P.E - 1)];
-      if (slot < 0 || slot >= P.n_slots) {
+      held = slot != kSlotAbsent;
+      if (held && (slot < 0 || slot >= P.n_slots)) {
         report(P.status, kDevBadSlot, mine_e);
         slot = 0;
       }
     }
-    const bool keep = sel && !(P.skip_from > 0 && lane >= P.skip_from && slot >= P.hot_slots);
+    const bool keep = sel && held && !(P.skip_from > 0 && lane >= P.skip_from && slot >= P.hot_slots);
     const unsigned kept = __ballot_sync(0xffffffffu, keep);
     int pos = 0;
 #pragma unroll 4
@@ -573,10 +575,12 @@ __device__ __noinline__ void ds_topk(const DSParams& P, int t, uint32_t tag, flo
 
 // Stable sort of the T*k pairs by expert in shared memory, the unique
 // experts and their slots. Every consumer thread takes part.
-// Pair p = t * k + j stays unless skipping is on, its rank j >= skip_from
-// and its expert's slot is not resident.
+// Pair p = t * k + j stays unless its expert is not held here (slot
+// kSlotAbsent), or skipping is on, its rank j >= skip_from and its expert's
+// slot is not resident.
 __device__ __forceinline__ bool ds_keep_pair(const DSParams& P, const DSRoute& R, int p, int e) {
-  return P.skip_from == 0 || p % P.k < P.skip_from || R.slot_s[e] < P.hot_slots;
+  const int slot = R.slot_s[e];
+  return slot != kSlotAbsent && (P.skip_from == 0 || p % P.k < P.skip_from || slot < P.hot_slots);
 }
 
 __device__ __noinline__ void ds_group(const DSParams& P, DSShared* S, int np, int CT) {
@@ -1360,7 +1364,7 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
         for (int p = tid; p < np; p += CT) {
           R.pair_token[p] = min(max(__ldcg(P.g.pair_token + p), 0), P.T - 1);
           R.pair_gate[p] = __ldcg(P.g.pair_gate + p);
-          R.pair_pos[p] = min(max(__ldcg(P.g.pair_pos + p), 0), np - 1);
+          R.pair_pos[p] = min(max(__ldcg(P.g.pair_pos + p), -1), np - 1);  // -1: a pair left out
         }
 #pragma unroll 1
         for (int u = tid; u <= nug; u += CT) R.uniq_off[u] = min(max(__ldcg(P.g.uniq_offset + u), 0), np);

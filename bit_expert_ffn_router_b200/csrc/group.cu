@@ -11,6 +11,10 @@
 //
 // Sorted order is (expert, token, j). Pairs are numbered p = t*k + j; within
 // one expert they appear in ascending p, which is ascending token.
+//
+// slot_of[e] == kSlotAbsent marks an expert this device does not hold (expert
+// parallelism): its pairs are left out of the sort (pair_pos = -1, count 0),
+// so the sorted pairs, the unique experts and the tiles cover the held ones.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -66,25 +70,29 @@ __device__ void write_tiles(int e, int count, int E, int T, int n_shared, int* s
 }
 
 // Per-expert totals -> offsets, unique list, slot lookup, tiles. Thread e
-// holds count (0 for e >= E). Returns the expert's first sorted position.
-__device__ int finish_counts(int e, int count, int E, int T, int n_pairs, int n_shared,
-                             const int32_t* slot_of, int n_slots, const GroupPtrs& g,
-                             int* s_warp, int* status, int* slot_out) {
+// holds count (0 for e >= E); an absent expert's count becomes 0. Returns
+// the expert's first sorted position.
+__device__ int finish_counts(int e, int count, int E, int T, int n_shared, const int32_t* slot_of, int n_slots,
+                             const GroupPtrs& g, int* s_warp, int* status, int* slot_out) {
+  int slot = 0;
+  if (e < E) {
+    slot = slot_of[e];
+    if (slot == kSlotAbsent) {
+      count = 0;
+    } else if (count > 0 && (slot < 0 || slot >= n_slots)) {
+      report(status, kDevBadSlot, e);
+      slot = 0;
+    }
+  }
   int total;
   const int off = block_exclusive_scan(count, s_warp, &total);
   int nu;
   const int u = block_exclusive_scan(count > 0 ? 1 : 0, s_warp, &nu);
-  int slot = 0;
   if (e < E) {
     g.expert_count[e] = count;
     g.expert_offset[e] = off;
     if (e == E - 1) g.expert_offset[E] = off + count;
     if (count > 0) {
-      slot = slot_of[e];
-      if (slot < 0 || slot >= n_slots) {
-        report(status, kDevBadSlot, e);
-        slot = 0;
-      }
       g.uniq_expert[u] = e;
       g.uniq_slot[u] = slot;
       g.uniq_offset[u] = off;
@@ -92,7 +100,7 @@ __device__ int finish_counts(int e, int count, int E, int T, int n_pairs, int n_
   }
   if (threadIdx.x == 0) {
     *g.n_uniq = nu;
-    g.uniq_offset[nu] = n_pairs;
+    g.uniq_offset[nu] = total;  // the sorted (held) pairs
   }
   write_tiles(e, count, E, T, n_shared, s_warp, g.tile_offset);
   *slot_out = slot;
@@ -125,10 +133,13 @@ group_small_kernel(const int32_t* __restrict__ idx, const float* __restrict__ ga
   if (e < E)
     for (int p = 0; p < n_pairs; ++p) count += (s_idx[p] == e);
   int slot;
-  int r = finish_counts(e, count, E, T, n_pairs, n_shared, slot_of, n_slots, g, s_warp, status, &slot);
+  int r = finish_counts(e, count, E, T, n_shared, slot_of, n_slots, g, s_warp, status, &slot);
+  const bool absent = e < E && slot_of[e] == kSlotAbsent;
   if (e < E && count > 0) {
     for (int p = 0; p < n_pairs; ++p) {
-      if (s_idx[p] == e) {
+      if (s_idx[p] == e && absent) {
+        g.pair_pos[p] = -1;
+      } else if (s_idx[p] == e) {
         g.pair_token[r] = p / k;
         g.pair_j[r] = p % k;
         g.pair_gate[r] = gate[p];
@@ -169,7 +180,9 @@ group_chunk_kernel(const int32_t* __restrict__ idx, const float* __restrict__ ga
     __syncwarp();
     if (valid && rank == 0) cnt[e] = before + __popc(peers);
     __syncwarp();
-    if (kScatter && valid) {
+    if (kScatter && valid && slot_of[e] == kSlotAbsent) {
+      g.pair_pos[p] = -1;
+    } else if (kScatter && valid) {
       const int r = g.expert_offset[e] + base[e] + before + rank;
       int slot = slot_of[e];
       if (slot < 0 || slot >= n_slots) slot = 0;
@@ -204,7 +217,7 @@ group_scan_kernel(int n_chunks, int T, int k, int E, const int32_t* __restrict__
     }
   }
   int slot;
-  finish_counts(e, running, E, T, T * k, n_shared, slot_of, n_slots, g, s_warp, status, &slot);
+  finish_counts(e, running, E, T, n_shared, slot_of, n_slots, g, s_warp, status, &slot);
 }
 
 cudaError_t launch_group(const Ctx& ctx, const moe_layer_cfg& c, const int32_t* idx,

@@ -16,6 +16,7 @@ namespace moe {
 constexpr int kBlock = 32;            // weights per fp16 scale
 constexpr int kMaxE = 1024;           // experts per layer
 constexpr int kMaxK = 32;             // experts per token
+constexpr int kSlotAbsent = -1;       // slot-table value of an expert this device does not hold
 constexpr int kGroupChunk = 512;      // pairs per chunk in the multi-CTA grouping
 constexpr int kTileN = 128;           // tokens per tile of the prefill grouped GEMM
 

@@ -57,7 +57,11 @@
  *
  * Expert pool: expert e of a layer lives at slot_pool + slot_of[e]*slot_stride
  * (the slot table stands for the pages' hot-expert cache; on one B200 every
- * expert is in HBM and the table is only an indirection).
+ * expert is in HBM and the table is only an indirection). slot_of[e] = -1
+ * (MOE_SLOT_ABSENT) marks an expert this device does not hold: its pairs are
+ * left out of the grouping (pair_pos = -1) and add nothing to y. This is how
+ * an expert-parallel step splits a layer over devices (each device holds a
+ * subset of the experts and produces a partial y; the partials are summed).
  */
 #ifndef MOE_H_
 #define MOE_H_
@@ -86,6 +90,9 @@ typedef int moe_status;
 
 typedef struct moe_ctx moe_ctx;
 typedef void* moe_stream; /* cudaStream_t */
+
+/* Slot-table value of an expert this device does not hold. */
+#define MOE_SLOT_ABSENT (-1)
 
 /* Largest T that takes the decode path (weight streaming, fused combine). */
 #define MOE_DECODE_MAX_T 8

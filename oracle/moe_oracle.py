@@ -303,11 +303,15 @@ def kept_pairs(idx: np.ndarray, slot_of, skip_from: int, hot_slots: int) -> np.n
     leaves out low-ranked experts that are not in GPU memory (news.blueqat.app
     /post/3262, section どう見るか); "low-ranked" is read as rank >= skip_from
     of the token's k, "not in GPU memory" as a slot outside the hot set, and
-    the remaining gates keep their values."""
+    the remaining gates keep their values. Independently of skipping, a pair
+    whose expert has slot -1 (not held by this device, the expert-parallel
+    split) is left out."""
     keep = np.ones(idx.shape, dtype=bool)
-    if skip_from:
+    if slot_of is not None:
         slots = np.asarray(slot_of)[idx]
-        keep[:, skip_from:] = slots[:, skip_from:] < hot_slots
+        keep &= slots != -1
+        if skip_from:
+            keep[:, skip_from:] &= slots[:, skip_from:] < hot_slots
     return keep
 
 
