@@ -48,7 +48,6 @@ constexpr int kDsGuDepth = 4;   // gate/up tasks a consumer warp has in flight
 constexpr int kDsGpd = 6;       // routed experts per down group (ring slot)
 constexpr int kQW = 18;         // words per quantised 32-value block: 16 int16 pairs, scale, sum
 constexpr int kDsMaxCtas = 256;  // grid size limit (done words per layer parity)
-constexpr int kDsLogitCopies = 4;  // copies of the logit words: CTA b reads copy b % 4
 constexpr int kDsPollNs = 64;      // back-off between polls of words that were not there yet
 
 // Tag source: every launch reads it and the last CTA to exit advances it by
@@ -59,8 +58,8 @@ __device__ unsigned int g_ds_exit;
 // output), one per 128-byte line: every CTA adds 1 per layer once its part
 // is written, so after layer l of a launch with tag base `base` each holds
 // (base + l + 1) * G (mod 2^32). They advance in step with the tag counter.
-constexpr int kCntLogits = 0, kCntH = 32, kCntOut = 64;
-__device__ unsigned int g_ds_cnt[96];
+constexpr int kCntLogits = 0, kCntH = 32, kCntOut = 64, kCntZero = 96;
+__device__ unsigned int g_ds_cnt[128];
 
 // Division by a runtime constant with one wide multiply: n / d for n < 2^31
 // and n < 2^32 / d, with m = floor(2^32 / d) + 1 (the remainder term stays
@@ -106,7 +105,9 @@ struct DSParams {
   size_t rec_bytes;
   RecOff ro;
   GroupPtrs g;                  // not route: the given grouping
-  unsigned long long* logits_ll;  // [kDsLogitCopies, T, E]
+  long long* lacc;                // [3, 2, T, E] router logits in fixed point: [part][parity]; parts in
+                                  // units of 2^-32, 2^22 and 2^76
+  int* lbad;                      // [2, T, E] flags: 1 a partial was not finite, 2 / 4 part 1 / 2 used
   unsigned long long* h_ll;       // [n_rows, f/32, kQW]
   unsigned long long* y_ll;       // [2, T, d/2]
   int* status;
@@ -122,7 +123,7 @@ struct DSParams {
   int n_ring, slot_bytes;       // weight ring: slots and bytes per slot
   int dn_stride, gpd;           // bytes per down stage, down stages per ring slot
   int hq_rows;
-  int sm_wr, sm_x, sm_xq, sm_hs, sm_zs, sm_route, sm_xres, sm_ring, sm_shdn;
+  int sm_ws, sm_ysl, sm_x, sm_xq, sm_hs, sm_zs, sm_route, sm_xres, sm_ring, sm_shdn;
   int sm_gub, gu_task_bytes, gu_depth;  // per-warp gate/up buffers: gu_depth tasks of gu_task_bytes each
   int max_blk;                  // gate/up blocks of one CTA in one layer (h staging slots)
 };
@@ -130,7 +131,7 @@ struct DSParams {
 struct DSShared {
   uint64_t full[kDsNS], empty[kDsNS];   // weight ring
   uint64_t shdn_full[2], shdn_empty[2];  // the shared expert's down rows, by layer parity
-  uint64_t wr_full, wr_empty, route_bar;
+  uint64_t route_bar;
   int abort_flag;
   unsigned base_tag;
   int n_uniq;
@@ -228,8 +229,8 @@ __device__ __forceinline__ bool ds_aborted(const DSShared* S) {
 
 // Counts this CTA's part of an exchange as written (the tagged words it
 // stored before the last CTA barrier); relaxed, fire and forget.
-__device__ __forceinline__ void cnt_add(int which) {
-  asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(&g_ds_cnt[which]) : "memory");
+__device__ __forceinline__ void cnt_add(int which, unsigned n = 1u) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(&g_ds_cnt[which]), "r"(n) : "memory");
 }
 
 // Polls an exchange counter (one thread) until it reaches `target`
@@ -326,11 +327,11 @@ constexpr int kXB = 1;
 
 template <int BITS, int GBPL>
 __device__ void ds_read_x(const DSParams& P, int l, uint32_t tag, uint16_t* xs, int* xq, float* xres, int r0,
-                          int r1, DSShared* S, uint64_t deadline, int CT) {
+                          int r1, DSShared* S, uint64_t deadline, int tid0, int CT) {
   const int nb = P.d / kBlock;
   const int words = kQW * nb;
   const int jobs = P.T * nb * 4;  // four threads per 32-value block
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x - tid0;  // the threads [tid0, tid0 + CT) take part (whole warps)
   const bool chained = l > 0;
   const unsigned long long* yl = P.y_ll + static_cast<size_t>((l - 1) & 1) * P.T * (P.d / 2);
   const int per_thread = (jobs + CT - 1) / CT;
@@ -437,122 +438,194 @@ __device__ __forceinline__ float ds_key_value(uint32_t k) {
 
 constexpr int kDsMaxE = 512;  // experts a decode launch supports
 
-// Warp t: polls token t's E <= 512 logit words (all of a lane's 16 at once),
-// turns them into order keys held in registers, selects its k experts and
-// gates into R. Selection: k rounds of a warp maximum over the keys (ties go
-// to the lower expert index through a second, minimum reduction over the
-// indices that hold the maximum); lane j keeps the j-th pick. The publishing
-// CTA also writes the plain logits.
-__device__ __noinline__ void ds_topk(const DSParams& P, int t, uint32_t tag, float* pub_logits, uint32_t* kr,
-                                     DSShared* S, uint64_t deadline, unsigned long long* td) {
-  const DSRoute R = ds_route(ds_smem + P.sm_route, P.T * P.k);
+// ---- router, split by rows: CTA b owns output rows [r0, r1) of every
+// layer. With x_{l+1} = y_l, its rows of y_l (bf16, as the next layer reads
+// them) against the same columns of layer l+1's router give a partial logit
+// for every (token, expert); the partials of all CTAs add up to the logits.
+// They are added as 64-bit integers, so the sum is exact and does not depend
+// on the order the CTAs arrive in. A partial p is cut into three parts in
+// units of 2^-32, 2^22 and 2^76: the multiple of 2^76 (p's bits at and above
+// 2^76), the multiple of 2^22 in what remains, and the rest rounded to
+// 2^-32. Every part is below 2^54 in magnitude, so up to 2^9 CTAs add without
+// overflow. The cut is exact for |p| >= 2^22 (its unit is then at least 2^-1);
+// below that, p is rounded to 2^-32 alone, the one rounding there is. A flag
+// word per logit tells the reader which of the upper parts were used; a
+// partial that is not finite sets flag 1 and the logit reads NaN.
+constexpr double kLogitUlp = 1.0 / 4294967296.0;
+constexpr double kLogitUnit1 = 4194304.0;                  // 2^22
+constexpr double kLogitUnit2 = 75557863725914323419136.0;  // 2^76
+
+__device__ __forceinline__ long long ld_relaxed_s64(const long long* p) {
+  long long v;
+  asm volatile("ld.relaxed.gpu.global.s64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_relaxed_s32(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Columns [r0, r1) of every row of layer l's router into ws (rpc floats per
+// expert), 8-byte cp.async pieces spread over the given threads; one commit.
+__device__ __forceinline__ void ds_wslice_load(const DSParams& P, int l, float* ws, int r0, int r1, int tid,
+                                               int nthreads) {
+  const int pairs = (r1 - r0) / 2, n = P.E * pairs;
+  const float* src = P.wr + static_cast<size_t>(l) * P.E * P.d + r0;
+#pragma unroll 1
+  for (int i = tid; i < n; i += nthreads) {
+    const int e = i / pairs, c = 2 * (i - e * pairs);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(ws + e * P.rpc + c)),
+                 "l"(src + static_cast<size_t>(e) * P.d + c)
+                 : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Warp t: reads token t's E <= 512 logits (all of a lane's 16 at once: the
+// fixed-point sums every CTA added, plus the bias), turns them into order
+// keys held in registers, selects its k experts and gates into R.
+// Selection: k rounds of a warp maximum over the keys (ties go to the lower
+// expert index through a second, minimum reduction over the indices that
+// hold the maximum); lane j keeps the j-th pick. The publishing CTA also
+// writes the plain logits.
+__device__ __noinline__ void ds_topk(const DSParams& P, int l, int t, float* pub_logits, unsigned long long* td) {
+  // the parameters this uses, in registers: P sits in shared memory, and the
+  // ordered loads below would make the compiler read it again each time
+  const int E = P.E, T = P.T, k = P.k, L = P.L;
+  const DSRoute R = ds_route(ds_smem + P.sm_route, T * k);
+  DSShared* S = reinterpret_cast<DSShared*>(ds_smem);
   constexpr int KPL = kDsMaxE / 32;  // keys a lane holds
   const int lane = threadIdx.x & 31;
-  const unsigned long long* row =
-      P.logits_ll + (static_cast<size_t>(blockIdx.x % kDsLogitCopies) * P.T + t) * P.E;
-  unsigned long long w[KPL];
+  const size_t o = (static_cast<size_t>(l & 1) * T + t) * E;
+  const long long* const acc = P.lacc + o;
+  const int* const flg = P.lbad + o;
+  const size_t part = 2 * static_cast<size_t>(T) * E;  // distance between the parts' accumulators
+  const float* const bias = P.bias != nullptr ? P.bias + (static_cast<size_t>(l) * T + t) * E : nullptr;
+  long long w[KPL];
+  int fl[KPL];
+  float bv[KPL];
 #pragma unroll
-  for (int v = 0; v < KPL; ++v) w[v] = ll_word(0u, v * 32 + lane < P.E ? tag - 1 : tag);  // absent words count as there
-  bool ok = true;
-#pragma unroll 1
-  for (int pass = 0;; ++pass) {  // (re-)load only the words not there yet, all at once
-    if (pass > 0) {
-      if (ds_aborted(S) || global_timer_ns() > deadline) {
-        ok = false;
-        break;
-      }
-      __nanosleep(kDsPollNs);
-    }
-#pragma unroll
-    for (int v = 0; v < KPL; ++v)
-      if (!tag_ok(w[v], tag)) w[v] = ld_ll(row + v * 32 + lane);
-    bool all = true;
-#pragma unroll
-    for (int v = 0; v < KPL; ++v) all = all && tag_ok(w[v], tag);
-    if (all) break;
+  for (int v = 0; v < KPL; ++v) {  // every load in flight at once
+    const int e = v * 32 + lane;
+    w[v] = e < E ? ld_relaxed_s64(acc + e) : 0;
+    fl[v] = e < E ? ld_relaxed_s32(flg + e) : 0;
+    bv[v] = (bias != nullptr && e < E) ? __ldg(bias + e) : 0.f;
   }
-  if (!__all_sync(0xffffffffu, ok)) {
-    if (lane == 0 && !ds_aborted(S)) ds_abort(S, P.status, 22);
-    return;
+  // the next layer's bias rows into L2 while this layer runs
+  if (bias != nullptr && l + 1 < L && lane * 32 < E)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(bias + static_cast<size_t>(T) * E + lane * 32));
+  // the logits: the 2^-32 part alone, rounded once to float (a power-of-two
+  // scale is exact), unless an upper part was used; NaN where a partial was
+  // not finite; then the bias
+  float lv[KPL];
+  bool upper = false;
+#pragma unroll
+  for (int v = 0; v < KPL; ++v) {
+    float c = __ll2float_rn(w[v]) * 2.3283064365386963e-10f;  // 2^-32
+    if (fl[v] & 1) c = __uint_as_float(0x7fc00000u);
+    lv[v] = bias != nullptr ? c + bv[v] : c;
+    upper = upper || (fl[v] & 6) != 0;
+  }
+  if (__any_sync(0xffffffffu, upper)) {  // seldom: upper parts first, then the 2^-32 part, in double
+#pragma unroll 1
+    for (int v = 0; v < KPL; ++v) {
+      const int e = v * 32 + lane;
+      if ((fl[v] & 6) == 0 || (fl[v] & 1) != 0 || e >= E) continue;
+      double sum = 0.0;
+      if (fl[v] & 4) sum = static_cast<double>(ld_relaxed_s64(acc + 2 * part + e)) * kLogitUnit2;
+      if (fl[v] & 2) sum += static_cast<double>(ld_relaxed_s64(acc + part + e)) * kLogitUnit1;
+      sum += static_cast<double>(w[v]) * kLogitUlp;
+      const float c = static_cast<float>(sum);
+      lv[v] = bias != nullptr ? c + __ldg(bias + e) : c;
+    }
   }
   uint32_t kv[KPL];  // order keys; 0 = absent (e >= E) or taken
 #pragma unroll
-  for (int v = 0; v < KPL; ++v) {
-    const int e = v * 32 + lane;
-    const float lv = __uint_as_float(static_cast<uint32_t>(w[v]));
-    kv[v] = e < P.E ? ds_order_key(lv) : 0u;
-    if (e < P.E) {
-      kr[e] = kv[v];
-      if (pub_logits != nullptr) pub_logits[static_cast<size_t>(t) * P.E + e] = lv;  // the publishing CTA
-    }
+  for (int v = 0; v < KPL; ++v) kv[v] = v * 32 + lane < E ? ds_order_key(lv[v]) : 0u;
+  if (pub_logits != nullptr) {  // the publishing CTA
+    float* const pl = pub_logits + static_cast<size_t>(t) * E;
+#pragma unroll
+    for (int v = 0; v < KPL; ++v)
+      if (v * 32 + lane < E) pl[v * 32 + lane] = lv[v];
   }
   if (td && lane == 0) td[29] = global_timer_ns();
+  // lane best: its largest key, ties to its lowest register index (so the
+  // lowest expert index), packed as key << 32 | (KPL - 1 - index)
+  auto lane_best = [&kv]() {
+    unsigned long long b[KPL];
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) b[i] = (static_cast<unsigned long long>(kv[i]) << 32) | (KPL - 1 - i);
+#pragma unroll
+    for (int h = KPL / 2; h > 0; h >>= 1)
+#pragma unroll
+      for (int i = 0; i < h; ++i) b[i] = b[i] > b[i + h] ? b[i] : b[i + h];
+    return b[0];
+  };
+  unsigned long long lb = lane_best();
   uint32_t mine_key = 0u;
   int mine_e = 0;
 #pragma unroll 1
-  for (int j = 0; j < P.k; ++j) {
-    // lane maximum and the lowest register index holding the warp maximum,
-    // both as trees (short dependency chains)
-    uint32_t t[KPL];
-#pragma unroll
-    for (int i = 0; i < KPL; ++i) t[i] = kv[i];
-#pragma unroll
-    for (int h = KPL / 2; h > 0; h >>= 1)
-#pragma unroll
-      for (int i = 0; i < h; ++i) t[i] = max(t[i], t[i + h]);
-    const uint32_t M = __reduce_max_sync(0xffffffffu, t[0]);
-#pragma unroll
-    for (int i = 0; i < KPL; ++i) t[i] = kv[i] == M ? static_cast<uint32_t>(i) : 0xffffu;
-#pragma unroll
-    for (int h = KPL / 2; h > 0; h >>= 1)
-#pragma unroll
-      for (int i = 0; i < h; ++i) t[i] = min(t[i], t[i + h]);
-    const unsigned le = t[0] < 0xffffu ? static_cast<unsigned>(lane + 32 * static_cast<int>(t[0])) : 0x7fffffffu;
+  for (int j = 0; j < k; ++j) {
+    // the warp maximum, then the lowest expert index holding it; only the
+    // lane that held it looks at its keys again
+    const uint32_t lk = static_cast<uint32_t>(lb >> 32);
+    const uint32_t M = __reduce_max_sync(0xffffffffu, lk);
+    const int li = KPL - 1 - static_cast<int>(lb & 0xffu);
+    const unsigned le = lk == M ? static_cast<unsigned>(lane + 32 * li) : 0x7fffffffu;
     const int e = static_cast<int>(__reduce_min_sync(0xffffffffu, le));
+    if (lane == (e & 31)) {
 #pragma unroll
-    for (int i = 0; i < KPL; ++i)
-      if (lane + 32 * i == e) kv[i] = 0u;
+      for (int i = 0; i < KPL; ++i) kv[i] = (i == (e >> 5)) ? 0u : kv[i];
+      lb = lane_best();
+    }
     if (lane == j) {
       mine_key = M;
       mine_e = e;
     }
   }
   if (td && lane == 0) td[30] = global_timer_ns();
-  const bool sel = lane < P.k;
+  const bool sel = lane < k;
   const float lj = sel ? ds_key_value(mine_key) : 0.f;
   const float l0 = __shfl_sync(0xffffffffu, lj, 0);
   const float ex = sel ? expf(lj - l0) : 0.f;
   float sum = ex;
   if (!P.renorm) {
-    // full-softmax denominator over the whole row (its keys in kr)
+    // full-softmax denominator over the whole row (lv, still in registers)
+    float ev[KPL];
+#pragma unroll
+    for (int v = 0; v < KPL; ++v) ev[v] = expf(lv[v] - l0);
     sum = 0.f;
-#pragma unroll 1
-    for (int e = lane; e < P.E; e += 32) sum += expf(ds_key_value(kr[e]) - l0);  // NaN logits make the sum NaN
+#pragma unroll
+    for (int v = 0; v < KPL; ++v)
+      if (v * 32 + lane < E) sum += ev[v];  // in order of e within the lane; NaN logits make the sum NaN
   }
   const float denom = warp_sum(sum);
+  const float gate = ex / denom;
   if (sel) {
-    R.idx[t * P.k + lane] = mine_e;
-    R.gate[t * P.k + lane] = ex / denom;
+    R.idx[t * k + lane] = mine_e;
+    R.gate[t * k + lane] = gate;
   }
-  if (P.T == 1) {
+  if (T == 1) {
     // one token: its k experts are distinct, so the grouping is the order of
     // the kept ones by expert index, found here by ranks instead of a
     // CTA-wide sort
     int slot = 0;
     bool held = true;
     if (sel) {
-      slot = R.slot_s[min(max(mine_e, 0), P.E - 1)];
+      slot = R.slot_s[min(max(mine_e, 0), E - 1)];
       held = slot != kSlotAbsent;
       if (held && (slot < 0 || slot >= P.n_slots)) {
         report(P.status, kDevBadSlot, mine_e);
         slot = 0;
       }
     }
-    const bool keep = sel && held && !(P.skip_from > 0 && lane >= P.skip_from && slot >= P.hot_slots);
+    const int skip_from = P.skip_from, hot_slots = P.hot_slots;
+    const bool keep = sel && held && !(skip_from > 0 && lane >= skip_from && slot >= hot_slots);
     const unsigned kept = __ballot_sync(0xffffffffu, keep);
     int pos = 0;
-#pragma unroll 4
-    for (int j = 0; j < 32; ++j) {
+#pragma unroll 1
+    for (int j = 0; j < k; ++j) {  // lanes at and above k hold no pick
       const int ej = __shfl_sync(0xffffffffu, mine_e, j);
       pos += (((kept >> j) & 1u) != 0u && ej < mine_e) ? 1 : 0;
     }
@@ -560,7 +633,7 @@ __device__ __noinline__ void ds_topk(const DSParams& P, int t, uint32_t tag, flo
     if (keep) {
       R.sorted_e[pos] = mine_e;
       R.pair_token[pos] = 0;
-      R.pair_gate[pos] = ex / denom;
+      R.pair_gate[pos] = gate;
       R.uniq_e[pos] = mine_e;
       R.uniq_slot[pos] = slot;
       R.uniq_off[pos] = pos;
@@ -583,23 +656,30 @@ __device__ __forceinline__ bool ds_keep_pair(const DSParams& P, const DSRoute& R
   return slot != kSlotAbsent && (P.skip_from == 0 || p % P.k < P.skip_from || slot < P.hot_slots);
 }
 
-__device__ __noinline__ void ds_group(const DSParams& P, DSShared* S, int np, int CT) {
+__device__ __noinline__ void ds_group(const DSParams& P, DSShared* S, int np, int CT, int* sk) {
   const DSRoute R = ds_route(ds_smem + P.sm_route, np);
   const int tid = threadIdx.x;
+  // a sort key per pair: expert, then pair index (np <= 1024) for a kept
+  // pair; past every such key for one left out
+  constexpr int kOut = 0x7fffffff;
 #pragma unroll 1
   for (int p = tid; p < np; p += CT) {
     const int e = min(max(R.idx[p], 0), P.E - 1);
-    if (!ds_keep_pair(P, R, p, e)) {
+    sk[p] = ds_keep_pair(P, R, p, e) ? (e << 10) + p : kOut;
+  }
+  named_sync(1, CT);
+  // a kept pair's place in the sorted order is the number of smaller keys
+#pragma unroll 1
+  for (int p = tid; p < np; p += CT) {
+    const int kp = sk[p];
+    if (kp == kOut) {
       R.pair_pos[p] = -1;
       continue;
     }
     int pos = 0;
-#pragma unroll 1
-    for (int q = 0; q < np; ++q) {
-      const int eq = min(max(R.idx[q], 0), P.E - 1);
-      pos += ((eq < e) || (eq == e && q < p)) && ds_keep_pair(P, R, q, eq);
-    }
-    R.sorted_e[pos] = e;
+#pragma unroll 8
+    for (int q = 0; q < np; ++q) pos += sk[q] < kp ? 1 : 0;
+    R.sorted_e[pos] = kp >> 10;
     R.pair_token[pos] = p / P.k;
     R.pair_gate[pos] = R.gate[p];
     R.pair_pos[p] = pos;
@@ -610,8 +690,7 @@ __device__ __noinline__ void ds_group(const DSParams& P, DSShared* S, int np, in
 #pragma unroll 1
     for (int c = 0; c < np; c += 32) {
       const int q = c + tid;
-      const bool k = q < np && ds_keep_pair(P, R, q, min(max(R.idx[q], 0), P.E - 1));
-      n_kept += __popc(__ballot_sync(0xffffffffu, k));
+      n_kept += __popc(__ballot_sync(0xffffffffu, q < np && sk[q] != kOut));
     }
     int base = 0;
 #pragma unroll 1
@@ -702,43 +781,50 @@ __device__ __noinline__ void ds_publish(const DSParams& P, int l, int np, int nu
   }
 }
 
-// ------------------------------------------------------------------ router
-// Router rows [e0, e1) of this CTA for every token (W_r rows and x in shared
-// memory); each logit goes out as a tagged word. Lanes take interleaved
-// 4-column groups and the warp sum is a fixed butterfly, so a token's logit
-// does not depend on the batch.
-__device__ void ds_router(const DSParams& P, int l, uint32_t tag, const float* wrs, const uint16_t* xs, int e0,
-                          int e1, int CW) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int n4 = P.d / 4, nr = e1 - e0;
-  const float* bias = P.bias != nullptr ? P.bias + static_cast<size_t>(l) * P.T * P.E : nullptr;
+// Adds this CTA's partial logits of the next layer: ysl [T, rpc] holds its
+// rows of that layer's input, ws the router's columns. buf: the layer's
+// parity.
+__device__ __noinline__ void ds_partial_logits(const DSParams& P, const float* ws, const float* ysl, int nr,
+                                               int buf, int CT) {
+  const int E = P.E, T = P.T, rpc = P.rpc;  // in registers (P is in shared memory)
+  long long* const acc = P.lacc + static_cast<size_t>(buf) * T * E;
+  const size_t part = 2 * static_cast<size_t>(T) * E;
+  int* const badf = P.lbad + static_cast<size_t>(buf) * T * E;
 #pragma unroll 1
-  for (int task = warp; task < nr * P.T; task += CW) {
-    int t = 0, rem = task;  // task -> (token, row) without a division: at most T rows of nr
-    while (rem >= nr) {
-      rem -= nr;
-      ++t;
+  for (int e = threadIdx.x; e < E; e += CT) {
+    const float* wrow = ws + e * rpc;
+#pragma unroll 1
+    for (int t = 0; t < T; ++t) {
+      const float* yrow = ysl + t * rpc;
+      float p = 0.f;
+#pragma unroll 2
+      for (int r = 0; r < nr; ++r) p = fmaf(yrow[r], wrow[r], p);
+      const size_t o = static_cast<size_t>(t) * E + e;
+      if (!isfinite(p)) {
+        asm volatile("red.relaxed.gpu.global.or.b32 [%0], 1;" ::"l"(badf + o) : "memory");
+        continue;
+      }
+      double rem = static_cast<double>(p);
+      int used = 0;
+      if (fabs(rem) >= kLogitUnit2) {  // the multiple of 2^76: below 2^52 for a finite float
+        const long long a = static_cast<long long>(trunc(rem * (1.0 / kLogitUnit2)));
+        rem -= static_cast<double>(a) * kLogitUnit2;
+        asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(acc + 2 * part + o), "l"(a) : "memory");
+        used |= 4;
+      }
+      if (fabs(rem) >= kLogitUnit1) {  // the multiple of 2^22 in a remainder below 2^76
+        const long long a = static_cast<long long>(trunc(rem * (1.0 / kLogitUnit1)));
+        rem -= static_cast<double>(a) * kLogitUnit1;
+        asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(acc + part + o), "l"(a) : "memory");
+        used |= 2;
+      }
+      const long long q = __double2ll_rn(rem * 4294967296.0);  // |rem| < 2^22
+      if (q != 0) asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(acc + o), "l"(q) : "memory");
+      if (used) asm volatile("red.relaxed.gpu.global.or.b32 [%0], %1;" ::"l"(badf + o), "r"(used) : "memory");
     }
-    const int e = e0 + rem;
-    const float4* w4 = reinterpret_cast<const float4*>(wrs + static_cast<size_t>(e - e0) * P.d);
-    const uint2* x2 = reinterpret_cast<const uint2*>(xs + static_cast<size_t>(t) * P.d);
-    const size_t o = static_cast<size_t>(t) * P.E + e;
-    const float bv = bias != nullptr ? __ldg(bias + o) : 0.f;
-    float acc = 0.f;
-#pragma unroll 4
-    for (int c4 = lane; c4 < n4; c4 += 32) {
-      const float4 w = w4[c4];
-      const uint2 xb = x2[c4];
-      acc = fmaf(w.x, __uint_as_float(xb.x << 16), acc);
-      acc = fmaf(w.y, __uint_as_float(xb.x & 0xffff0000u), acc);
-      acc = fmaf(w.z, __uint_as_float(xb.y << 16), acc);
-      acc = fmaf(w.w, __uint_as_float(xb.y & 0xffff0000u), acc);
-    }
-    acc = warp_sum(acc);
-    if (lane < kDsLogitCopies)
-      st_ll(P.logits_ll + static_cast<size_t>(lane) * P.T * P.E + o, ll_word(__float_as_uint(acc + bv), tag));
   }
 }
+
 
 // ------------------------------------------------------------------ gate/up
 // Rows of h: routed pair p at p (sorted order), shared token t at np + t.
@@ -791,7 +877,8 @@ __device__ __forceinline__ void cp_async_wait_pending(int n) {
   if (n <= 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
   else if (n == 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
   else if (n == 2) asm volatile("cp.async.wait_group 2;" ::: "memory");
-  else asm volatile("cp.async.wait_group 3;" ::: "memory");
+  else if (n == 3) asm volatile("cp.async.wait_group 3;" ::: "memory");
+  else asm volatile("cp.async.wait_group 4;" ::: "memory");
 }
 static_assert(kDsGuDepth == 4, "cp_async_wait_pending covers depths up to 4");
 
@@ -1075,8 +1162,8 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
   DSShared* S = reinterpret_cast<DSShared*>(smem);
   const int np = P.T * P.k;
   const DSRoute R = ds_route(smem + P.sm_route, np);
-  float* wrs = reinterpret_cast<float*>(smem + P.sm_wr);
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + P.sm_x);
+  float* wsl = reinterpret_cast<float*>(smem + P.sm_ws);    // this CTA's columns of the next router
+  float* ysl = reinterpret_cast<float*>(smem + P.sm_ysl);   // this CTA's rows of the next layer's input
   // quantised h rows of a round of down stages: the gate/up buffers and the
   // x staging area behind them (both idle during the down phase)
   int* hq = reinterpret_cast<int*>(smem + P.sm_gub);
@@ -1091,10 +1178,8 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
   const int G = gridDim.x, b = blockIdx.x;
   const int nbf = P.f / kBlock;
 
-  // static splits: router rows, output rows (units of `gran` rows) and the
-  // shared expert's channel blocks of this CTA
-  const int e0 = split_at(P.E, b, G);
-  const int e1 = split_at(P.E, b + 1, G);
+  // static splits: output rows (units of `gran` rows; the router columns
+  // follow them) and the shared expert's channel blocks of this CTA
   const int r0 = P.gran * split_at(P.n_units, b, G);
   const int r1 = P.gran * split_at(P.n_units, b + 1, G);
   // gate/up blocks are split among the CTAs by work (h rows x channels):
@@ -1109,7 +1194,6 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
   const int sb1 = P.has_shared ? min(nbf, (gu_hi + P.T - 1) / P.T) : 0;
   const int nsh = sb1 - sb0;
   const bool has_rows = r1 > r0;
-  const bool wr_rows = ROUTE && e1 > e0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kDsNS; ++i) {
@@ -1120,8 +1204,6 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
       mbar_init(&S->shdn_full[i], 1);
       mbar_init(&S->shdn_empty[i], 1);
     }
-    mbar_init(&S->wr_full, 1);
-    mbar_init(&S->wr_empty, CW);
     mbar_init(&S->route_bar, 1);
     S->abort_flag = 0;
     S->n_uniq = 0;
@@ -1152,7 +1234,7 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
     // one slot, so every wait is for the phase right after the one the
     // previous window saw complete (mbarrier parity cannot tell phase k
     // from phase k - 2).
-    uint32_t seq = 0, wr_count = 0, shdn_count = 0;
+    uint32_t seq = 0, shdn_count = 0;
     bool ok = true;
     // waits (lane-local, bounded) until ring slot `q` may be reused
     auto slot_ready = [&](uint32_t q) -> bool {
@@ -1163,11 +1245,6 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
         if (ds_aborted(S) || global_timer_ns() > deadline) return false;
       }
       return true;
-    };
-    auto issue_wr = [&](int l) {
-      const uint32_t bytes = static_cast<uint32_t>((e1 - e0) * P.d * 4);
-      mbar_arrive_expect_tx(&S->wr_full, bytes);
-      bulk_g2s(wrs, P.wr + (static_cast<size_t>(l) * P.E + e0) * P.d, bytes, &S->wr_full);
     };
     // layer l's shared-expert down rows: buffer l & 1, its (l >> 1)-th use
     auto issue_shdn = [&](int l) -> bool {
@@ -1184,9 +1261,8 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
     };
     const bool sh_dn = P.has_shared && has_rows;
     // Iteration l issues layer l's routed items (l >= 0), then layer l + 1's
-    // inputs that do not depend on its x: router rows, shared-expert down
-    // rows and gate/up stages. wr_count (lane 0) and shdn_count (lane 1)
-    // count the copies each lane actually issued.
+    // shared-expert down rows (they do not depend on its x). shdn_count
+    // (lane 1) counts the copies the lane actually issued.
 #pragma unroll 1
     for (int l = -1; l < P.L && ok; ++l) {
       if (ds_aborted_warp(S)) break;
@@ -1243,20 +1319,6 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
       if (l + 1 < P.L) {
         const int ln = l + 1;
         int okn = 1;
-        if (wr_rows && lane == 0) {
-          if (ln > 0) {
-            while (!mbar_try_wait(&S->wr_empty, l & 1, 100000u)) {
-              if (ds_aborted(S) || global_timer_ns() > deadline) {
-                okn = 0;
-                break;
-              }
-            }
-          }
-          if (okn) {
-            issue_wr(ln);
-            ++wr_count;
-          }
-        }
         if (sh_dn && lane == 1) {
           okn = issue_shdn(ln) ? 1 : 0;
           shdn_count += okn;
@@ -1274,9 +1336,6 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
       for (uint32_t q = seq > static_cast<uint32_t>(P.n_ring) ? seq - P.n_ring : 0; q < seq; ++q)
         while (!mbar_try_wait(&S->full[q % P.n_ring], (q / P.n_ring) & 1, 20000u) && global_timer_ns() < d2) {
         }
-      if (wr_count > 0)
-        while (!mbar_try_wait(&S->wr_full, (wr_count - 1) & 1, 20000u) && global_timer_ns() < d2) {
-        }
     }
     if (lane == 1)
 #pragma unroll 1
@@ -1287,9 +1346,49 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
   } else {
     // ============================================================ consumers
     const int tid = threadIdx.x;
+    const int nr_out = r1 - r0;
     uint32_t seq = 0;
     // this warp's shared-expert gate/up rows of the next layer, issued ahead
     int n_pre = (P.has_shared && !ds_aborted(S)) ? gu_prefetch_shared<CW>(Q, 0, nsh, sb0) : 0;
+    if (ROUTE) {
+      // ---- layer 0's logits: every CTA zeroes its share of the first
+      // accumulator, waits for all, then adds its rows of x against its
+      // columns of layer 0's router
+      ds_wslice_load(P, 0, wsl, r0, r1, tid, CT);
+      if (P.bias != nullptr && tid < P.T * 32 && (tid & 31) * 32 < P.E)  // layer 0's bias rows into L2
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(P.bias + static_cast<size_t>(tid >> 5) * P.E + (tid & 31) * 32));
+      {
+        const int n0 = split_at(P.T * P.E, b, G), n1 = split_at(P.T * P.E, b + 1, G);
+#pragma unroll 1
+        for (int i = n0 + tid; i < n1; i += CT) {
+          P.lacc[i] = 0;
+          P.lacc[2 * static_cast<size_t>(P.T) * P.E + i] = 0;
+          P.lacc[4 * static_cast<size_t>(P.T) * P.E + i] = 0;
+          P.lbad[i] = 0;
+        }
+      }
+#pragma unroll 1
+      for (int i = tid; i < P.T * nr_out; i += CT) {
+        const int t = i / nr_out, r = i - t * nr_out;
+        ysl[t * P.rpc + r] = bf16_bits_to_float(P.x[static_cast<size_t>(t) * P.d + r0 + r]);
+      }
+      __threadfence();
+      named_sync(1, CT);
+      // the counters advance by L per CTA and launch, in step with the tags
+      if (tid == 0) {
+        cnt_add(kCntZero, static_cast<unsigned>(P.L));
+        if (!ds_aborted(S)) cnt_wait(kCntZero, (base + P.L) * G, S, P.status, 19, deadline);
+      }
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      named_sync(1, CT);
+      if (!ds_aborted(S)) ds_partial_logits(Q, wsl, ysl, nr_out, 0, CT);
+      __threadfence();
+      named_sync(1, CT);
+      if (tid == 0) cnt_add(kCntLogits, static_cast<unsigned>(P.L));
+    } else if (tid == 0) {
+      cnt_add(kCntZero, static_cast<unsigned>(P.L));  // no logits here, but the counters advance in step
+      cnt_add(kCntLogits, static_cast<unsigned>(P.L));
+    }
 #pragma unroll 1
     for (int l = 0; l < P.L; ++l) {
       const uint32_t tag = base + 1 + static_cast<uint32_t>(l);
@@ -1299,53 +1398,50 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
       const bool traced = trace != nullptr && l < 2 && tid == 0;
       unsigned long long* tdet = (trace != nullptr && l == dl) ? trace : nullptr;
       if (traced) trace[8 * l] = global_timer_ns();
-      // ---- x of this layer: layer l > 0 waits until every CTA has written
-      // its part of layer l - 1's output (and so has read all of layer l - 1)
-      if (ROUTE && l > 0) {
-        if (tid == 0 && !ds_aborted(S)) cnt_wait(kCntOut, (base + l) * G, S, P.status, 20, deadline);
-        named_sync(1, CT);
-        if (tdet && tid == 0) tdet[31] = global_timer_ns();
-      }
-      if (!ds_aborted_warp(S))
-        ds_read_x<BITS, GBPL>(P, ROUTE ? l : 0, tag, wr_rows ? xs : nullptr, xq, xres, r0, r1, S, deadline, CT);
+      int nu = 0;
       if (ROUTE) {
 #pragma unroll 1
         for (int e = tid; e < P.E; e += CT) R.slot_s[e] = __ldg(P.slot_of + static_cast<size_t>(l) * P.E + e);
-      }
-      named_sync(1, CT);
-      if (traced) trace[8 * l + 1] = global_timer_ns();
-      int nu = 0;
-      if (ROUTE) {
-        // ---- router rows of this CTA
-        if (wr_rows) {
-          if (ds_wait_warp(&S->wr_full, l & 1, S, deadline)) {
-            if (!ds_aborted_warp(S)) ds_router(P, l, tag, wrs, xs, e0, e1, CW);
-          } else if (lane == 0 && !ds_aborted(S)) {
-            ds_abort(S, P.status, 1);
+        // the logits of this layer are complete once every CTA has added its
+        // partials: at the end of the previous layer (with its output rows),
+        // or in the prologue for layer 0
+        if (tid == 0 && !ds_aborted(S)) {
+          if (l == 0) cnt_wait(kCntLogits, (base + P.L) * G, S, P.status, 22, deadline);
+          else cnt_wait(kCntOut, (base + l) * G, S, P.status, 20, deadline);
+          __threadfence();
+        }
+        named_sync(1, CT);
+        if (tdet && tid == 0) tdet[31] = global_timer_ns();
+        if (traced) trace[8 * l + 1] = global_timer_ns();
+        // the next layer's accumulator: every CTA read it in the previous layer
+        if (l + 1 < P.L) {
+          const size_t n0 = split_at(P.T * P.E, b, G), n1 = split_at(P.T * P.E, b + 1, G);
+          const size_t nb1 = static_cast<size_t>((l + 1) & 1) * P.T * P.E;
+#pragma unroll 1
+          for (size_t i = n0 + tid; i < n1; i += CT) {
+            P.lacc[nb1 + i] = 0;
+            P.lacc[2 * static_cast<size_t>(P.T) * P.E + nb1 + i] = 0;
+            P.lacc[4 * static_cast<size_t>(P.T) * P.E + nb1 + i] = 0;
+            P.lbad[nb1 + i] = 0;
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&S->wr_empty);
         }
-        // every CTA counts its logit rows as written, then waits for all
-        named_sync(1, CT);
-        if (tid == 0) {
-          cnt_add(kCntLogits);
-          if (!ds_aborted(S)) cnt_wait(kCntLogits, (base + l + 1) * G, S, P.status, 22, deadline);
-        }
-        named_sync(1, CT);
-        if (traced) trace[8 * l + 2] = global_timer_ns();
-        // ---- top-k (warp t) and grouping (all)
-        // (publisher: the CTA that writes this layer's routing record)
+        // ---- top-k (warp t) while the other warps read x for gate/up
         float* pub = publisher ? reinterpret_cast<float*>(P.rec + static_cast<size_t>(l) * P.rec_bytes + P.ro.logits)
                                : nullptr;
-        if (warp < P.T && !ds_aborted_warp(S))
-          ds_topk(Q, warp, tag, pub, reinterpret_cast<uint32_t*>(smem + P.sm_x) + warp * P.E, S, deadline,
-                  (tdet && warp == 0) ? tdet : nullptr);
+        if (warp < P.T) {
+          if (!ds_aborted_warp(S))
+            ds_topk(Q, l, warp, pub,
+                    (tdet && warp == 0) ? tdet : nullptr);
+        } else if (!ds_aborted_warp(S)) {
+          ds_read_x<BITS, GBPL>(P, l, tag, nullptr, xq, xres, r0, r1, S, deadline, P.T * 32, CT - P.T * 32);
+          if (tdet && tid == P.T * 32) tdet[24] = global_timer_ns();
+        }
         if (tdet && tid == 0) tdet[20] = global_timer_ns();
         named_sync(1, CT);
+        if (traced) trace[8 * l + 2] = global_timer_ns();
         if (P.T > 1) {  // (one token: the top-k warp has grouped its pairs)
-          if (!ds_aborted_warp(S)) ds_group(Q, S, np, CT);
-          else named_sync(1, CT), named_sync(1, CT);
+          if (!ds_aborted_warp(S)) ds_group(Q, S, np, CT, reinterpret_cast<int*>(smem + P.sm_x));
+          else named_sync(1, CT), named_sync(1, CT), named_sync(1, CT);
         }
         // the routing is complete unless some thread gave up: one decision
         // for every consumer thread, which the producer reads behind route_bar
@@ -1358,6 +1454,7 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
         }
         if (route_bad) break;  // every consumer thread leaves the layer loop here
       } else {
+        if (!ds_aborted_warp(S)) ds_read_x<BITS, GBPL>(P, 0, tag, nullptr, xq, xres, r0, r1, S, deadline, 0, CT);
         // the grouping was written by moe_group_tokens
         const int nug = min(max(__ldcg(P.g.n_uniq), 0), min(np, P.E));
 #pragma unroll 1
@@ -1377,10 +1474,7 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
           }
           R.uniq_slot[u] = slot;
         }
-        if (tid == 0) {
-          S->n_uniq = nug;
-          cnt_add(kCntLogits);  // no logits here, but the counters advance in step
-        }
+        if (tid == 0) S->n_uniq = nug;
         const bool route_bad = named_sync_or(1, CT, ds_aborted(S));
         nu = route_bad ? 0 : nug;
         if (tid == 0) {
@@ -1411,8 +1505,11 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
         }
       }
       named_sync(1, CT);
-      // every CTA counts its h blocks as written, then waits for all; the
+      // every CTA counts its h blocks as written (and the next layer's
+      // zeroed accumulator share behind a fence), then waits for all; the
       // publishing CTA writes the layer's routing record meanwhile
+      if (ROUTE && l + 1 < P.L) __threadfence();
+      named_sync(1, CT);
       if (tid == 0) cnt_add(kCntH);
       if (publisher) ds_publish(Q, l, np, nu, CT);
       if (tid == 0 && !ds_aborted(S)) cnt_wait(kCntH, (base + l + 1) * G, S, P.status, 23, deadline);
@@ -1426,8 +1523,8 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
       // previous use in this layer is still pending.
       const int sh = (P.has_shared && has_rows) ? 1 : 0;
       const int n_dn = has_rows ? nu + sh : 0;
-      const int nr_out = r1 - r0;
       const uint32_t grp0 = seq;  // sequence number of this layer's first down group
+      bool sliced = false;
 #pragma unroll 1
       for (int i0 = 0; i0 < n_dn;) {
         int i1 = i0, rows = 0;
@@ -1450,6 +1547,13 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
         if (!ds_aborted(S)) ds_stage_h<DBPL>(P, R, np, i0, i1, sh, tag, hq, S, deadline, CT);
         named_sync(1, CT);
         if (traced && i0 == 0) trace[8 * l + 5] = global_timer_ns();
+        if (ROUTE && i0 == 0 && l + 1 < P.L && !ds_aborted(S)) {
+          // the next router's columns, for the partial logits at the end of
+          // this layer: issued once this CTA's reads of other CTAs' words
+          // are done, so that its many small copies delay none of them
+          ds_wslice_load(P, l + 1, wsl, r0, r1, tid, CT);
+          sliced = true;
+        }
         // each warp takes whole stages; the hq row of stage i is the rows of
         // the stages before it in this round
 #pragma unroll 1
@@ -1499,6 +1603,7 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
         i0 = i1;
       }
       seq += has_rows ? (nu + P.gpd - 1) / P.gpd : 0;
+      if (ROUTE && !sliced && has_rows && l + 1 < P.L && !ds_aborted(S)) ds_wslice_load(P, l + 1, wsl, r0, r1, tid, CT);
       if (traced) trace[8 * l + 6] = global_timer_ns();
       // the down phase is done with the buffers: this warp's shared-expert
       // gate/up rows of the next layer go in now
@@ -1536,15 +1641,29 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
           } else {
             const __nv_bfloat162 hv = __floats2bfloat162_rn(a0, a1);
             *reinterpret_cast<__nv_bfloat162*>(yl + o * 2) = hv;
-            if (ROUTE && l + 1 < P.L)
+            if (ROUTE && l + 1 < P.L) {
               st_ll(yll + o / 2, ll_word(*reinterpret_cast<const uint32_t*>(&hv), tag));
+              ysl[t * P.rpc + rr] = __low2float(hv);  // the next layer's input, as it will read it
+              ysl[t * P.rpc + rr + 1] = __high2float(hv);
+            }
           }
         }
       }
       if (l + 2 == P.L && tid == 0) grid_dep_launch();
       named_sync(1, CT);
-      // this CTA's output rows are written and it has read everything of
-      // layer l that other CTAs wrote
+      if (ROUTE && l + 1 < P.L) {
+        // the next layer's logits: this CTA's rows of its input against its
+        // columns of the next router (loaded during this layer's down phase;
+        // the warp's shared-expert copies for the next layer, issued after
+        // them, may stay in flight)
+        cp_async_wait_pending(n_pre);
+        named_sync(1, CT);
+        if (!ds_aborted(S) && has_rows) ds_partial_logits(Q, wsl, ysl, nr_out, (l + 1) & 1, CT);
+        __threadfence();
+        named_sync(1, CT);
+      }
+      // this CTA's output rows and its partial logits are written, and it has
+      // read everything of layer l that other CTAs wrote
       if (tid == 0) cnt_add(kCntOut);
       if (traced) trace[8 * l + 7] = global_timer_ns();
     }
@@ -1572,6 +1691,7 @@ __global__ void ds_skip_tags_kernel(int G) {
   atomicExch(&g_ds_cnt[kCntLogits], e * G);
   atomicExch(&g_ds_cnt[kCntH], e * G);
   atomicExch(&g_ds_cnt[kCntOut], e * G);
+  atomicExch(&g_ds_cnt[kCntZero], e * G);
 }
 
 // ------------------------------------------------------------------ host side
@@ -1618,7 +1738,7 @@ bool decode_geometry_ok(int d, int f) {
 
 size_t decode_exchange_bytes(const moe_layer_cfg& c, int T) {
   const size_t n_rows = static_cast<size_t>(T) * c.k + (c.n_shared ? T : 0);
-  const size_t lg = ds_align(static_cast<size_t>(kDsLogitCopies) * T * c.E * 8, 256);
+  const size_t lg = ds_align(2 * static_cast<size_t>(T) * c.E * (3 * 8 + 4), 256);  // fixed-point logits + flags
   const size_t h = ds_align(n_rows * (c.f / kBlock) * kQW * 8, 256);
   const size_t y = ds_align(2 * static_cast<size_t>(T) * (c.d / 2) * 8, 256);
   return lg + h + y;
@@ -1645,8 +1765,8 @@ cudaError_t decode_init(Ctx& ctx) {
     const unsigned start = (static_cast<unsigned>(rd()) & 0xfff00000u) | 0x00010000u;
     e = cudaMemcpyToSymbol(g_ds_epoch, &start, sizeof(start));
     if (e != cudaSuccess) return e;
-    unsigned cnt[96] = {};
-    cnt[kCntLogits] = cnt[kCntH] = cnt[kCntOut] = start * static_cast<unsigned>(ctx.num_sms);
+    unsigned cnt[128] = {};
+    cnt[kCntLogits] = cnt[kCntH] = cnt[kCntOut] = cnt[kCntZero] = start * static_cast<unsigned>(ctx.num_sms);
     e = cudaMemcpyToSymbol(g_ds_cnt, cnt, sizeof(cnt));
     if (e != cudaSuccess) return e;
   }
@@ -1725,10 +1845,10 @@ cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const St
   if (a.g != nullptr) P.g = *a.g;
   {
     char* ex = a.exchange;
-    const size_t lg = ds_align(static_cast<size_t>(kDsLogitCopies) * T * c.E * 8, 256);
+    const size_t lg = ds_align(2 * static_cast<size_t>(T) * c.E * (3 * 8 + 4), 256);
     const size_t h = ds_align(static_cast<size_t>(n_rows) * nbf * kQW * 8, 256);
-    const size_t y = ds_align(2 * static_cast<size_t>(T) * (c.d / 2) * 8, 256);
-    P.logits_ll = reinterpret_cast<unsigned long long*>(ex);
+    P.lacc = reinterpret_cast<long long*>(ex);
+    P.lbad = reinterpret_cast<int*>(ex + 6 * static_cast<size_t>(T) * c.E * 8);
     P.h_ll = reinterpret_cast<unsigned long long*>(ex + lg);
     P.y_ll = reinterpret_cast<unsigned long long*>(ex + lg + h);
   }
@@ -1753,7 +1873,6 @@ cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const St
   P.gran = gran;
   P.n_units = c.d / gran;
   P.rpc = gran * ((P.n_units + G - 1) / G);
-  const int wr_rows = a.route ? (c.E + G - 1) / G : 0;
   // ring slots hold a group of down stages (this CTA's output rows of up to
   // kDsGpd experts); a gate/up task is the two rows of one channel
   P.dn_stride = static_cast<int>(ds_align(static_cast<size_t>(P.rpc) * (P.dn_row + P.dn_sc), 16));
@@ -1781,21 +1900,23 @@ cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const St
   o = ds_align(o + hs_bytes, 128);
   P.sm_xq = static_cast<int>(o);
   o = ds_align(o + static_cast<size_t>(T) * kQW * nbd * 4, 128);
-  P.sm_wr = static_cast<int>(o);
-  o = ds_align(o + static_cast<size_t>(wr_rows) * c.d * 4, 128);
+  // the next router's columns of this CTA's rows, and its rows of the next input
+  P.sm_ws = static_cast<int>(o);
+  o = ds_align(o + (a.route ? static_cast<size_t>(c.E) * P.rpc * 4 : 0), 128);
+  P.sm_ysl = static_cast<int>(o);
+  o = ds_align(o + static_cast<size_t>(T) * P.rpc * 4, 128);
   P.sm_shdn = static_cast<int>(o);
   o = ds_align(o + 2 * static_cast<size_t>(P.dn_stride), 128);
   const size_t before_gub = o;
   // then the per-warp gate/up buffers, the staging area and the ring. The
-  // staging area holds raw x for the router, then the top-k key rows; the
-  // gate/up buffers and the staging area together hold the quantised h rows
-  // of a round of down stages (at least T rows). The first of (gate/up
-  // depth, experts per down group) from (4, 6) down to (2, 1) that leaves
-  // room for two ring slots wins.
-  const size_t xs_bytes = a.route ? static_cast<size_t>(T) * c.d * 2 : 0;
+  // staging area holds the top-k key rows; the gate/up buffers and the
+  // staging area together hold the quantised h rows of a round of down
+  // stages (at least T rows). The first of (gate/up depth, experts per down
+  // group) from (4, 6) down to (2, 1) that leaves room for two ring slots
+  // wins.
   const size_t hq_row = static_cast<size_t>(kQW) * nbf * 4;
-  const size_t keys_bytes = static_cast<size_t>(T) * c.E * 4;
-  size_t x_min = xs_bytes > keys_bytes ? xs_bytes : keys_bytes;
+  const size_t keys_bytes = static_cast<size_t>(T) * c.k * 4;  // the grouping's sort keys
+  size_t x_min = keys_bytes;
   if (x_min < T * hq_row) x_min = T * hq_row;
   int n_ring = 0;
   size_t fixed = 0, x_bytes = 0;
