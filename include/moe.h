@@ -292,8 +292,10 @@ MOE_API moe_status moe_layer_routing(const moe_layer_cfg* cfg, int T, void* ws, 
  * the per-layer join of the pages' engine between them: vramglass.com,
  * section その2). Per layer the same step as moe_layer_forward (router,
  * top-k, grouping, experts, combine; with cfg->residual, y[l] = x_l + moe(x_l)).
- * While layer l runs, layer l + 1's router rows and shared expert, which do
- * not depend on x, are already being fetched.
+ * While layer l runs, layer l + 1's router columns and shared expert, which
+ * do not depend on x, are already being fetched, and layer l + 1's logits are
+ * summed from every CTA's rows of y[l] as they are written (exact fixed-point
+ * partial sums, so the logits do not depend on the order of the adds).
  *   - T: 1..MOE_DECODE_MAX_T tokens; cfg->E <= 512; L >= 1.
  *   - w_router: [L, E, d] fp32; logit_bias: NULL or [L, T, E] fp32;
  *     slot_of: [L, E] int32 (the stack's slot table, one row per layer);
