@@ -1050,10 +1050,10 @@ __device__ __noinline__ void gu_publish(const DSParams& P, int u, int cb, int np
 // expert's T rows (when stage 0 is in the round) followed by the routed rows
 // [uniq_off[ua], uniq_off[ub]), one contiguous range of h. A thread loads up
 // to kHB 16-byte units at once and re-polls, together, only the words that
-// were not there yet.
-constexpr int kHB = 4;
-
-template <int DBPL>
+// were not there yet. kHB: 6 with the 15 consumer warps of the 2-bit kernel
+// (one token's 11 rows in one round of loads), 4 with the 11 of the 3-bit one
+// (fewer registers to spare).
+template <int DBPL, int kHB>
 __device__ void ds_stage_h(const DSParams& P, const DSRoute& R, int np, int i0, int i1, int sh, uint32_t tag,
                            int* hq, DSShared* S, uint64_t deadline, int CT) {
   const int nbf = P.f / kBlock;
@@ -1544,7 +1544,7 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
           if (tid == 0) ds_abort(S, P.status, 24);
           break;
         }
-        if (!ds_aborted(S)) ds_stage_h<DBPL>(P, R, np, i0, i1, sh, tag, hq, S, deadline, CT);
+        if (!ds_aborted(S)) ds_stage_h<DBPL, BITS == 2 ? 6 : 4>(P, R, np, i0, i1, sh, tag, hq, S, deadline, CT);
         named_sync(1, CT);
         if (traced && i0 == 0) trace[8 * l + 5] = global_timer_ns();
         if (ROUTE && i0 == 0 && l + 1 < P.L && !ds_aborted(S)) {

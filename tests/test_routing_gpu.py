@@ -8,8 +8,9 @@ oracle; the selected experts bit-exactly equal to the oracle's selection on
 the kernel's own fp32 logits, and equal to the fp64 selection except at fp64
 near-ties; the gates; and every grouping array bit-exactly. Tie cases set
 W_r = 0 so that the logits are exactly the given bias rows: heavy ties, +-0,
-+-inf and NaN, and rows where more than 32 values reach the k-th largest
-lane maximum (the selection's slower branch)."""
++-inf and NaN, and rows where 32 or 33 values tie at the top. Inputs scaled
+by 2^40 and 2^90 make the CTAs' partial logits large enough to use the upper
+parts of the kernel's fixed-point accumulators."""
 import numpy as np
 import pytest
 import torch
@@ -133,6 +134,22 @@ def test_fused_decode_selection_on_ties_nan_and_zeros(cfg):
     num = ~np.isnan(rows)
     assert np.array_equal(lg[num], rows[num])
     assert np.array_equal(r["idx"], O.topk(rows.astype(np.float64), cfg.k))
+
+
+@pytest.mark.parametrize("shift", [40, 90])
+def test_fused_decode_logits_of_large_inputs(shift):
+    """x ~ N(0, 2^(2 shift)): each CTA's partial logits are ~2^(shift-4), above
+    2^22 (shift 40) and above 2^76 (shift 90), so they are carried by the
+    accumulators in units of 2^22 and 2^76. The logits stay within 1e-5 of the
+    fp64 oracle's and the selection is exact."""
+    base = _layer(M.FULL, 82)
+    x = synth.activations(2, base.cfg.d, 1700 + shift, scale=2.0 ** shift)
+    L = base.with_inputs(x, None)
+    y, ws = L.forward()
+    torch.cuda.synchronize()
+    assert H.ctx().check_device_status() == M.OK
+    r = check_published_routing(L, ws)
+    assert np.abs(r["logits"]).max() > 2.0 ** (shift - 10)
 
 
 def test_fused_decode_routing_256_experts_and_renorm0():
