@@ -11,22 +11,25 @@
 // steps around ~16-50 MB of weight reads. This kernel keeps that chain short:
 //
 //  * One CTA per SM (a cooperative launch, so all CTAs are resident), one
-//    producer warp issuing cp.async.bulk copies and 15 (2-bit) or 11 (3-bit)
-//    consumer warps.
-//  * Cross-CTA data moves as 64-bit words that carry a 32-bit payload and a
-//    32-bit tag naming the layer; a reader polls the words themselves until
-//    every tag matches. There are no grid barriers, fences or atomics on the
-//    critical path. Tags come from a per-device counter that every launch
-//    advances, so words left by earlier launches never match.
-//  * Per layer: x (every CTA reads all of it) -> router rows of this CTA ->
-//    logits words -> top-k and grouping in every CTA -> the producer issues
-//    ALL of this CTA's routed gate/up and down rows at once into two
-//    fixed-slot rings -> gate/up + SwiGLU, each 32-channel block of h
-//    requantised to int16 by the CTA that owns it and published as words ->
-//    every CTA stages all of h and computes its slice of output rows for
-//    every expert -> combine -> output words (the next layer's x).
-//  * Layer l + 1's router rows and shared expert do not depend on x: the
-//    producer fetches them while layer l is still running.
+//    producer warp issuing cp.async.bulk copies of down rows and 15 (2-bit)
+//    or 11 (3-bit) consumer warps.
+//  * Cross-CTA data (x, h) moves as 64-bit words that carry a 32-bit payload
+//    and a 32-bit tag naming the layer; a reader polls the words themselves
+//    until every tag matches. Tags come from a per-device counter that every
+//    launch advances, so words left by earlier launches never match. Where
+//    every CTA must have finished a step (the logits, h), each adds 1 to a
+//    per-device completion counter and one thread per CTA waits for it.
+//  * Per layer: the logits are already summed (below) -> top-k and grouping
+//    in every CTA while the other warps read x -> each consumer warp streams
+//    the gate/up rows of its own channel tasks with cp.async while the
+//    producer streams this CTA's down rows into a ring -> gate/up + SwiGLU,
+//    each 32-channel block of h requantised to int16 by the CTA that owns it
+//    and published as words -> every CTA stages all of h and computes its
+//    slice of output rows for every expert -> combine -> output words (the
+//    next layer's x) -> this CTA's partial logits of the next layer from
+//    those rows, added into exact fixed-point accumulators.
+//  * Layer l + 1's router columns and shared expert do not depend on x: they
+//    are fetched while layer l is still running.
 //
 // Every wait is bounded by a global-timer deadline; on expiry the kernel
 // records MOE_ETIMEOUT in the context's status word, stops working and
@@ -54,10 +57,13 @@ constexpr int kDsPollNs = 64;      // back-off between polls of words that were 
 // the number of layers; tags of a launch are base + 1 .. base + L.
 __device__ unsigned int g_ds_epoch;
 __device__ unsigned int g_ds_exit;
-// Completion counters of the three exchanges of a layer (logits, h, layer
-// output), one per 128-byte line: every CTA adds 1 per layer once its part
-// is written, so after layer l of a launch with tag base `base` each holds
-// (base + l + 1) * G (mod 2^32). They advance in step with the tag counter.
+// Completion counters, one per 128-byte line: kCntH (a layer's h blocks) and
+// kCntOut (a layer's output rows and the next layer's partial logits) take 1
+// from every CTA per layer, so after layer l of a launch with tag base
+// `base` each holds (base + l + 1) * G (mod 2^32); kCntZero (the first
+// accumulator set zeroed) and kCntLogits (layer 0's partial logits added)
+// take L from every CTA in the prologue. All advance in step with the tag
+// counter.
 constexpr int kCntLogits = 0, kCntH = 32, kCntOut = 64, kCntZero = 96;
 __device__ unsigned int g_ds_cnt[128];
 
