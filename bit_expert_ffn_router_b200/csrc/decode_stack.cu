@@ -1419,18 +1419,6 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
         named_sync(1, CT);
         if (tdet && tid == 0) tdet[31] = global_timer_ns();
         if (traced) trace[8 * l + 1] = global_timer_ns();
-        // the next layer's accumulator: every CTA read it in the previous layer
-        if (l + 1 < P.L) {
-          const size_t n0 = split_at(P.T * P.E, b, G), n1 = split_at(P.T * P.E, b + 1, G);
-          const size_t nb1 = static_cast<size_t>((l + 1) & 1) * P.T * P.E;
-#pragma unroll 1
-          for (size_t i = n0 + tid; i < n1; i += CT) {
-            P.lacc[nb1 + i] = 0;
-            P.lacc[2 * static_cast<size_t>(P.T) * P.E + nb1 + i] = 0;
-            P.lacc[4 * static_cast<size_t>(P.T) * P.E + nb1 + i] = 0;
-            P.lbad[nb1 + i] = 0;
-          }
-        }
         // ---- top-k (warp t) while the other warps read x for gate/up
         float* pub = publisher ? reinterpret_cast<float*>(P.rec + static_cast<size_t>(l) * P.rec_bytes + P.ro.logits)
                                : nullptr;
@@ -1438,8 +1426,24 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
           if (!ds_aborted_warp(S))
             ds_topk(Q, l, warp, pub,
                     (tdet && warp == 0) ? tdet : nullptr);
-        } else if (!ds_aborted_warp(S)) {
-          ds_read_x<BITS, GBPL>(P, l, tag, nullptr, xq, xres, r0, r1, S, deadline, P.T * 32, CT - P.T * 32);
+        } else {
+          // the next layer's accumulator set (every CTA read it in the
+          // previous layer), zeroed off the top-k's path; the fence before
+          // this CTA's h count publishes it
+          if (l + 1 < P.L) {
+            const size_t n0 = split_at(P.T * P.E, b, G), n1 = split_at(P.T * P.E, b + 1, G);
+            const size_t nb1 = static_cast<size_t>((l + 1) & 1) * P.T * P.E;
+            const size_t tp = 2 * static_cast<size_t>(P.T) * P.E;  // between the parts
+#pragma unroll 1
+            for (size_t i = n0 + tid - P.T * 32; i < n1; i += CT - P.T * 32) {
+              P.lacc[nb1 + i] = 0;
+              P.lacc[tp + nb1 + i] = 0;
+              P.lacc[2 * tp + nb1 + i] = 0;
+              P.lbad[nb1 + i] = 0;
+            }
+          }
+          if (!ds_aborted_warp(S))
+            ds_read_x<BITS, GBPL>(P, l, tag, nullptr, xq, xres, r0, r1, S, deadline, P.T * 32, CT - P.T * 32);
           if (tdet && tid == P.T * 32) tdet[24] = global_timer_ns();
         }
         if (tdet && tid == 0) tdet[20] = global_timer_ns();
