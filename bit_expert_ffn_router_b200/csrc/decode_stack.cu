@@ -57,13 +57,13 @@ constexpr int kDsPollNs = 64;      // back-off between polls of words that were 
 // the number of layers; tags of a launch are base + 1 .. base + L.
 __device__ unsigned int g_ds_epoch;
 __device__ unsigned int g_ds_exit;
-// Completion counters, one per 128-byte line: kCntH (a layer's h blocks) and
-// kCntOut (a layer's output rows and the next layer's partial logits) take 1
-// from every CTA per layer, so after layer l of a launch with tag base
-// `base` each holds (base + l + 1) * G (mod 2^32); kCntZero (the first
-// accumulator set zeroed) and kCntLogits (layer 0's partial logits added)
-// take L from every CTA in the prologue. All advance in step with the tag
-// counter.
+// Completion counters, one per 128-byte line: kCntOut (a layer's output rows
+// and the next layer's partial logits) takes 1 from every CTA per layer, so
+// after layer l of a launch with tag base `base` it holds (base + l + 1) * G
+// (mod 2^32); kCntZero (the first two accumulator sets zeroed) and
+// kCntLogits (layer 0's partial logits added) take L from every CTA in the
+// prologue. All advance in step with the tag counter. (kCntH, once the count
+// of a layer's h blocks, is no longer added to: the h words carry tags.)
 constexpr int kCntLogits = 0, kCntH = 32, kCntOut = 64, kCntZero = 96;
 __device__ unsigned int g_ds_cnt[128];
 
@@ -111,9 +111,9 @@ struct DSParams {
   size_t rec_bytes;
   RecOff ro;
   GroupPtrs g;                  // not route: the given grouping
-  long long* lacc;                // [3, 2, T, E] router logits in fixed point: [part][parity]; parts in
-                                  // units of 2^-32, 2^22 and 2^76
-  int* lbad;                      // [2, T, E] flags: 1 a partial was not finite, 2 / 4 part 1 / 2 used
+  long long* lacc;                // [3, 3, T, E] router logits in fixed point: [part][layer % 3]; parts
+                                  // in units of 2^-32, 2^22 and 2^76
+  int* lbad;                      // [3, T, E] flags: 1 a partial was not finite, 2 / 4 part 1 / 2 used
   unsigned long long* h_ll;       // [n_rows, f/32, kQW]
   unsigned long long* y_ll;       // [2, T, d/2]
   int* status;
@@ -503,10 +503,10 @@ __device__ __noinline__ void ds_topk(const DSParams& P, int l, int t, float* pub
   DSShared* S = reinterpret_cast<DSShared*>(ds_smem);
   constexpr int KPL = kDsMaxE / 32;  // keys a lane holds
   const int lane = threadIdx.x & 31;
-  const size_t o = (static_cast<size_t>(l & 1) * T + t) * E;
+  const size_t o = (static_cast<size_t>(l % 3) * T + t) * E;
   const long long* const acc = P.lacc + o;
   const int* const flg = P.lbad + o;
-  const size_t part = 2 * static_cast<size_t>(T) * E;  // distance between the parts' accumulators
+  const size_t part = 3 * static_cast<size_t>(T) * E;  // distance between the parts' accumulators
   const float* const bias = P.bias != nullptr ? P.bias + (static_cast<size_t>(l) * T + t) * E : nullptr;
   long long w[KPL];
   int fl[KPL];
@@ -794,7 +794,7 @@ __device__ __noinline__ void ds_partial_logits(const DSParams& P, const float* w
                                                int buf, int CT) {
   const int E = P.E, T = P.T, rpc = P.rpc;  // in registers (P is in shared memory)
   long long* const acc = P.lacc + static_cast<size_t>(buf) * T * E;
-  const size_t part = 2 * static_cast<size_t>(T) * E;
+  const size_t part = 3 * static_cast<size_t>(T) * E;
   int* const badf = P.lbad + static_cast<size_t>(buf) * T * E;
 #pragma unroll 1
   for (int e = threadIdx.x; e < E; e += CT) {
@@ -1357,19 +1357,20 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
     // this warp's shared-expert gate/up rows of the next layer, issued ahead
     int n_pre = (P.has_shared && !ds_aborted(S)) ? gu_prefetch_shared<CW>(Q, 0, nsh, sb0) : 0;
     if (ROUTE) {
-      // ---- layer 0's logits: every CTA zeroes its share of the first
-      // accumulator, waits for all, then adds its rows of x against its
-      // columns of layer 0's router
+      // ---- layer 0's logits: every CTA zeroes its share of the first two
+      // accumulator sets (layers 0 and 1), waits for all, then adds its rows
+      // of x against its columns of layer 0's router
       ds_wslice_load(P, 0, wsl, r0, r1, tid, CT);
       if (P.bias != nullptr && tid < P.T * 32 && (tid & 31) * 32 < P.E)  // layer 0's bias rows into L2
         asm volatile("prefetch.global.L2 [%0];" ::"l"(P.bias + static_cast<size_t>(tid >> 5) * P.E + (tid & 31) * 32));
       {
-        const int n0 = split_at(P.T * P.E, b, G), n1 = split_at(P.T * P.E, b + 1, G);
+        const int n0 = split_at(2 * P.T * P.E, b, G), n1 = split_at(2 * P.T * P.E, b + 1, G);
+        const size_t tp = 3 * static_cast<size_t>(P.T) * P.E;  // between the parts
 #pragma unroll 1
         for (int i = n0 + tid; i < n1; i += CT) {
           P.lacc[i] = 0;
-          P.lacc[2 * static_cast<size_t>(P.T) * P.E + i] = 0;
-          P.lacc[4 * static_cast<size_t>(P.T) * P.E + i] = 0;
+          P.lacc[tp + i] = 0;
+          P.lacc[2 * tp + i] = 0;
           P.lbad[i] = 0;
         }
       }
@@ -1427,13 +1428,14 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
             ds_topk(Q, l, warp, pub,
                     (tdet && warp == 0) ? tdet : nullptr);
         } else {
-          // the next layer's accumulator set (every CTA read it in the
-          // previous layer), zeroed off the top-k's path; the fence before
-          // this CTA's h count publishes it
-          if (l + 1 < P.L) {
+          // the accumulator set of layer l + 2 (every CTA read it as layer
+          // l - 1's), zeroed off the top-k's path; the fence before this
+          // CTA's count at the end of the layer publishes it before any CTA
+          // adds to it (at the end of layer l + 1)
+          if (l + 2 < P.L) {
             const size_t n0 = split_at(P.T * P.E, b, G), n1 = split_at(P.T * P.E, b + 1, G);
-            const size_t nb1 = static_cast<size_t>((l + 1) & 1) * P.T * P.E;
-            const size_t tp = 2 * static_cast<size_t>(P.T) * P.E;  // between the parts
+            const size_t nb1 = static_cast<size_t>((l + 2) % 3) * P.T * P.E;
+            const size_t tp = 3 * static_cast<size_t>(P.T) * P.E;  // between the parts
 #pragma unroll 1
             for (size_t i = n0 + tid - P.T * 32; i < n1; i += CT - P.T * 32) {
               P.lacc[nb1 + i] = 0;
@@ -1515,14 +1517,10 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
         }
       }
       named_sync(1, CT);
-      // every CTA counts its h blocks as written (and the next layer's
-      // zeroed accumulator share behind a fence), then waits for all; the
-      // publishing CTA writes the layer's routing record meanwhile
-      if (ROUTE && l + 1 < P.L) __threadfence();
-      named_sync(1, CT);
-      if (tid == 0) cnt_add(kCntH);
+      // the publishing CTA writes the layer's routing record; the h words
+      // of the other CTAs are tagged, so the staging below waits for each
+      // word itself (no count of the CTAs that have published)
       if (publisher) ds_publish(Q, l, np, nu, CT);
-      if (tid == 0 && !ds_aborted(S)) cnt_wait(kCntH, (base + l + 1) * G, S, P.status, 23, deadline);
       named_sync(1, CT);
       if (traced) trace[8 * l + 4] = global_timer_ns();
 
@@ -1668,7 +1666,7 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
         // them, may stay in flight)
         cp_async_wait_pending(n_pre);
         named_sync(1, CT);
-        if (!ds_aborted(S) && has_rows) ds_partial_logits(Q, wsl, ysl, nr_out, (l + 1) & 1, CT);
+        if (!ds_aborted(S) && has_rows) ds_partial_logits(Q, wsl, ysl, nr_out, (l + 1) % 3, CT);
         __threadfence();
         named_sync(1, CT);
       }
@@ -1748,7 +1746,7 @@ bool decode_geometry_ok(int d, int f) {
 
 size_t decode_exchange_bytes(const moe_layer_cfg& c, int T) {
   const size_t n_rows = static_cast<size_t>(T) * c.k + (c.n_shared ? T : 0);
-  const size_t lg = ds_align(2 * static_cast<size_t>(T) * c.E * (3 * 8 + 4), 256);  // fixed-point logits + flags
+  const size_t lg = ds_align(3 * static_cast<size_t>(T) * c.E * (3 * 8 + 4), 256);  // fixed-point logits + flags
   const size_t h = ds_align(n_rows * (c.f / kBlock) * kQW * 8, 256);
   const size_t y = ds_align(2 * static_cast<size_t>(T) * (c.d / 2) * 8, 256);
   return lg + h + y;
@@ -1855,10 +1853,10 @@ cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const St
   if (a.g != nullptr) P.g = *a.g;
   {
     char* ex = a.exchange;
-    const size_t lg = ds_align(2 * static_cast<size_t>(T) * c.E * (3 * 8 + 4), 256);
+    const size_t lg = ds_align(3 * static_cast<size_t>(T) * c.E * (3 * 8 + 4), 256);
     const size_t h = ds_align(static_cast<size_t>(n_rows) * nbf * kQW * 8, 256);
     P.lacc = reinterpret_cast<long long*>(ex);
-    P.lbad = reinterpret_cast<int*>(ex + 6 * static_cast<size_t>(T) * c.E * 8);
+    P.lbad = reinterpret_cast<int*>(ex + 9 * static_cast<size_t>(T) * c.E * 8);
     P.h_ll = reinterpret_cast<unsigned long long*>(ex + lg);
     P.y_ll = reinterpret_cast<unsigned long long*>(ex + lg + h);
   }
