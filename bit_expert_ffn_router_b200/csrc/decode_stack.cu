@@ -491,12 +491,11 @@ __device__ __forceinline__ void ds_wslice_load(const DSParams& P, int l, float* 
 // Warp t: reads token t's E <= 512 logits (all of a lane's 16 at once: the
 // fixed-point sums every CTA added, plus the bias), turns them into order
 // keys held in registers, selects its k experts and gates into R.
-// Selection: the candidates at or above the k-th largest lane maximum ranked
-// directly, or (more than 32 of them) k rounds of a warp maximum over the
-// keys; ties go to the lower expert index; lane j keeps the j-th pick. The
-// publishing CTA also writes the plain logits.
-__device__ __noinline__ void ds_topk(const DSParams& P, int l, int t, float* pub_logits, unsigned long long* scr,
-                                     unsigned long long* td) {
+// Selection: k rounds of a warp maximum over the keys (ties go to the lower
+// expert index through a second, minimum reduction over the indices that
+// hold the maximum); lane j keeps the j-th pick. The publishing CTA also
+// writes the plain logits.
+__device__ __noinline__ void ds_topk(const DSParams& P, int l, int t, float* pub_logits, unsigned long long* td) {
   // the parameters this uses, in registers: P sits in shared memory, and the
   // ordered loads below would make the compiler read it again each time
   const int E = P.E, T = P.T, k = P.k, L = P.L;
@@ -557,117 +556,57 @@ __device__ __noinline__ void ds_topk(const DSParams& P, int l, int t, float* pub
       if (v * 32 + lane < E) pl[v * 32 + lane] = lv[v];
   }
   if (td && lane == 0) td[29] = global_timer_ns();
-  // Selection order: larger key first, ties to the lower expert index; as one
-  // 64-bit value per expert, key << 32 | ~e (every value distinct).
-  auto pk_of = [&kv, lane](int v) {
-    return (static_cast<unsigned long long>(kv[v]) << 32) | static_cast<uint32_t>(~(v * 32 + lane));
-  };
-  uint32_t mine_key = 0u;
-  int mine_e = 0;
-  // l0: the largest logit (the first pick's); with it the full-softmax
-  // denominator, so that lv is no longer needed during the selection
-  uint32_t kmax = 0u;
-#pragma unroll
-  for (int v = 0; v < KPL; ++v) kmax = max(kmax, kv[v]);
-  const float l0 = ds_key_value(__reduce_max_sync(0xffffffffu, kmax));
-  float full_sum = 0.f;
-  if (!P.renorm) {
-    float ev[KPL];
-#pragma unroll
-    for (int v = 0; v < KPL; ++v) ev[v] = expf(lv[v] - l0);
-#pragma unroll
-    for (int v = 0; v < KPL; ++v)
-      if (v * 32 + lane < E) full_sum += ev[v];  // in order of e within the lane; NaN logits make the sum NaN
-  }
-  // The k-th largest of the 32 lane maxima bounds the k-th pick from below
-  // (k lanes hold a value at least as large), so the picks are among the
-  // values at or above it: usually few. Those (at most 32) are ranked
-  // directly in the scratch; more of them (ties over a whole row, say) take k
-  // rounds of warp maxima.
-  unsigned long long lb;
-  {
+  // lane best: its largest key, ties to its lowest register index (so the
+  // lowest expert index), packed as key << 32 | (KPL - 1 - index)
+  auto lane_best = [&kv]() {
     unsigned long long b[KPL];
 #pragma unroll
-    for (int i = 0; i < KPL; ++i) b[i] = pk_of(i);
+    for (int i = 0; i < KPL; ++i) b[i] = (static_cast<unsigned long long>(kv[i]) << 32) | (KPL - 1 - i);
 #pragma unroll
     for (int h = KPL / 2; h > 0; h >>= 1)
 #pragma unroll
       for (int i = 0; i < h; ++i) b[i] = b[i] > b[i + h] ? b[i] : b[i + h];
-    lb = b[0];
-  }
-  int rank = 0;
-#pragma unroll 4
-  for (int m = 1; m < 32; ++m) rank += __shfl_xor_sync(0xffffffffu, lb, m) > lb ? 1 : 0;
-  const unsigned tsel = __ballot_sync(0xffffffffu, rank == k - 1);
-  const unsigned long long tau = __shfl_sync(0xffffffffu, lb, __ffs(tsel) - 1);
-  int c = 0;
-#pragma unroll
-  for (int v = 0; v < KPL; ++v) c += pk_of(v) >= tau ? 1 : 0;
-  const int C = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c)));
-  if (C <= 32) {
-    int inc = c;  // inclusive prefix of the counts over the lanes
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, inc, d);
-      if (lane >= d) inc += y;
-    }
-    int off = inc - c;
-#pragma unroll
-    for (int v = 0; v < KPL; ++v) {
-      const unsigned long long q = pk_of(v);
-      if (q >= tau) scr[off++] = q;
-    }
-    __syncwarp();
-    const unsigned long long my = lane < C ? scr[lane] : 0ull;
-    int r = 0;
-#pragma unroll 4
-    for (int j = 0; j < C; ++j) r += scr[j] > my ? 1 : 0;
-    if (lane < C && r < k) scr[32 + r] = my;
-    __syncwarp();
-    if (lane < k) {
-      const unsigned long long q = scr[32 + lane];
-      mine_key = static_cast<uint32_t>(q >> 32);
-      mine_e = static_cast<int>(~static_cast<uint32_t>(q));
-    }
-    __syncwarp();
-  } else {
-    // lane best as key << 32 | (KPL - 1 - register index): the same order
-    auto lane_best = [&kv]() {
-      unsigned long long b[KPL];
-#pragma unroll
-      for (int i = 0; i < KPL; ++i) b[i] = (static_cast<unsigned long long>(kv[i]) << 32) | (KPL - 1 - i);
-#pragma unroll
-      for (int h = KPL / 2; h > 0; h >>= 1)
-#pragma unroll
-        for (int i = 0; i < h; ++i) b[i] = b[i] > b[i + h] ? b[i] : b[i + h];
-      return b[0];
-    };
-    unsigned long long lr = lane_best();
+    return b[0];
+  };
+  unsigned long long lb = lane_best();
+  uint32_t mine_key = 0u;
+  int mine_e = 0;
 #pragma unroll 1
-    for (int j = 0; j < k; ++j) {
-      // the warp maximum, then the lowest expert index holding it; only the
-      // lane that held it looks at its keys again
-      const uint32_t lk = static_cast<uint32_t>(lr >> 32);
-      const uint32_t M = __reduce_max_sync(0xffffffffu, lk);
-      const int li = KPL - 1 - static_cast<int>(lr & 0xffu);
-      const unsigned le = lk == M ? static_cast<unsigned>(lane + 32 * li) : 0x7fffffffu;
-      const int e = static_cast<int>(__reduce_min_sync(0xffffffffu, le));
-      if (lane == (e & 31)) {
+  for (int j = 0; j < k; ++j) {
+    // the warp maximum, then the lowest expert index holding it; only the
+    // lane that held it looks at its keys again
+    const uint32_t lk = static_cast<uint32_t>(lb >> 32);
+    const uint32_t M = __reduce_max_sync(0xffffffffu, lk);
+    const int li = KPL - 1 - static_cast<int>(lb & 0xffu);
+    const unsigned le = lk == M ? static_cast<unsigned>(lane + 32 * li) : 0x7fffffffu;
+    const int e = static_cast<int>(__reduce_min_sync(0xffffffffu, le));
+    if (lane == (e & 31)) {
 #pragma unroll
-        for (int i = 0; i < KPL; ++i) kv[i] = (i == (e >> 5)) ? 0u : kv[i];
-        lr = lane_best();
-      }
-      if (lane == j) {
-        mine_key = M;
-        mine_e = e;
-      }
+      for (int i = 0; i < KPL; ++i) kv[i] = (i == (e >> 5)) ? 0u : kv[i];
+      lb = lane_best();
+    }
+    if (lane == j) {
+      mine_key = M;
+      mine_e = e;
     }
   }
   if (td && lane == 0) td[30] = global_timer_ns();
   const bool sel = lane < k;
   const float lj = sel ? ds_key_value(mine_key) : 0.f;
+  const float l0 = __shfl_sync(0xffffffffu, lj, 0);
   const float ex = sel ? expf(lj - l0) : 0.f;
-  const float denom = warp_sum(P.renorm ? ex : full_sum);
+  float sum = ex;
+  if (!P.renorm) {
+    // full-softmax denominator over the whole row (lv, still in registers)
+    float ev[KPL];
+#pragma unroll
+    for (int v = 0; v < KPL; ++v) ev[v] = expf(lv[v] - l0);
+    sum = 0.f;
+#pragma unroll
+    for (int v = 0; v < KPL; ++v)
+      if (v * 32 + lane < E) sum += ev[v];  // in order of e within the lane; NaN logits make the sum NaN
+  }
+  const float denom = warp_sum(sum);
   const float gate = ex / denom;
   if (sel) {
     R.idx[t * k + lane] = mine_e;
@@ -1486,7 +1425,7 @@ __global__ void __launch_bounds__((ds_consumer_warps(BITS) + 1) * 32, 1) decode_
                                : nullptr;
         if (warp < P.T) {
           if (!ds_aborted_warp(S))
-            ds_topk(Q, l, warp, pub, reinterpret_cast<unsigned long long*>(smem + P.sm_x) + warp * 64,
+            ds_topk(Q, l, warp, pub,
                     (tdet && warp == 0) ? tdet : nullptr);
         } else {
           // the accumulator set of layer l + 2 (every CTA read it as layer
@@ -1987,7 +1926,6 @@ cudaError_t launch_decode_stack(const Ctx& ctx, const moe_layer_cfg& c, const St
   const size_t keys_bytes = static_cast<size_t>(T) * c.k * 4;  // the grouping's sort keys
   size_t x_min = keys_bytes;
   if (x_min < T * hq_row) x_min = T * hq_row;
-  if (x_min < static_cast<size_t>(T) * 64 * 8) x_min = static_cast<size_t>(T) * 64 * 8;  // top-k scratch
   int n_ring = 0;
   size_t fixed = 0, x_bytes = 0;
   for (int depth = kDsGuDepth; depth >= 2 && n_ring < 2; --depth) {
